@@ -1,0 +1,217 @@
+"""CPU oracle for the RWKV-4 WKV operator and the diagonal linear scan.
+
+TEST INFRASTRUCTURE ONLY.  The test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` are the only callers.  The CUDA
+library never imports or links anything here, and nothing here imports the
+CUDA library: the two share no code.  Only the seeded input generators in
+``workloads`` feed both.
+
+Pieces (all float64; each cites the page it follows):
+
+* ``wkv_direct``          -- eq. (14) of "RWKV：基于RNN的LLM" (section 二.1,
+  Time-mixing block) evaluated literally, O(T^2) per channel (C code).
+* ``wkv_direct_points``   -- the same definition at chosen (b, t, c) points,
+  O(t) each, for full-size workloads (C code).
+* ``wkv_direct_np``       -- eq. (14) again, as a masked log-sum-exp over a
+  [T, T] logit matrix in numpy; small inputs only.
+* ``wkv_rnn``             -- the RNN-mode state update (RWKV evolution
+  article, section RWKV-V4), max-stabilised; the full-tensor oracle and the
+  timed CPU baseline (C code, OpenMP over channels).
+* ``wkv_slru_ratio_np``   -- the "RWKV = ratio of two SLRUs" form from the
+  review of "Resurrecting Recurrent Neural Networks for Long Sequences"
+  (section on the RWKV variant), unstabilised; |k| small only.
+* ``scan_rnn``            -- h_t = a_t h_{t-1} + b_t ("Were RNNs All We
+  Needed?" article, scan form) (C code).
+* ``scan_direct_points``  -- the unrolled sum of the same scan at chosen points
+  (LRU review, linear-RNN section) (C code).
+
+Parity status: every function above is pinned by the ``-m "not gpu"`` tests
+(closed forms, invariants, brute force, cross-formulation agreement); none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wkv_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+__all__ = [
+    "build", "max_threads", "wkv_direct", "wkv_direct_points", "wkv_direct_np",
+    "wkv_rnn", "wkv_slru_ratio_np", "scan_rnn", "scan_direct_points",
+]
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                               "-fno-fast-math", "-Wall", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _get():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            i64, p = ctypes.c_int64, ctypes.c_void_p
+            lib.oracle_max_threads.restype = ctypes.c_int
+            for name, args in {
+                "oracle_wkv_direct": [i64, i64, i64, p, p, p, p, p, ctypes.c_int],
+                "oracle_wkv_direct_points": [i64, i64, i64, p, p, p, p, i64, p, p, ctypes.c_int],
+                "oracle_wkv_rnn": [i64, i64, i64, p, p, p, p, p, ctypes.c_int],
+                "oracle_scan_rnn": [i64, i64, i64, p, p, p, p, ctypes.c_int],
+                "oracle_scan_direct_points": [i64, i64, i64, p, p, p, i64, p, p, ctypes.c_int],
+            }.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = None
+            _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_get().oracle_max_threads())
+
+
+def _f64(x):
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(x):
+    return x.ctypes.data_as(ctypes.c_void_p)
+
+
+def _wkv_args(w, u, k, v):
+    k, v = _f64(k), _f64(v)
+    if k.ndim != 3 or k.shape != v.shape:
+        raise ValueError("k and v must be [B, T, C] of one shape")
+    B, T, C = k.shape
+    w, u = _f64(w).reshape(-1), _f64(u).reshape(-1)
+    if w.shape != (C,) or u.shape != (C,):
+        raise ValueError("w and u must be [C]")
+    return B, T, C, w, u, k, v
+
+
+def wkv_direct(w, u, k, v, nthreads: int = 0) -> np.ndarray:
+    """Eq. (14) at every output, O(T^2) per channel."""
+    B, T, C, w, u, k, v = _wkv_args(w, u, k, v)
+    y = np.empty((B, T, C), dtype=np.float64)
+    _get().oracle_wkv_direct(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(y), nthreads)
+    return y
+
+
+def wkv_direct_points(w, u, k, v, points, nthreads: int = 0) -> np.ndarray:
+    """Eq. (14) at the flat output indices ``points`` (b*T*C + t*C + c)."""
+    B, T, C, w, u, k, v = _wkv_args(w, u, k, v)
+    pts = np.ascontiguousarray(points, dtype=np.int64).reshape(-1)
+    if pts.size and (pts.min() < 0 or pts.max() >= B * T * C):
+        raise IndexError("point out of range")
+    out = np.empty(pts.size, dtype=np.float64)
+    _get().oracle_wkv_direct_points(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v),
+                                    pts.size, _ptr(pts), _ptr(out), nthreads)
+    return out
+
+
+def wkv_rnn(w, u, k, v, nthreads: int = 0) -> np.ndarray:
+    """RNN-mode recurrence, max-stabilised, float64; all outputs."""
+    B, T, C, w, u, k, v = _wkv_args(w, u, k, v)
+    y = np.empty((B, T, C), dtype=np.float64)
+    _get().oracle_wkv_rnn(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(y), nthreads)
+    return y
+
+
+def wkv_direct_np(w, u, k, v) -> np.ndarray:
+    """Eq. (14) as a masked softmax over a [T, T] logit matrix (numpy).
+
+    logit[t, i] = -(t-1-i) w + k_i for i < t, u + k_t on the diagonal, and no
+    weight for i > t; the output is the logit-softmax-weighted mean of v_i.
+    """
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64).reshape(-1)
+    u = np.asarray(u, dtype=np.float64).reshape(-1)
+    B, T, C = k.shape
+    t_idx = np.arange(T)[:, None]
+    i_idx = np.arange(T)[None, :]
+    dist = (t_idx - 1 - i_idx).astype(np.float64)            # t-1-i
+    logit = -dist[None, :, :, None] * w[None, None, None, :] + k[:, None, :, :]   # [B,T,T,C]
+    diag = u[None, None, :] + k                              # [B,T,C]
+    eye = (t_idx == i_idx)
+    logit = np.where(eye[None, :, :, None], diag[:, :, None, :], logit)
+    logit = np.where((i_idx > t_idx)[None, :, :, None], -np.inf, logit)
+    m = logit.max(axis=2, keepdims=True)
+    e = np.exp(logit - m)
+    return (e * v[:, None, :, :]).sum(axis=2) / e.sum(axis=2)
+
+
+def wkv_slru_ratio_np(w, u, k, v) -> np.ndarray:
+    """Ratio of two real diagonal linear RNNs (LRU review, RWKV variant):
+
+        Y_t = lam Y_{t-1} + e^{k_t} v_t,    Z_t = lam Z_{t-1} + e^{k_t},
+        y_t = (Y_t + (gam lam - 1) e^{k_t} v_t) / (Z_t + (gam lam - 1) e^{k_t}),
+
+    with lam = e^{-w} and gam = e^{u}; the sigma(r) gate of that page is not
+    part of WKV.  No stabilisation, so only for inputs with small |k|.
+    """
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    lam = np.exp(-np.asarray(w, dtype=np.float64).reshape(-1))
+    gam = np.exp(np.asarray(u, dtype=np.float64).reshape(-1))
+    B, T, C = k.shape
+    Y = np.zeros((B, C))
+    Z = np.zeros((B, C))
+    out = np.empty((B, T, C))
+    for t in range(T):
+        ek = np.exp(k[:, t, :])
+        Y = lam * Y + ek * v[:, t, :]
+        Z = lam * Z + ek
+        out[:, t, :] = (Y + (gam * lam - 1.0) * ek * v[:, t, :]) / (Z + (gam * lam - 1.0) * ek)
+    return out
+
+
+def _scan_args(a, b, h0):
+    a, b = _f64(a), _f64(b)
+    if a.ndim != 3 or a.shape != b.shape:
+        raise ValueError("a and b must be [B, T, D] of one shape")
+    B, T, D = a.shape
+    if h0 is not None:
+        h0 = _f64(h0)
+        if h0.shape != (B, D):
+            raise ValueError("h0 must be [B, D]")
+    return B, T, D, a, b, h0
+
+
+def scan_rnn(a, b, h0=None, nthreads: int = 0) -> np.ndarray:
+    """h_t = a_t h_{t-1} + b_t with h_{-1} = h0 (zeros if None), float64."""
+    B, T, D, a, b, h0 = _scan_args(a, b, h0)
+    h = np.empty((B, T, D), dtype=np.float64)
+    _get().oracle_scan_rnn(B, T, D, _ptr(a), _ptr(b), None if h0 is None else _ptr(h0),
+                           _ptr(h), nthreads)
+    return h
+
+
+def scan_direct_points(a, b, h0, points, nthreads: int = 0) -> np.ndarray:
+    """Unrolled scan sum at the flat output indices ``points``."""
+    B, T, D, a, b, h0 = _scan_args(a, b, h0)
+    pts = np.ascontiguousarray(points, dtype=np.int64).reshape(-1)
+    if pts.size and (pts.min() < 0 or pts.max() >= B * T * D):
+        raise IndexError("point out of range")
+    out = np.empty(pts.size, dtype=np.float64)
+    _get().oracle_scan_direct_points(B, T, D, _ptr(a), _ptr(b),
+                                     None if h0 is None else _ptr(h0),
+                                     pts.size, _ptr(pts), _ptr(out), nthreads)
+    return out

@@ -1,0 +1,303 @@
+"""Pins for WKV and diagonal-scan implementations.
+
+Each check takes an implementation ``fn`` (numpy arrays in, float64 array out)
+and returns a list of failure messages.  The values they compare against come
+from outside the implementation under test:
+
+* hand-worked examples in exact rational arithmetic (``tests/golden``);
+* closed forms of special cases (running mean, geometric series, two-token
+  softmax limit, cumulative sum / product);
+* invariants the definition fixes (convex combination, shift invariance in k,
+  affine equivariance in v, causality).
+
+Used by the oracle's CPU tests (including the planted-mistake tests, which
+check that every planted mistake trips at least one pin) and by the GPU
+parity tests.
+"""
+from __future__ import annotations
+
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def read_golden(name):
+    recs = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            recs[key] = [Fraction(x) for x in vals]
+    return recs
+
+
+def _close(got, want, tol):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    if got.shape != want.shape:
+        return f"shape {got.shape} != {want.shape}"
+    err = np.max(np.abs(got - want)) if got.size else 0.0
+    if not np.isfinite(err) or err > tol:
+        return f"max err {err:.3e} > {tol:.1e}"
+    return None
+
+
+# ---------------------------------------------------------------------------
+# WKV pins
+# ---------------------------------------------------------------------------
+def wkv_worked_example(fn, tol=1e-12):
+    g = read_golden("wkv_worked_example.txt")
+    w = np.array([-np.log(float(g["w_exp_neg"][0]))])
+    u = np.array([np.log(float(g["u_exp"][0]))])
+    k = np.log(np.array([float(x) for x in g["k_exp"]]))[None, :, None]
+    v = np.array([float(x) for x in g["v"]])[None, :, None]
+    want = np.array([float(x) for x in g["y"]])[None, :, None]
+    msg = _close(fn(w, u, k, v), want, tol)
+    return [f"worked example: {msg}"] if msg else []
+
+
+def wkv_exact_rational(fn, seed=3, T=7, C=3, tol=1e-12):
+    """Brute force in exact rationals: pick e^{k}, e^{-w}, e^{u} rational."""
+    rng = np.random.default_rng(seed)
+    r = [[Fraction(int(rng.integers(1, 9)), int(rng.integers(1, 9))) for _ in range(C)] for _ in range(T)]
+    lam = [Fraction(int(rng.integers(1, 8)), 8) for _ in range(C)]
+    gam = [Fraction(int(rng.integers(1, 7)), int(rng.integers(1, 7))) for _ in range(C)]
+    vv = [[Fraction(int(rng.integers(-9, 10))) for _ in range(C)] for _ in range(T)]
+    want = np.zeros((1, T, C))
+    for c in range(C):
+        for t in range(T):
+            num = gam[c] * r[t][c] * vv[t][c]
+            den = gam[c] * r[t][c]
+            for i in range(t):
+                wt = lam[c] ** (t - 1 - i) * r[i][c]
+                num += wt * vv[i][c]
+                den += wt
+            want[0, t, c] = float(num / den)
+    k = np.log(np.array([[float(x) for x in row] for row in r]))[None]
+    w = -np.log(np.array([float(x) for x in lam]))
+    u = np.log(np.array([float(x) for x in gam]))
+    v = np.array([[float(x) for x in row] for row in vv])[None]
+    msg = _close(fn(w, u, k, v), want, tol)
+    return [f"exact rational: {msg}"] if msg else []
+
+
+def wkv_single_step(fn, tol=0.0):
+    rng = np.random.default_rng(1)
+    k = rng.normal(0, 2, (3, 1, 5)); v = rng.normal(0, 1, (3, 1, 5))
+    w = np.exp(rng.normal(0, 1, 5)); u = rng.normal(0, 1, 5)
+    msg = _close(fn(w, u, k, v), v, tol)
+    return [f"T=1 gives v: {msg}"] if msg else []
+
+
+def wkv_running_mean(fn, tol=1e-12):
+    """w = 0, u = 0, constant k: every past token and the current one weigh
+    the same, so y_t is the mean of v_0..v_t."""
+    rng = np.random.default_rng(2)
+    T, C = 40, 4
+    v = rng.normal(0, 1, (2, T, C))
+    k = np.full((2, T, C), 0.7)
+    want = np.cumsum(v, axis=1) / np.arange(1, T + 1)[None, :, None]
+    msg = _close(fn(np.zeros(C), np.zeros(C), k, v), want, tol)
+    return [f"running mean: {msg}"] if msg else []
+
+
+def wkv_past_mean(fn, tol=1e-9):
+    """w = 0, constant k, bonus u -> -inf (u = -40): the current token's
+    weight vanishes, y_t (t >= 1) is the mean of v_0..v_{t-1}."""
+    rng = np.random.default_rng(4)
+    T, C = 30, 3
+    v = rng.normal(0, 1, (1, T, C))
+    k = np.zeros((1, T, C))
+    got = np.asarray(fn(np.zeros(C), np.full(C, -40.0), k, v))
+    want = np.cumsum(v, axis=1)[:, :-1, :] / np.arange(1, T)[None, :, None]
+    msg = _close(got[:, 1:, :], want, tol)
+    return [f"past-only mean: {msg}"] if msg else []
+
+
+def wkv_geometric(fn, tol=1e-12):
+    """k = 0, u = 0, decay lam = e^{-w}, v one-hot at step j: the weight of
+    token j at step t > j is lam^{t-1-j}, the denominator is the geometric
+    sum (1 - lam^t) / (1 - lam) + 1."""
+    T, j = 24, 5
+    lam = np.array([0.5, 0.9, 0.25])
+    w = -np.log(lam)
+    C = lam.size
+    v = np.zeros((1, T, C)); v[0, j, :] = 1.0
+    k = np.zeros((1, T, C))
+    want = np.zeros((1, T, C))
+    for t in range(T):
+        den = (1 - lam ** t) / (1 - lam) + 1.0
+        if t == j:
+            want[0, t] = 1.0 / den
+        elif t > j:
+            want[0, t] = lam ** (t - 1 - j) / den
+    msg = _close(fn(w, np.zeros(C), k, v), want, tol)
+    return [f"geometric one-hot: {msg}"] if msg else []
+
+
+def wkv_fast_decay(fn, tol=1e-12):
+    """w -> inf (w = 60): only the previous token (weight e^{k_{t-1}}) and
+    the current one (weight e^{u + k_t}) survive."""
+    rng = np.random.default_rng(5)
+    T, C = 20, 4
+    k = rng.normal(0, 1, (1, T, C)); v = rng.normal(0, 1, (1, T, C))
+    u = rng.normal(0, 0.5, C)
+    want = v.copy()
+    ep = np.exp(k[:, :-1]); ec = np.exp(u + k[:, 1:])
+    want[:, 1:] = (ep * v[:, :-1] + ec * v[:, 1:]) / (ep + ec)
+    msg = _close(fn(np.full(C, 60.0), u, k, v), want, tol)
+    return [f"fast decay two-token limit: {msg}"] if msg else []
+
+
+def wkv_large_bonus(fn, tol=1e-12):
+    """u -> inf (u = 60) with |k| small: y_t = v_t."""
+    rng = np.random.default_rng(6)
+    k = rng.normal(0, 1, (1, 16, 3)); v = rng.normal(0, 1, (1, 16, 3))
+    msg = _close(fn(np.full(3, 0.1), np.full(3, 60.0), k, v), v, tol)
+    return [f"large bonus: {msg}"] if msg else []
+
+
+def _rand_wkv(seed, B=2, T=48, C=5, ksig=2.0):
+    rng = np.random.default_rng(seed)
+    return (np.exp(rng.normal(-0.5, 1.0, C)), rng.normal(0, 1, C),
+            rng.normal(0, ksig, (B, T, C)), rng.normal(0, 1, (B, T, C)))
+
+
+def wkv_invariants(fn, rel=1e-11):
+    out = []
+    w, u, k, v = _rand_wkv(7)
+    y = np.asarray(fn(w, u, k, v))
+    # convex combination of v_0..v_t
+    lo = np.minimum.accumulate(v, axis=1); hi = np.maximum.accumulate(v, axis=1)
+    if np.any(y < lo - rel) or np.any(y > hi + rel):
+        out.append("convex bound violated")
+    # shift invariance in k (common factor of numerator and denominator)
+    msg = _close(fn(w, u, k + 3.25, v), y, rel * 10)
+    if msg: out.append(f"k-shift invariance: {msg}")
+    # affine equivariance in v
+    msg = _close(fn(w, u, k, 2.5 * v - 1.5), 2.5 * y - 1.5, rel * 10)
+    if msg: out.append(f"affine equivariance: {msg}")
+    # constant v gives v
+    msg = _close(fn(w, u, k, np.full_like(v, 0.375)), np.full_like(v, 0.375), rel)
+    if msg: out.append(f"constant v: {msg}")
+    # causality: editing step j leaves every earlier output unchanged
+    j = 30
+    v2 = v.copy(); k2 = k.copy(); v2[:, j:] += 5.0; k2[:, j:] -= 2.0
+    y2 = np.asarray(fn(w, u, k2, v2))
+    if not np.array_equal(y2[:, :j], y[:, :j]):
+        out.append("causality: future tokens changed past outputs")
+    # channels and batch rows are independent
+    yb = np.asarray(fn(w[1:3], u[1:3], k[1:, :, 1:3], v[1:, :, 1:3]))
+    msg = _close(yb, y[1:, :, 1:3], 0.0)
+    if msg: out.append(f"channel/batch independence: {msg}")
+    return out
+
+
+WKV_PINS = [wkv_worked_example, wkv_exact_rational, wkv_single_step, wkv_running_mean,
+            wkv_past_mean, wkv_geometric, wkv_fast_decay, wkv_large_bonus, wkv_invariants]
+
+
+def run_wkv_pins(fn):
+    fails = []
+    for pin in WKV_PINS:
+        try:
+            fails += pin(fn)
+        except Exception as e:  # a mutant may crash a pin; that counts as caught
+            fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
+    return fails
+
+
+# ---------------------------------------------------------------------------
+# diagonal scan pins
+# ---------------------------------------------------------------------------
+def scan_worked_example(fn, tol=1e-12):
+    g = read_golden("scan_worked_example.txt")
+    a = np.array([float(x) for x in g["a"]])[None, :, None]
+    b = np.array([float(x) for x in g["b"]])[None, :, None]
+    h0 = np.array([[float(g["h0"][0])]])
+    want = np.array([float(x) for x in g["h"]])[None, :, None]
+    msg = _close(fn(a, b, h0), want, tol)
+    return [f"worked example: {msg}"] if msg else []
+
+
+def scan_closed_forms(fn, tol=1e-10):
+    out = []
+    rng = np.random.default_rng(11)
+    B, T, D = 2, 50, 3
+    b = rng.normal(0, 1, (B, T, D))
+    h0 = rng.normal(0, 1, (B, D))
+    # a = 1: cumulative sum on top of h0
+    msg = _close(fn(np.ones((B, T, D)), b, h0), h0[:, None, :] + np.cumsum(b, axis=1), tol)
+    if msg: out.append(f"a=1 cumsum: {msg}")
+    # a = 0: h = b
+    msg = _close(fn(np.zeros((B, T, D)), b, h0), b, 0.0)
+    if msg: out.append(f"a=0: {msg}")
+    # b = 0: h_t = h0 * prod_{j<=t} a_j
+    a = rng.uniform(0.5, 1.2, (B, T, D))
+    msg = _close(fn(a, np.zeros((B, T, D)), h0), h0[:, None, :] * np.cumprod(a, axis=1), tol)
+    if msg: out.append(f"b=0 cumprod: {msg}")
+    # constant a = lam, constant b = beta, h0 = 0: beta (1 - lam^{t+1}) / (1 - lam)
+    lam, beta = 0.8, 1.25
+    t = np.arange(T)
+    want = np.broadcast_to((beta * (1 - lam ** (t + 1)) / (1 - lam))[None, :, None], (B, T, D))
+    msg = _close(fn(np.full((B, T, D), lam), np.full((B, T, D), beta), None), want, tol)
+    if msg: out.append(f"geometric series: {msg}")
+    # no h0 equals h0 = 0
+    msg = _close(fn(a, b, None), fn(a, b, np.zeros((B, D))), 0.0)
+    if msg: out.append(f"h0=None vs zeros: {msg}")
+    return out
+
+
+def scan_chaining(fn, tol=1e-12):
+    rng = np.random.default_rng(12)
+    B, T, D, T1 = 2, 40, 3, 17
+    a = rng.uniform(0.3, 1.0, (B, T, D)); b = rng.normal(0, 1, (B, T, D))
+    h0 = rng.normal(0, 1, (B, D))
+    full = np.asarray(fn(a, b, h0))
+    first = np.asarray(fn(a[:, :T1], b[:, :T1], h0))
+    second = np.asarray(fn(a[:, T1:], b[:, T1:], first[:, -1, :]))
+    msg = _close(np.concatenate([first, second], axis=1), full, tol)
+    return [f"chaining: {msg}"] if msg else []
+
+
+def scan_mingru_convex(fn, tol=1e-12):
+    """minGRU form a = 1 - z, b = z h~ with z in (0, 1): each h_t is a convex
+    combination of h0 and h~_0..h~_t."""
+    rng = np.random.default_rng(13)
+    B, T, D = 2, 64, 4
+    z = 1 / (1 + np.exp(-rng.normal(0, 1, (B, T, D))))
+    ht = rng.normal(0, 1, (B, T, D))
+    h0 = rng.normal(0, 1, (B, D))
+    h = np.asarray(fn(1 - z, z * ht, h0))
+    lo = np.minimum(np.minimum.accumulate(ht, axis=1), h0[:, None, :])
+    hi = np.maximum(np.maximum.accumulate(ht, axis=1), h0[:, None, :])
+    if np.any(h < lo - tol) or np.any(h > hi + tol):
+        return ["minGRU convex bound violated"]
+    return []
+
+
+def scan_linearity(fn, tol=1e-11):
+    rng = np.random.default_rng(14)
+    B, T, D = 1, 30, 3
+    a = rng.uniform(0.2, 1.1, (B, T, D))
+    b1, b2 = rng.normal(0, 1, (2, B, T, D))
+    msg = _close(fn(a, 2 * b1 - 3 * b2, None), 2 * np.asarray(fn(a, b1, None)) - 3 * np.asarray(fn(a, b2, None)), tol)
+    return [f"linearity in b: {msg}"] if msg else []
+
+
+SCAN_PINS = [scan_worked_example, scan_closed_forms, scan_chaining, scan_mingru_convex, scan_linearity]
+
+
+def run_scan_pins(fn):
+    fails = []
+    for pin in SCAN_PINS:
+        try:
+            fails += pin(fn)
+        except Exception as e:
+            fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
+    return fails

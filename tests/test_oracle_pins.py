@@ -1,0 +1,253 @@
+"""The CPU oracle against what the pages and the mathematics fix.
+
+Every oracle function must pass every pin in ``pins.py`` (hand-worked
+examples in exact rationals, closed forms, invariants), the independent
+formulations must agree with each other, and a set of planted mistakes --
+the plausible errors an implementation of eq. (14) could make -- must each
+trip at least one pin.
+"""
+import os
+import shutil
+import subprocess
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+import pins
+
+
+# --- wrappers with the common pin signature -------------------------------
+def c_direct(w, u, k, v):
+    return oracle.wkv_direct(w, u, k, v)
+
+
+def c_rnn(w, u, k, v):
+    return oracle.wkv_rnn(w, u, k, v)
+
+
+def c_points(w, u, k, v):
+    k = np.asarray(k)
+    return oracle.wkv_direct_points(w, u, k, v, np.arange(k.size)).reshape(k.shape)
+
+
+def np_direct(w, u, k, v):
+    return oracle.wkv_direct_np(w, u, k, v)
+
+
+def slru_ratio(w, u, k, v):
+    return oracle.wkv_slru_ratio_np(w, u, k, v)
+
+
+@pytest.mark.parametrize("fn", [c_direct, c_rnn, c_points, np_direct],
+                         ids=["c_direct", "c_rnn", "c_points", "np_direct"])
+def test_wkv_oracle_passes_pins(fn):
+    assert pins.run_wkv_pins(fn) == []
+
+
+def test_slru_ratio_form_passes_pins_in_range():
+    # The unstabilised two-SLRU form overflows for |u|, w or |k| of tens;
+    # check it on the pins whose inputs stay in range.
+    # (its T = 1 output is (Y + (gam lam - 1) e^k v) / (Z + ...), exact only up
+    # to rounding, hence the small tolerance there)
+    for pin in (pins.wkv_worked_example, pins.wkv_exact_rational,
+                lambda fn: pins.wkv_single_step(fn, tol=1e-12),
+                pins.wkv_running_mean, pins.wkv_geometric, pins.wkv_invariants):
+        assert pin(slru_ratio) == [], getattr(pin, "__name__", "single_step")
+
+
+@pytest.mark.parametrize("seed,B,T,C,ksig", [(0, 2, 64, 7, 1.0), (1, 1, 200, 3, 2.0),
+                                             (2, 3, 33, 5, 0.3)])
+def test_wkv_formulations_agree(seed, B, T, C, ksig):
+    """Definition (C and numpy), RNN mode and the two-SLRU ratio from a
+    different page all give the same numbers."""
+    rng = np.random.default_rng(seed)
+    k = rng.normal(0, ksig, (B, T, C)); v = rng.normal(0, 1, (B, T, C))
+    w = np.exp(rng.uniform(-3, 1, C)); u = rng.normal(0, 0.5, C)
+    ref = oracle.wkv_direct_np(w, u, k, v)
+    for got in (oracle.wkv_direct(w, u, k, v), oracle.wkv_rnn(w, u, k, v),
+                oracle.wkv_slru_ratio_np(w, u, k, v)):
+        assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_wkv_stabilised_under_large_keys():
+    """k ~ N(0, 30): e^{k} alone overflows float64 sums of the raw form; the
+    direct and RNN forms keep every exponent <= 0 and agree."""
+    rng = np.random.default_rng(9)
+    B, T, C = 1, 300, 4
+    k = rng.normal(0, 30, (B, T, C)); v = rng.normal(0, 1, (B, T, C))
+    k[0, 100, :] = 800.0   # e^{800} is inf in float64
+    w = np.array([0.0, 1e-3, 1.0, 50.0]); u = np.array([0.0, -3.0, 2.0, 700.0])
+    d = oracle.wkv_direct(w, u, k, v)
+    r = oracle.wkv_rnn(w, u, k, v)
+    assert np.all(np.isfinite(d)) and np.all(np.isfinite(r))
+    assert np.max(np.abs(d - r)) < 1e-12
+
+
+def test_wkv_points_match_full():
+    x = workloads.make_wkv("wkv_tiny")
+    full = oracle.wkv_direct(x.w, x.u, x.k, x.v)
+    pts = np.random.default_rng(0).choice(x.k.size, 300, replace=False)
+    got = oracle.wkv_direct_points(x.w, x.u, x.k, x.v, pts)
+    assert np.array_equal(got, full.reshape(-1)[pts])
+
+
+def test_wkv_tiny_workload_direct_vs_rnn():
+    x = workloads.make_wkv("wkv_tiny")
+    d = oracle.wkv_direct_np(x.w, x.u, x.k, x.v)
+    r = oracle.wkv_rnn(x.w, x.u, x.k, x.v)
+    assert np.max(np.abs(d - r)) < 1e-12
+    assert np.array_equal(r[:, 0, :], x.v[:, 0, :].astype(np.float64))
+
+
+def test_eq10_offset_is_eq14_with_shifted_bonus():
+    """Eq. (10) of the RWKV page decays by (t-i) w while eq. (14) uses
+    (t-1-i) w; the two differ only by a constant factor e^{-w} on every past
+    token, i.e. eq. (10) with bonus u equals eq. (14) with bonus u + w."""
+    rng = np.random.default_rng(10)
+    B, T, C = 1, 40, 3
+    k = rng.normal(0, 1, (B, T, C)); v = rng.normal(0, 1, (B, T, C))
+    w = np.exp(rng.normal(0, 1, C)); u = rng.normal(0, 1, C)
+    eq10 = np.empty((B, T, C))
+    for t in range(T):
+        i = np.arange(t)
+        lg = np.concatenate([-(t - i)[:, None] * w[None] + k[0, :t], (u + k[0, t])[None]], 0)
+        e = np.exp(lg - lg.max(0))
+        eq10[0, t] = (e * v[0, :t + 1]).sum(0) / e.sum(0)
+    assert np.max(np.abs(eq10 - oracle.wkv_direct(w, u + w, k, v))) < 1e-12
+
+
+# --- planted mistakes in a numpy copy of the definition -------------------
+def _direct_variant(kind):
+    def fn(w, u, k, v):
+        k = np.asarray(k, float); v = np.asarray(v, float)
+        w = np.asarray(w, float).reshape(-1); u = np.asarray(u, float).reshape(-1)
+        if kind == "swap_kv":
+            k, v = v, k
+        B, T, C = k.shape
+        y = np.empty((B, T, C))
+        for t in range(T):
+            i = np.arange(t + 1 if kind == "future_token" and t + 1 < T else t)
+            off = {"eq10_offset": t - i, "sign_w": -(t - 1 - i)}.get(kind, t - 1 - i)
+            past = -off[:, None] * w[None] + k[:, i]
+            cur = (k[:, t] if kind == "no_bonus" else u + k[:, t])[:, None]
+            if kind == "future_token" and t + 1 < T:
+                past = past.copy(); past[:, -1] = k[:, t + 1]   # leaks v_{t+1}
+            lg = np.concatenate([past, cur], 1)
+            vals = np.concatenate([v[:, i], v[:, t][:, None]], 1)
+            e = np.exp(lg - lg.max(1, keepdims=True))
+            num = (e * vals).sum(1)
+            den = e[:, :-1].sum(1) if kind == "drop_current_den" else e.sum(1)
+            if kind == "drop_current_den":
+                den = den + (t == 0)
+            y[:, t] = num / den
+        return y
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["eq10_offset", "sign_w", "no_bonus", "swap_kv",
+                                  "future_token", "drop_current_den"])
+def test_planted_mistake_in_definition_is_caught(kind):
+    assert _direct_variant("none")(np.ones(2), np.zeros(2), np.zeros((1, 3, 2)),
+                                   np.ones((1, 3, 2))).shape == (1, 3, 2)
+    assert pins.run_wkv_pins(_direct_variant("none")) == []
+    assert pins.run_wkv_pins(_direct_variant(kind)) != []
+
+
+# --- planted mistakes in a copy of the C oracle ---------------------------
+C_MUTANTS = {
+    "decay_sign": ("double pd = p - wc;", "double pd = p + wc;"),
+    "bonus_dropped": ("double x = uc + kt;", "double x = kt;"),
+    # past decayed once more at output time: the (t-i) offset of eq. (10)
+    "extra_decay_at_output": ("double ep = exp(p - q), ex = exp(x - q);",
+                              "double ep = exp(p - wc - q), ex = exp(x - q);"),
+    "state_new_weight": ("double f_old = exp(pd - q2), f_new = exp(kt - q2);",
+                         "double f_old = exp(pd - q2), f_new = exp(kt - q2 + uc);"),
+    "den_uses_v": ("d = f_old * d + f_new;", "d = f_old * d + f_new * vt;"),
+}
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+@pytest.mark.parametrize("name", sorted(C_MUTANTS))
+def test_planted_mistake_in_c_oracle_is_caught(name, tmp_path):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "wkv_oracle.c")).read()
+    old, new = C_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation anchor for {name} not found"
+    mpath = tmp_path / "mut.c"
+    mpath.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-o", str(so),
+                           str(mpath), "-lm"])
+    lib = ctypes.CDLL(str(so))
+    i64, p = ctypes.c_int64, ctypes.c_void_p
+    lib.oracle_wkv_rnn.argtypes = [i64, i64, i64, p, p, p, p, p, ctypes.c_int]
+    lib.oracle_wkv_rnn.restype = None
+
+    def mut(w, u, k, v):
+        k = np.ascontiguousarray(k, float); v = np.ascontiguousarray(v, float)
+        w = np.ascontiguousarray(w, float).reshape(-1); u = np.ascontiguousarray(u, float).reshape(-1)
+        y = np.empty(k.shape)
+        B, T, C = k.shape
+        lib.oracle_wkv_rnn(B, T, C, *(x.ctypes.data_as(p) for x in (w, u, k, v, y)), 1)
+        return y
+
+    assert pins.run_wkv_pins(mut) != []
+
+
+# --- diagonal scan ---------------------------------------------------------
+def scan_rnn(a, b, h0):
+    return oracle.scan_rnn(a, b, h0)
+
+
+def scan_points(a, b, h0):
+    a = np.asarray(a)
+    return oracle.scan_direct_points(a, b, h0, np.arange(a.size)).reshape(a.shape)
+
+
+@pytest.mark.parametrize("fn", [scan_rnn, scan_points], ids=["rnn", "points"])
+def test_scan_oracle_passes_pins(fn):
+    assert pins.run_scan_pins(fn) == []
+
+
+@pytest.mark.parametrize("name,mut", [
+    ("drop_h0", lambda a, b, h0: oracle.scan_rnn(a, b, None)),
+    ("shift_a", lambda a, b, h0: oracle.scan_rnn(np.roll(a, 1, axis=1), b, h0)),
+    ("swap_ab", lambda a, b, h0: oracle.scan_rnn(b, a, h0)),
+    ("exclusive", lambda a, b, h0: np.concatenate(
+        [np.broadcast_to(np.zeros(1) if h0 is None else np.asarray(h0)[:, None, :],
+                         (np.asarray(a).shape[0], 1, np.asarray(a).shape[2])),
+         oracle.scan_rnn(a, b, h0)[:, :-1]], axis=1)),
+])
+def test_planted_mistake_in_scan_is_caught(name, mut):
+    assert pins.run_scan_pins(mut) != []
+
+
+def test_scan_rnn_vs_points_on_mingru_workload():
+    x = workloads.make_scan("scan_mingru", B=2, T=300, D=8, with_h0=True)
+    full = oracle.scan_rnn(x.a, x.b, x.h0)
+    pts = np.random.default_rng(1).choice(x.a.size, 400, replace=False)
+    got = oracle.scan_direct_points(x.a, x.b, x.h0, pts)
+    assert np.max(np.abs(got - full.reshape(-1)[pts])) < 1e-12
+
+
+def test_scan_variance_formula():
+    """Variance of x_t = lam x_{t-1} + u_t for iid zero-mean u (LRU review,
+    initialisation section): E x_t^2 = (1 - lam^{2(t+1)}) / (1 - lam^2) E u^2.
+    Checked statistically over 40000 independent channels."""
+    rng = np.random.default_rng(21)
+    B, T, D, lam = 10, 60, 4000, 0.95
+    b = rng.normal(0, 1, (B, T, D))
+    h = oracle.scan_rnn(np.full((B, T, D), lam), b, None)
+    emp = (h ** 2).mean(axis=(0, 2))
+    t = np.arange(T)
+    want = (1 - lam ** (2 * (t + 1))) / (1 - lam ** 2)
+    assert np.max(np.abs(emp / want - 1)) < 0.05
+
+
+def test_worked_examples_read():
+    g = pins.read_golden("wkv_worked_example.txt")
+    assert len(g["y"]) == len(g["v"]) == 4
+    g = pins.read_golden("scan_worked_example.txt")
+    assert len(g["h"]) == len(g["a"]) == 4

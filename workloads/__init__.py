@@ -1,0 +1,183 @@
+"""Seeded synthetic inputs for the WKV operator and the diagonal linear scan.
+
+This module is shared by the CPU oracle's tests, the CUDA parity tests and
+``bench.py``.  It holds none of the operator's arithmetic: it only draws
+random numbers, applies the input recipes below (which describe what the
+inputs look like, not what the operator computes) and rounds them to the
+storage type the GPU path consumes.
+
+Recipe (every workload): ``numpy.random.default_rng(seed)``; values drawn in
+float64, in the order listed per workload; then rounded to float32 (round to
+nearest even); for bf16 workloads the float32 values of k and v are rounded
+once more to bfloat16 (round to nearest even) and the oracle is fed the
+rounded values widened back to float.  ``N(mu, sigma)`` takes the standard
+deviation as its second argument, ``U(lo, hi)`` is uniform.
+
+Named workloads (shapes from RWKV-4 models and the minGRU scan form):
+
+* ``wkv_tiny``   WKV fp32, B=1 T=64 C=32; k, v ~ N(0,1); w = exp(N(-0.5,0.5));
+  u ~ N(0,0.5)
+* ``wkv_169m``   WKV fp32, B=8 T=1024 C=768 (RWKV-4-169M width); k, v ~ N(0,1);
+  w = exp(U(-3,1)); u ~ N(0,0.5)
+* ``wkv_3b_bf16`` WKV bf16 k/v/y with fp32 state, B=8 T=4096 C=2560 (RWKV-4-3B
+  width); same distributions as ``wkv_169m``
+* ``wkv_long``   WKV fp32, B=1 T=131072 C=1024; k ~ N(0,3), v ~ N(0,1);
+  w = exp(U(-6,0)); u ~ N(0,1)
+* ``scan_mingru`` diagonal scan fp32, B=64 T=4096 D=256 in minGRU form:
+  z = sigmoid(N(0,1)), h~ ~ N(0,1), a = 1 - z, b = z * h~, h0 = 0
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+__all__ = [
+    "WkvSpec", "ScanSpec", "WORKLOADS", "WkvInputs", "ScanInputs",
+    "make_wkv", "make_scan", "bf16_round", "bf16_bits", "bf16_bits_to_f32",
+    "get_workload",
+]
+
+
+@dataclasses.dataclass(frozen=True)
+class WkvSpec:
+    """Shape and input distributions of one WKV workload."""
+    name: str
+    B: int
+    T: int
+    C: int
+    dtype: str = "f32"            # "f32" or "bf16" storage of k, v, y
+    k_sigma: float = 1.0          # k ~ N(0, k_sigma)
+    v_sigma: float = 1.0          # v ~ N(0, v_sigma)
+    w_log: tuple = ("normal", -0.5, 0.5)   # log w ~ N(m, s) or U(lo, hi)
+    u_sigma: float = 0.5          # u ~ N(0, u_sigma)
+    seed: int = 0
+
+    @property
+    def elements(self) -> int:
+        return self.B * self.T * self.C
+
+
+@dataclasses.dataclass(frozen=True)
+class ScanSpec:
+    """Shape of one minGRU-form diagonal scan workload."""
+    name: str
+    B: int
+    T: int
+    D: int
+    seed: int = 0
+    with_h0: bool = False         # minGRU recipe uses h0 = 0 (passed as "none")
+
+    @property
+    def elements(self) -> int:
+        return self.B * self.T * self.D
+
+
+WORKLOADS = {
+    "wkv_tiny": WkvSpec("wkv_tiny", 1, 64, 32, "f32", 1.0, 1.0, ("normal", -0.5, 0.5), 0.5),
+    "wkv_169m": WkvSpec("wkv_169m", 8, 1024, 768, "f32", 1.0, 1.0, ("uniform", -3.0, 1.0), 0.5),
+    "wkv_3b_bf16": WkvSpec("wkv_3b_bf16", 8, 4096, 2560, "bf16", 1.0, 1.0, ("uniform", -3.0, 1.0), 0.5),
+    "wkv_long": WkvSpec("wkv_long", 1, 131072, 1024, "f32", 3.0, 1.0, ("uniform", -6.0, 0.0), 1.0),
+    "scan_mingru": ScanSpec("scan_mingru", 64, 4096, 256),
+}
+
+
+def get_workload(name: str):
+    return WORKLOADS[name]
+
+
+# ---------------------------------------------------------------------------
+# bfloat16 storage helpers (numpy has no bfloat16 type)
+# ---------------------------------------------------------------------------
+def bf16_bits(x32: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns (uint16), round to nearest even.
+
+    Inputs are finite, so the NaN special case is not needed."""
+    x32 = np.ascontiguousarray(x32, dtype=np.float32)
+    bits = x32.view(np.uint32).astype(np.uint64)
+    bias = ((bits >> 16) & 1) + 0x7FFF
+    return ((bits + bias) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b16: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns (uint16) -> float32 (exact widening)."""
+    return (np.ascontiguousarray(b16, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def bf16_round(x32: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16, returned as float32."""
+    return bf16_bits_to_f32(bf16_bits(x32))
+
+
+# ---------------------------------------------------------------------------
+# generators
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class WkvInputs:
+    """float32 host arrays; for bf16 workloads k and v hold the rounded values
+    and ``k_bits``/``v_bits`` the uint16 storage the GPU path reads."""
+    spec: WkvSpec
+    w: np.ndarray   # [C] float32, w >= 0
+    u: np.ndarray   # [C] float32
+    k: np.ndarray   # [B, T, C] float32
+    v: np.ndarray   # [B, T, C] float32
+    k_bits: Optional[np.ndarray] = None
+    v_bits: Optional[np.ndarray] = None
+
+
+@dataclasses.dataclass
+class ScanInputs:
+    spec: ScanSpec
+    a: np.ndarray   # [B, T, D] float32
+    b: np.ndarray   # [B, T, D] float32
+    h0: Optional[np.ndarray]   # [B, D] float32 or None (zeros)
+
+
+def _draw_log_w(rng, spec_w, C):
+    kind, p0, p1 = spec_w
+    if kind == "normal":
+        return rng.normal(p0, p1, size=C)
+    if kind == "uniform":
+        return rng.uniform(p0, p1, size=C)
+    raise ValueError(kind)
+
+
+def make_wkv(spec, *, B=None, T=None, C=None, seed=None) -> WkvInputs:
+    """Draw one WKV workload. ``spec`` is a WkvSpec or a workload name; the
+    keyword overrides give the same distributions at another shape."""
+    if isinstance(spec, str):
+        spec = WORKLOADS[spec]
+    if B is not None or T is not None or C is not None or seed is not None:
+        spec = dataclasses.replace(
+            spec, B=spec.B if B is None else B, T=spec.T if T is None else T,
+            C=spec.C if C is None else C, seed=spec.seed if seed is None else seed,
+            name=f"{spec.name}@{B or spec.B}x{T or spec.T}x{C or spec.C}")
+    rng = np.random.default_rng(spec.seed)
+    shape = (spec.B, spec.T, spec.C)
+    k = rng.normal(0.0, spec.k_sigma, size=shape).astype(np.float32)
+    v = rng.normal(0.0, spec.v_sigma, size=shape).astype(np.float32)
+    w = np.exp(_draw_log_w(rng, spec.w_log, spec.C)).astype(np.float32)
+    u = rng.normal(0.0, spec.u_sigma, size=spec.C).astype(np.float32)
+    if spec.dtype == "bf16":
+        kb, vb = bf16_bits(k), bf16_bits(v)
+        return WkvInputs(spec, w, u, bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), kb, vb)
+    return WkvInputs(spec, w, u, k, v)
+
+
+def make_scan(spec, *, B=None, T=None, D=None, seed=None, with_h0=None) -> ScanInputs:
+    """Draw one minGRU-form diagonal-scan workload (a = 1 - z, b = z * h~)."""
+    if isinstance(spec, str):
+        spec = WORKLOADS[spec]
+    spec = dataclasses.replace(
+        spec, B=spec.B if B is None else B, T=spec.T if T is None else T,
+        D=spec.D if D is None else D, seed=spec.seed if seed is None else seed,
+        with_h0=spec.with_h0 if with_h0 is None else with_h0)
+    rng = np.random.default_rng(spec.seed)
+    shape = (spec.B, spec.T, spec.D)
+    z = 1.0 / (1.0 + np.exp(-rng.normal(0.0, 1.0, size=shape)))
+    h_tilde = rng.normal(0.0, 1.0, size=shape)
+    a = (1.0 - z).astype(np.float32)
+    b = (z * h_tilde).astype(np.float32)
+    h0 = rng.normal(0.0, 1.0, size=(spec.B, spec.D)).astype(np.float32) if spec.with_h0 else None
+    return ScanInputs(spec, a, b, h0)
