@@ -1,0 +1,526 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 WKV forward / diagonal scan library.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step is one pass of the hot path over one batch of synthetic input
+already resident in HBM: a WKV forward (or, for ``--workload scan_mingru``,
+a diagonal scan).  The default workload is the RWKV-4-169M-shaped WKV forward
+(fp32, B=8, T=1024, C=768).  W untimed warm-up steps and a short untimed soak
+run first; then exactly K steps are timed with CUDA events on the launching
+stream, bracketed by a barrier and a device synchronisation, and the maximum
+over ranks is taken.  Inputs rotate over enough buffer sets that the data a
+step touches is not in L2 from the step before (each set is re-read only
+after >= 3x the L2 size of other traffic).
+
+Printed (rank 0): one JSON line with the metric, the roofline of the kernel
+(algorithmic bytes / average CUDA-event launch duration against the measured
+HBM peak), the float64 CPU oracle timed on this host's cores, an end-to-end
+number through the C ABI with host buffers (host->device copies, the call,
+device->host copy of the result, every step), SM clocks sampled during the
+timed region, and the number of library kernel launches timed.
+
+``--impl reference`` times the CPU oracle instead (the only reference this
+project has: a plain float64 implementation of the pages' definition), on a
+bounded sample of the same workload, and prints the same line with
+"impl": "reference".  Multi-GPU runs (torchrun) give every rank its own copy
+of the workload (weak scaling, no collective in the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "WKV fwd B·T·C elems/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+FALLBACK_HBM_GBS = 6650.0
+CSRC = os.path.join(ROOT, "rwkv_wkv_mixing_b200", "csrc")
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default="wkv_169m", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--soak-seconds", type=float, default=1.0,
+                    help="untimed steps before the timed region, so clocks settle")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="budget of the CPU-oracle baseline (rank 0, N=1)")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args(argv)
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def src_hash():
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the kernel sources as they are now; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+    except Exception:
+        return None
+    if not rec or rec.get("src_sha") != src_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples every 100 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id=None):
+        self.samples = []
+        self.proc = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if gpu_id:
+            cmd += ["-i", gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm, smax = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            self.samples.append((time.time(), sm, smax, parts[2], parts[4:8]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if not win:
+            win = self.samples
+            window = "run"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({names[i] for s in win for i, r in enumerate(s[4])
+                          if r.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(s[1] for s in win),
+                "sm_max_mhz": max(s[2] for s in win), "reasons": reasons,
+                "samples": len(win), "window": window}
+
+
+# ---------------------------------------------------------------------------
+# workloads on the device
+# ---------------------------------------------------------------------------
+class DeviceWorkload:
+    """Inputs resident in HBM, rotated over `n_sets` copies, and the C-ABI
+    call of one step with raw device pointers."""
+
+    def __init__(self, name, torch, lib, l2_bytes):
+        self.name = name
+        self.spec = workloads.WORKLOADS[name]
+        self.torch = torch
+        self.lib = lib
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.is_scan = isinstance(self.spec, workloads.ScanSpec)
+        if self.is_scan:
+            x = workloads.make_scan(name)
+            B, T, C = x.a.shape
+            self.host = {"x0": x.a, "x1": x.b}
+            self.dtype, self.es, self.tdtype = "f32", 4, torch.float32
+            self.params = []
+            self.param_bytes = 0
+        else:
+            x = workloads.make_wkv(name)
+            B, T, C = x.k.shape
+            if x.spec.dtype == "bf16":
+                self.host = {"x0": x.k_bits.view(np.int16), "x1": x.v_bits.view(np.int16)}
+                self.dtype, self.es, self.tdtype = "bf16", 2, torch.bfloat16
+            else:
+                self.host = {"x0": x.k, "x1": x.v}
+                self.dtype, self.es, self.tdtype = "f32", 4, torch.float32
+            self.params = [torch.from_numpy(x.w).to(dev), torch.from_numpy(x.u).to(dev)]
+            self.param_bytes = 2 * 4 * C
+        self.inputs = x
+        self.B, self.T, self.C = B, T, C
+        self.elements = B * T * C
+        self.alg_bytes = 3 * self.es * self.elements + self.param_bytes
+        set_bytes = 3 * self.es * self.elements
+        self.n_sets = 1 if set_bytes >= 3 * l2_bytes else int(np.ceil(3 * l2_bytes / set_bytes)) + 1
+        x0 = self._to_dev(self.host["x0"], dev)
+        x1 = self._to_dev(self.host["x1"], dev)
+        self.sets = []
+        for i in range(self.n_sets):
+            a = x0 if i == 0 else x0.clone()
+            b = x1 if i == 0 else x1.clone()
+            self.sets.append((a, b, torch.empty_like(a)))
+        self.stream = torch.cuda.current_stream()
+        self.sh = self.stream.cuda_stream
+
+    def _to_dev(self, arr, dev):
+        t = self.torch.from_numpy(np.ascontiguousarray(arr))
+        if self.dtype == "bf16":
+            t = t.view(self.torch.bfloat16)
+        return t.to(dev)
+
+    def call(self, x0, x1, y):
+        lib = self.lib
+        if self.is_scan:
+            return lib.diag_scan(self.B, self.T, self.C, x0.data_ptr(), x1.data_ptr(), None,
+                                 y.data_ptr(), self.sh)
+        fn = lib.wkv_forward_bf16 if self.dtype == "bf16" else lib.wkv_forward
+        return fn(self.B, self.T, self.C, self.params[0].data_ptr(), self.params[1].data_ptr(),
+                  x0.data_ptr(), x1.data_ptr(), y.data_ptr(), self.sh)
+
+    def step(self, i):
+        st = self.call(*self.sets[i % self.n_sets])
+        if st != 0:
+            raise RuntimeError(f"library call failed: {st}: {self.lib.wkv_last_error().decode()}")
+
+
+def time_steps(torch, wl, K):
+    """K steps back to back; events around the whole region and around every
+    launch (all on the launching stream)."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(wl.stream)
+    for i in range(K):
+        ev[i][0].record(wl.stream)
+        wl.step(i)
+        ev[i][1].record(wl.stream)
+    end.record(wl.stream)
+    end.synchronize()
+    total_ms = start.elapsed_time(end)
+    per = [a.elapsed_time(b) for a, b in ev]
+    return total_ms, per
+
+
+def e2e_leg(torch, wl, steps):
+    """Through the C ABI with host buffers: pinned host inputs are copied to
+    the device, the library runs, the result is copied back, every step."""
+    hx0 = torch.from_numpy(np.ascontiguousarray(wl.host["x0"])).pin_memory()
+    hx1 = torch.from_numpy(np.ascontiguousarray(wl.host["x1"])).pin_memory()
+    if wl.dtype == "bf16":
+        hx0, hx1 = hx0.view(torch.bfloat16), hx1.view(torch.bfloat16)
+    hy = torch.empty_like(hx0).pin_memory()
+    hp = [p.cpu().pin_memory() for p in wl.params]
+    dx0, dx1, dy = wl.sets[0]
+
+    def one():
+        for h, d in zip(hp, wl.params):
+            d.copy_(h, non_blocking=True)
+        dx0.copy_(hx0, non_blocking=True)
+        dx1.copy_(hx1, non_blocking=True)
+        st = wl.call(dx0, dx1, dy)
+        if st != 0:
+            raise RuntimeError("library call failed")
+        hy.copy_(dy, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(wl.stream)
+    for _ in range(steps):
+        one()
+    b.record(wl.stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / steps
+    h2d = hx0.numel() * hx0.element_size() * 2 + wl.param_bytes
+    d2h = hy.numel() * hy.element_size()
+    return {"value": wl.elements / (ms / 1e3), "unit": "elem/s", "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "host_buffers": "pinned"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_runner(name, max_elements=None):
+    """A callable running the float64 oracle once over a sample of the
+    workload, and the sample's element count and description."""
+    import oracle
+    spec = workloads.WORKLOADS[name]
+    if isinstance(spec, workloads.ScanSpec):
+        x = workloads.make_scan(name)
+        a, b = x.a.astype(np.float64), x.b.astype(np.float64)
+        B, T, C = a.shape
+        rows = B if max_elements is None else max(1, min(B, max_elements // (T * C)))
+        a, b = np.ascontiguousarray(a[:rows]), np.ascontiguousarray(b[:rows])
+        fn = lambda: oracle.scan_rnn(a, b, None)   # noqa: E731
+        return fn, rows * T * C, f"{rows} of {B} batch rows (all T={T}, D={C})"
+    x = workloads.make_wkv(name)
+    k, v = x.k.astype(np.float64), x.v.astype(np.float64)
+    w, u = x.w.astype(np.float64), x.u.astype(np.float64)
+    B, T, C = k.shape
+    rows, chans = B, C
+    if max_elements is not None:
+        rows = max(1, min(B, max_elements // (T * C)))
+        if rows * T * C > max_elements:   # even one row is too much: fewer channels
+            chans = max(1, min(C, max_elements // T))
+    k = np.ascontiguousarray(k[:rows, :, :chans]); v = np.ascontiguousarray(v[:rows, :, :chans])
+    w, u = w[:chans], u[:chans]
+    fn = lambda: oracle.wkv_rnn(w, u, k, v)   # noqa: E731
+    return fn, rows * T * chans, f"{rows} of {B} batch rows x {chans} of {C} channels (all T={T})"
+
+
+def cpu_baseline(name, seconds):
+    import oracle
+    fn, n, desc = oracle_runner(name, max_elements=None)
+    t0 = time.perf_counter(); fn(); one = time.perf_counter() - t0
+    if one > seconds:   # a smaller sample of the same workload
+        fn, n, desc = oracle_runner(name, max_elements=max(1, int(n * seconds / one / 2)))
+        t0 = time.perf_counter(); fn(); one = time.perf_counter() - t0
+    reps = max(1, int(seconds / max(one, 1e-6)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        fn()
+    dt = time.perf_counter() - t0
+    return {"value": n * reps / dt, "unit": "elem/s", "cores": oracle.max_threads(),
+            "kind": "oracle", "sample": f"{desc}, {reps} passes, float64 RNN-mode oracle",
+            "seconds": dt, "cpu": cpu_model()}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    budget = 150.0   # whole run within a few minutes
+    fn, n, desc = oracle_runner(args.workload)
+    t0 = time.perf_counter(); fn(); one = time.perf_counter() - t0
+    per_step = budget / max(1, args.steps + args.warmup)
+    if one > per_step:
+        fn, n, desc = oracle_runner(args.workload, max_elements=max(1, int(n * per_step / one)))
+    for _ in range(args.warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    spec = workloads.WORKLOADS[args.workload]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "elem/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(spec, args.workload),
+        "cpu_baseline": {"value": value, "unit": "elem/s", "cores": oracle.max_threads(),
+                         "kind": "oracle", "sample": f"{desc} per step, float64 RNN-mode oracle"},
+        "e2e": {"value": value, "unit": "elem/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(spec, name):
+    if isinstance(spec, workloads.ScanSpec):
+        return {"workload": name, "op": "diag_scan", "B": spec.B, "T": spec.T, "D": spec.D,
+                "io": "f32"}
+    return {"workload": name, "op": "wkv_forward" + ("_bf16" if spec.dtype == "bf16" else ""),
+            "B": spec.B, "T": spec.T, "C": spec.C, "io": spec.dtype}
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+
+    import rwkv_wkv_mixing_b200 as wkv
+    props = torch.cuda.get_device_properties(local)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    wl = DeviceWorkload(args.workload, torch, wkv.lib, l2)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up, then an untimed soak so clocks and caches reach steady state
+    for i in range(args.warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
+    wkv.wkv_device_status()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(props.uuid)
+    except Exception:
+        pass
+    sampler = None if args.no_clocks else ClockSampler(uuid)
+    t_soak = time.time()
+    if args.soak_seconds > 0:
+        t_end = time.time() + args.soak_seconds
+        i = 0
+        while time.time() < t_end:
+            for _ in range(64):
+                wl.step(i); i += 1
+            torch.cuda.synchronize()
+
+    barrier()
+    t_timed0 = time.time()
+    total_ms, per = time_steps(torch, wl, args.steps)
+    barrier()
+    t_timed1 = time.time()
+    if sampler is not None:
+        time.sleep(0.25)
+        sampler.stop()
+    wkv.wkv_device_status()   # raises if a device-side wait gave up
+
+    if pg is not None:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    ms_per_step = total_ms / args.steps
+    value = wl.elements * world / (ms_per_step / 1e3)
+    launch_ms = statistics.mean(per)
+    peak, peak_kind = read_peaks()
+    achieved = wl.alg_bytes / (launch_ms / 1e3) / 1e9
+    traffic = recorded_traffic(args.workload)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_leg(torch, wl, args.e2e_steps)
+        if pg is not None:
+            t = torch.tensor([e2e["ms_per_step"]], device="cuda", dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(t.item())
+            e2e["value"] = wl.elements * world / (e2e["ms_per_step"] / 1e3)
+        wkv.wkv_device_status()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(args.workload, args.cpu_seconds)
+
+    spec = wl.spec
+    cfg = workload_config(spec, args.workload)
+    cfg.update({"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "l2": (f"inputs rotate over {wl.n_sets} buffer sets "
+                       f"({wl.n_sets * 3 * wl.es * wl.elements / 1e6:.0f} MB > L2 "
+                       f"{l2 / 1e6:.0f} MB)"),
+                "tile_steps": wkv.wkv_get_tile_steps(),
+                "gpu": props.name, "sms": props.multi_processor_count})
+    line = {
+        "metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (seeded, distributions of the named workload)",
+        "config": cfg,
+        "hbm_gbs": wl.alg_bytes * world / (ms_per_step / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind,
+                     "traffic": traffic, "alg_bytes_per_launch": wl.alg_bytes,
+                     "launch_ms_mean": launch_ms,
+                     "launch_ms_median": statistics.median(per),
+                     "kernel": "chunked_scan_kernel"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(t_timed0, t_timed1) if sampler is not None else None,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,127 @@
+/*
+ * wkv_b200.h -- C ABI of the B200 (sm_100a) RWKV-4 WKV forward and
+ * per-channel diagonal linear scan library (libwkv_b200.so).
+ *
+ * Operations
+ * ----------
+ * wkv_forward / wkv_forward_bf16
+ *   The RWKV-4 time-mixing WKV operator, eq. (14) of "RWKV：基于RNN的LLM"
+ *   (section 二.1, Time-mixing block), written 0-based: for every batch row
+ *   b, channel c and step t,
+ *
+ *     y[b,t,c] = ( sum_{i<t} e^{-(t-1-i) w[c] + k[b,i,c]} v[b,i,c] + e^{u[c] + k[b,t,c]} v[b,t,c] )
+ *              / ( sum_{i<t} e^{-(t-1-i) w[c] + k[b,i,c]}          + e^{u[c] + k[b,t,c]} )
+ *
+ *   w is the per-channel decay, non-negative per eq. (10) of the same page
+ *   (section 一.2); u is the bonus of the current token.  y[b,0,c] = v[b,0,c].
+ *
+ * diag_scan
+ *   The per-channel diagonal linear recurrence the LRU and minGRU pages reduce
+ *   their RNNs to ("Were RNNs All We Needed?", model-architecture section:
+ *   v_t = a_t (.) v_{t-1} + b_t; review of "Resurrecting Recurrent Neural
+ *   Networks for Long Sequences", linear-RNN section):
+ *
+ *     h[b,t,d] = a[b,t,d] * h[b,t-1,d] + b[b,t,d],    h[b,-1,d] = h0[b,d] (or 0).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout    k, v, y, a, b, h are dense row-major [B, T, C] (or [B, T, D])
+ *           tensors with the channel index fastest; w, u are [C]; h0 is [B, D].
+ * Memory    every pointer is a DEVICE pointer on the current CUDA device,
+ *           owned by the caller.  Outputs must not overlap inputs.
+ * Streams   calls are asynchronous on `stream` (NULL = legacy default stream):
+ *           a return of WKV_OK means the work was queued.
+ * Types     fp32 entry points read and write IEEE float.  wkv_forward_bf16
+ *           reads k, v and writes y as bfloat16 bit patterns (wkv_bf16_t),
+ *           computes in fp32 and rounds y to nearest even; w, u stay fp32.
+ * Sizes     B, T, C (D) >= 0; an empty tensor (any size 0) is a no-op.
+ *           B*T*C must be < 2^62.
+ * Scratch   inputs with T longer than one tile (256 steps) carry state between
+ *           thread blocks through a small library-owned device workspace, one
+ *           per (device, stream), allocated with cudaMalloc on first use and
+ *           grown when a larger problem needs it.  Make one call of each size
+ *           before capturing a stream into a CUDA graph.  Calls on different
+ *           streams use different workspaces and may run concurrently.
+ * Errors    argument errors are detected on the host before anything is
+ *           launched and return a non-zero wkv_status; wkv_last_error()
+ *           then describes the problem (thread-local, valid until the next
+ *           call on that thread).  Value preconditions (w >= 0, finite
+ *           inputs) are documented, not checked: NaN propagates.
+ *           A device-side wait that gives up (see wkv_device_status) writes
+ *           NaN outputs for the affected tile and raises WKV_ERR_TIMEOUT
+ *           instead of hanging.
+ */
+#ifndef WKV_B200_H
+#define WKV_B200_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define WKV_API __attribute__((visibility("default")))
+#else
+#define WKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WKV_OK = 0,
+    WKV_ERR_INVALID_ARG = 1,  /* bad size, NULL pointer, overlapping output  */
+    WKV_ERR_ALIGNMENT = 2,    /* pointer not aligned to its element size     */
+    WKV_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed           */
+    WKV_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up          */
+    WKV_ERR_OOM = 5           /* workspace allocation failed                 */
+} wkv_status;
+
+/* bfloat16 storage: the upper 16 bits of the IEEE float32 pattern */
+typedef uint16_t wkv_bf16_t;
+
+/* WKV forward, fp32 I/O.  k, v, y: [B, T, C] float; w, u: [C] float.
+ * Pointers must be 4-byte aligned.  (16-byte aligned pointers with C a
+ * multiple of 4 take the TMA tile path; anything else takes the same kernel
+ * with element-wise tile loads.) */
+WKV_API wkv_status wkv_forward(int64_t B, int64_t T, int64_t C,
+                       const float *w, const float *u,
+                       const float *k, const float *v, float *y,
+                       cudaStream_t stream);
+
+/* WKV forward, bfloat16 k/v/y with fp32 state.  w, u: [C] float.
+ * Pointers must be 2-byte aligned (TMA path: 16-byte and C % 8 == 0). */
+WKV_API wkv_status wkv_forward_bf16(int64_t B, int64_t T, int64_t C,
+                            const float *w, const float *u,
+                            const wkv_bf16_t *k, const wkv_bf16_t *v, wkv_bf16_t *y,
+                            cudaStream_t stream);
+
+/* Diagonal linear scan, fp32.  a, b, h: [B, T, D] float; h0: [B, D] float or
+ * NULL (zero initial state).  Pointers must be 4-byte aligned. */
+WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,
+                     const float *a, const float *b, const float *h0, float *h,
+                     cudaStream_t stream);
+
+/* Synchronise `stream`, then return and clear the device status word of that
+ * stream's workspace: WKV_OK, or WKV_ERR_TIMEOUT if a device-side wait gave up
+ * since the last query.  WKV_ERR_CUDA if the synchronisation itself failed. */
+WKV_API wkv_status wkv_device_status(cudaStream_t stream);
+
+/* Message for the last non-OK return on the calling thread ("" if none). */
+WKV_API const char *wkv_last_error(void);
+
+/* Free every workspace the library holds on the current device (synchronises
+ * the device first).  Later calls allocate again on demand. */
+WKV_API wkv_status wkv_release_workspaces(void);
+
+/* Tuning knob, process-wide: the number of steps one thread block stages per
+ * tile (8, 32, 64, 128 or 256; default 256).  Results do not depend on it
+ * beyond rounding: it only moves the boundaries where chunk summaries are
+ * combined.  WKV_ERR_INVALID_ARG for any other value. */
+WKV_API wkv_status wkv_set_tile_steps(int steps);
+WKV_API int wkv_get_tile_steps(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_B200_H */

@@ -1,0 +1,167 @@
+"""Python binding of libwkv_b200.so (RWKV-4 WKV forward and the diagonal
+linear scan on B200 / sm_100a).
+
+Argument marshalling only: every entry point takes torch CUDA tensors, checks
+dtype / shape / contiguity, and calls the C function of the same name with
+raw device pointers and the current torch CUDA stream.  All arithmetic runs
+in the library's kernels; there is no CPU fallback, and importing this module
+raises if the library has not been built.
+
+    y = wkv_forward(w, u, k, v)            # fp32 [B,T,C] k, v; [C] w, u
+    y = wkv_forward_bf16(w, u, k, v)       # bf16 k, v -> bf16 y, fp32 state
+    h = diag_scan(a, b, h0=None)           # fp32 [B,T,D]; h0 [B,D] or None
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwkv_b200.so")
+
+WKV_OK = 0
+WKV_ERR_INVALID_ARG = 1
+WKV_ERR_ALIGNMENT = 2
+WKV_ERR_CUDA = 3
+WKV_ERR_TIMEOUT = 4
+WKV_ERR_OOM = 5
+STATUS_NAMES = {0: "WKV_OK", 1: "WKV_ERR_INVALID_ARG", 2: "WKV_ERR_ALIGNMENT",
+                3: "WKV_ERR_CUDA", 4: "WKV_ERR_TIMEOUT", 5: "WKV_ERR_OOM"}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m rwkv_wkv_mixing_b200.build` (nvcc, sm_100a)")
+
+_i64, _p, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+lib = ctypes.CDLL(LIB_PATH)
+_SIGS = {
+    "wkv_forward": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_bf16": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
+    "diag_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
+    "wkv_device_status": ([_p], _i32),
+    "wkv_last_error": ([], ctypes.c_char_p),
+    "wkv_release_workspaces": ([], _i32),
+    "wkv_set_tile_steps": ([_i32], _i32),
+    "wkv_get_tile_steps": ([], _i32),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+class WkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.wkv_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != WKV_OK:
+        raise WkvError(status, where)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, ndim):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _wkv(fn_name, io_dtype, w, u, k, v, y, stream):
+    import torch
+    _need(k, "k", io_dtype, 3)
+    _need(v, "v", io_dtype, 3)
+    _need(w, "w", torch.float32, 1)
+    _need(u, "u", torch.float32, 1)
+    if k.shape != v.shape:
+        raise ValueError("k and v must have one shape")
+    B, T, C = k.shape
+    if w.shape[0] != C or u.shape[0] != C:
+        raise ValueError("w and u must be [C]")
+    if y is None:
+        y = torch.empty_like(k)
+    else:
+        _need(y, "y", io_dtype, 3)
+        if y.shape != k.shape:
+            raise ValueError("y must have the shape of k")
+    _check(getattr(lib, fn_name)(B, T, C, w.data_ptr(), u.data_ptr(), k.data_ptr(),
+                                 v.data_ptr(), y.data_ptr(), _stream_handle(stream)), fn_name)
+    return y
+
+
+def wkv_forward(w, u, k, v, y=None, stream=None):
+    """WKV forward, fp32: y[b,t,c] per eq. (14) of the RWKV page."""
+    import torch
+    return _wkv("wkv_forward", torch.float32, w, u, k, v, y, stream)
+
+
+def wkv_forward_bf16(w, u, k, v, y=None, stream=None):
+    """WKV forward, bf16 k/v/y with fp32 state and fp32 w, u."""
+    import torch
+    return _wkv("wkv_forward_bf16", torch.bfloat16, w, u, k, v, y, stream)
+
+
+def diag_scan(a, b, h0=None, h=None, stream=None):
+    """h_t = a_t * h_{t-1} + b_t per channel, h_{-1} = h0 (zeros if None)."""
+    import torch
+    _need(a, "a", torch.float32, 3)
+    _need(b, "b", torch.float32, 3)
+    if a.shape != b.shape:
+        raise ValueError("a and b must have one shape")
+    B, T, D = a.shape
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, 2)
+        if tuple(h0.shape) != (B, D):
+            raise ValueError("h0 must be [B, D]")
+    if h is None:
+        h = torch.empty_like(a)
+    else:
+        _need(h, "h", torch.float32, 3)
+        if h.shape != a.shape:
+            raise ValueError("h must have the shape of a")
+    _check(lib.diag_scan(B, T, D, a.data_ptr(), b.data_ptr(),
+                         None if h0 is None else h0.data_ptr(), h.data_ptr(),
+                         _stream_handle(stream)), "diag_scan")
+    return h
+
+
+def wkv_device_status(stream=None):
+    """Synchronise the stream; raise WkvError if a device-side wait gave up."""
+    _check(lib.wkv_device_status(_stream_handle(stream)), "wkv_device_status")
+
+
+def wkv_last_error() -> str:
+    return lib.wkv_last_error().decode(errors="replace")
+
+
+def wkv_release_workspaces():
+    _check(lib.wkv_release_workspaces(), "wkv_release_workspaces")
+
+
+def wkv_set_tile_steps(steps: int):
+    _check(lib.wkv_set_tile_steps(int(steps)), "wkv_set_tile_steps")
+
+
+def wkv_get_tile_steps() -> int:
+    return int(lib.wkv_get_tile_steps())
+
+
+__all__ = ["wkv_forward", "wkv_forward_bf16", "diag_scan", "wkv_device_status",
+           "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
+           "wkv_get_tile_steps", "WkvError", "lib", "LIB_PATH"]

@@ -1,0 +1,441 @@
+// C ABI of libwkv_b200.so: argument checks, tensor maps, per-stream
+// workspaces and kernel dispatch.  The declarations and their contracts are
+// in include/wkv_b200.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "chunked_scan.cuh"
+#include "wkv_b200.h"
+#include "wkv_ops.cuh"
+
+using namespace wkvb;
+
+namespace {
+
+thread_local std::string t_err;
+
+wkv_status fail(wkv_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_err = buf;
+    return st;
+}
+
+wkv_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(WKV_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ---- driver entry points (no link-time dependency on libcuda) --------------
+struct Driver {
+    PFN_cuTensorMapEncodeTiled_v12000 encode_tiled = nullptr;
+    PFN_cuMemGetAddressRange_v3020 get_address_range = nullptr;
+};
+
+const Driver &driver() {
+    static Driver d;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            d.encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            d.get_address_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(p);
+        cudaGetLastError();
+    });
+    return d;
+}
+
+// ---- tuning knob: tile length in steps ---------------------------------------
+std::atomic<int> g_tile_steps{256};
+
+// ---- argument checks ------------------------------------------------------------
+// `p` must be device (or managed) memory of device `dev` holding `bytes`.
+wkv_status check_buffer(const void *p, size_t bytes, size_t align, const char *name, int dev) {
+    if (p == nullptr) return fail(WKV_ERR_INVALID_ARG, "%s is NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) % align != 0)
+        return fail(WKV_ERR_ALIGNMENT, "%s is not %zu-byte aligned", name, align);
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(WKV_ERR_INVALID_ARG, "%s: not a CUDA pointer (%s)", name, cudaGetErrorName(e));
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+        return fail(WKV_ERR_INVALID_ARG, "%s is not device memory", name);
+    if (attr.type == cudaMemoryTypeDevice && attr.device != dev)
+        return fail(WKV_ERR_INVALID_ARG, "%s lives on device %d, current device is %d", name,
+                    attr.device, dev);
+    const Driver &d = driver();
+    if (d.get_address_range != nullptr) {
+        CUdeviceptr base = 0;
+        size_t size = 0;
+        if (d.get_address_range(&base, &size, reinterpret_cast<CUdeviceptr>(p)) == CUDA_SUCCESS) {
+            const uintptr_t end = static_cast<uintptr_t>(base) + size;
+            if (reinterpret_cast<uintptr_t>(p) + bytes > end)
+                return fail(WKV_ERR_INVALID_ARG,
+                            "%s: %zu bytes needed but its allocation ends %zu bytes after it",
+                            name, bytes, static_cast<size_t>(end - reinterpret_cast<uintptr_t>(p)));
+        }
+    }
+    return WKV_OK;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+wkv_status check_sizes(int64_t B, int64_t T, int64_t C, bool *empty) {
+    if (B < 0 || T < 0 || C < 0)
+        return fail(WKV_ERR_INVALID_ARG, "negative size (B=%lld T=%lld C=%lld)",
+                    static_cast<long long>(B), static_cast<long long>(T),
+                    static_cast<long long>(C));
+    *empty = B == 0 || T == 0 || C == 0;
+    if (*empty) return WKV_OK;
+    if (B > INT32_MAX || T > INT32_MAX || C > INT32_MAX)
+        return fail(WKV_ERR_INVALID_ARG, "each of B, T, C must be below 2^31");
+    const unsigned __int128 n = static_cast<unsigned __int128>(B) * T * C;
+    if (n >= (static_cast<unsigned __int128>(1) << 62))
+        return fail(WKV_ERR_INVALID_ARG, "B*T*C must be below 2^62");
+    return WKV_OK;
+}
+
+// ---- per-(device, stream) workspaces for the cross-tile look-back -------------
+// A workspace is only ever used by launches on its own stream, which run one
+// after another; its counters reset themselves on the device (see Workspace in
+// chunked_scan.cuh).  When a larger problem needs a larger workspace the old
+// buffer is retired, not freed, so CUDA graphs captured earlier keep valid
+// pointers; wkv_release_workspaces() frees everything.
+struct WsEntry {
+    int device = -1;
+    cudaStream_t stream = nullptr;
+    char *base = nullptr;
+    size_t bytes = 0;
+};
+
+std::mutex g_mu;                  // guards g_ws and g_retired
+std::vector<WsEntry *> g_ws;
+std::vector<std::pair<int, void *>> g_retired;  // (device, buffer)
+
+// header: [0] u32 ticket, [4] u32 done, [8] u64 epoch, [16] i32 status
+constexpr size_t kWsHeader = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+    size_t flags, agg, incl, total;
+};
+
+WsLayout ws_layout(size_t tiles, size_t floats_per_tile) {
+    WsLayout l;
+    l.flags = kWsHeader;
+    l.agg = round_up(l.flags + tiles * sizeof(unsigned long long), 256);
+    l.incl = round_up(l.agg + tiles * floats_per_tile * sizeof(float), 256);
+    l.total = round_up(l.incl + tiles * floats_per_tile * sizeof(float), 256);
+    return l;
+}
+
+WsEntry *find_ws(int dev, cudaStream_t stream) {
+    for (WsEntry *e : g_ws)
+        if (e->device == dev && e->stream == stream) return e;
+    return nullptr;
+}
+
+// caller holds g_mu
+wkv_status ensure_ws(int dev, cudaStream_t stream, size_t need, WsEntry **out) {
+    WsEntry *e = find_ws(dev, stream);
+    if (e != nullptr && e->bytes >= need) {
+        *out = e;
+        return WKV_OK;
+    }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) == cudaSuccess && cap != cudaStreamCaptureStatusNone)
+        return fail(WKV_ERR_CUDA,
+                    "this call needs a %zu-byte look-back workspace for its stream, which "
+                    "cannot be allocated during stream capture: make one call of this size "
+                    "on the stream before capturing it", need);
+    cudaGetLastError();
+    const size_t nb = round_up(e != nullptr && need < 2 * e->bytes ? 2 * e->bytes : need, 1 << 20);
+    void *p = nullptr;
+    cudaError_t err = cudaMalloc(&p, nb);
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return fail(WKV_ERR_OOM, "workspace of %zu bytes: %s", nb, cudaGetErrorName(err));
+    }
+    err = cudaMemsetAsync(p, 0, nb, stream);
+    if (err != cudaSuccess) {
+        cudaFree(p);
+        return cuda_fail(err, "cudaMemsetAsync(workspace)");
+    }
+    if (e == nullptr) {
+        e = new WsEntry;
+        e->device = dev;
+        e->stream = stream;
+        g_ws.push_back(e);
+    } else if (e->base != nullptr) {
+        g_retired.emplace_back(dev, e->base);
+    }
+    e->base = static_cast<char *>(p);
+    e->bytes = nb;
+    *out = e;
+    return WKV_OK;
+}
+
+// ---- tensor maps ------------------------------------------------------------------
+bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, size_t es, int64_t B,
+              int64_t T, int64_t C, int box_c, int box_t) {
+    const Driver &d = driver();
+    if (d.encode_tiled == nullptr) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T),
+                          static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(C * es), static_cast<cuuint64_t>(T * C * es)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_c), static_cast<cuuint32_t>(box_t), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = d.encode_tiled(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// TMA tile copies need 16-byte aligned bases, rows of a multiple of 16 bytes
+// and a batch stride below 2^40 bytes.
+bool tma_eligible(const void *const *ptrs, int n, size_t es, int64_t T, int64_t C) {
+    for (int i = 0; i < n; ++i)
+        if (reinterpret_cast<uintptr_t>(ptrs[i]) % 16 != 0) return false;
+    if ((C * es) % 16 != 0) return false;
+    if (static_cast<unsigned __int128>(T) * C * es >= (static_cast<unsigned __int128>(1) << 40))
+        return false;
+    return driver().encode_tiled != nullptr;
+}
+
+// ---- launch -------------------------------------------------------------------------
+constexpr long long kSpinLimit = 1ll << 21;  // ~0.1-1 s of polling
+
+template <class Op, int LT, int NW>
+wkv_status launch_tiles(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
+                        CUtensorMapDataType dt, cudaStream_t stream, int dev) {
+    constexpr int CG = 32 * Op::CPT;
+    using io_t = typename Op::io_t;
+    Geometry g;
+    g.B = static_cast<int>(B);
+    g.T = static_cast<int>(T);
+    g.C = static_cast<int>(C);
+    g.n_cg = static_cast<int>((C + CG - 1) / CG);
+    g.n_seg = static_cast<int>((T + LT - 1) / LT);
+    const long long tiles_per_seg = B * static_cast<long long>(g.n_cg);
+    const long long tiles = tiles_per_seg * g.n_seg;
+    if (tiles > INT32_MAX) return fail(WKV_ERR_INVALID_ARG, "problem has too many tiles");
+    g.tiles_per_seg = static_cast<int>(tiles_per_seg);
+    g.tiles = static_cast<int>(tiles);
+    g.spin_limit = kSpinLimit;
+
+    CUtensorMap maps[3];
+    std::memset(maps, 0, sizeof maps);
+    const void *ptrs[3] = {args.x0, args.x1, args.y};
+    g.use_tma = tma_eligible(ptrs, 3, sizeof(io_t), T, C) ? 1 : 0;
+    if (g.use_tma) {
+        for (int i = 0; i < 3 && g.use_tma; ++i)
+            if (!make_map(&maps[i], ptrs[i], dt, sizeof(io_t), B, T, C, CG, LT)) g.use_tma = 0;
+    }
+
+    constexpr size_t smem = chunked_scan_smem_bytes<Op, LT, NW>();
+    auto kern = chunked_scan_kernel<Op, LT, NW>;
+    static std::atomic<uint64_t> configured{0};  // one bit per device
+    if (dev < 64 && !(configured.load() & (1ull << dev))) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        configured.fetch_or(1ull << dev);
+    }
+
+    Workspace ws;
+    std::memset(&ws, 0, sizeof ws);
+    if (g.n_seg > 1) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        const WsLayout l = ws_layout(static_cast<size_t>(tiles), Op::NV * CG);
+        WsEntry *e = nullptr;
+        wkv_status st = ensure_ws(dev, stream, l.total, &e);
+        if (st != WKV_OK) return st;
+        ws.ticket = reinterpret_cast<unsigned int *>(e->base);
+        ws.done = reinterpret_cast<unsigned int *>(e->base + 4);
+        ws.epoch = reinterpret_cast<unsigned long long *>(e->base + 8);
+        ws.status = reinterpret_cast<int *>(e->base + 16);
+        ws.flags = reinterpret_cast<unsigned long long *>(e->base + l.flags);
+        ws.agg = reinterpret_cast<float *>(e->base + l.agg);
+        ws.incl = reinterpret_cast<float *>(e->base + l.incl);
+    }
+    cudaGetLastError();  // clear a stale error so the check below is about this launch
+    kern<<<static_cast<unsigned>(tiles), NW * 32, smem, stream>>>(maps[0], maps[1], maps[2], args,
+                                                                 g, ws);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
+template <class Op>
+wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
+                    CUtensorMapDataType dt, cudaStream_t stream, int dev) {
+    switch (g_tile_steps.load()) {
+        case 8: return launch_tiles<Op, 8, 8>(args, B, T, C, dt, stream, dev);
+        case 32: return launch_tiles<Op, 32, 8>(args, B, T, C, dt, stream, dev);
+        case 64: return launch_tiles<Op, 64, 8>(args, B, T, C, dt, stream, dev);
+        case 128: return launch_tiles<Op, 128, 8>(args, B, T, C, dt, stream, dev);
+        default: return launch_tiles<Op, 256, 8>(args, B, T, C, dt, stream, dev);
+    }
+}
+
+wkv_status current_device(int *dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    return WKV_OK;
+}
+
+template <typename IO>
+wkv_status wkv_common(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                      const IO *k, const IO *v, IO *y, cudaStream_t stream,
+                      CUtensorMapDataType dt) {
+    t_err.clear();
+    bool empty = false;
+    wkv_status st = check_sizes(B, T, C, &empty);
+    if (st != WKV_OK || empty) return st;
+    int dev = 0;
+    if ((st = current_device(&dev)) != WKV_OK) return st;
+    const size_t n = static_cast<size_t>(B) * T * C * sizeof(IO);
+    const size_t nc = static_cast<size_t>(C) * sizeof(float);
+    if ((st = check_buffer(w, nc, 4, "w", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(u, nc, 4, "u", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(k, n, sizeof(IO), "k", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(v, n, sizeof(IO), "v", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(y, n, sizeof(IO), "y", dev)) != WKV_OK) return st;
+    if (overlaps(y, n, k, n) || overlaps(y, n, v, n) || overlaps(y, n, w, nc) ||
+        overlaps(y, n, u, nc))
+        return fail(WKV_ERR_INVALID_ARG, "y overlaps an input");
+    typename WkvOp<IO, sizeof(IO) == 2 ? 2 : 1>::Args args{k, v, y, w, u};
+    return dispatch<WkvOp<IO, sizeof(IO) == 2 ? 2 : 1>>(args, B, T, C, dt, stream, dev);
+}
+
+}  // namespace
+
+extern "C" {
+
+wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                       const float *k, const float *v, float *y, cudaStream_t stream) {
+    return wkv_common<float>(B, T, C, w, u, k, v, y, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+}
+
+wkv_status wkv_forward_bf16(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                            const wkv_bf16_t *k, const wkv_bf16_t *v, wkv_bf16_t *y,
+                            cudaStream_t stream) {
+    return wkv_common<__nv_bfloat16>(B, T, C, w, u, reinterpret_cast<const __nv_bfloat16 *>(k),
+                                     reinterpret_cast<const __nv_bfloat16 *>(v),
+                                     reinterpret_cast<__nv_bfloat16 *>(y), stream,
+                                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+wkv_status diag_scan(int64_t B, int64_t T, int64_t D, const float *a, const float *b,
+                     const float *h0, float *h, cudaStream_t stream) {
+    t_err.clear();
+    bool empty = false;
+    wkv_status st = check_sizes(B, T, D, &empty);
+    if (st != WKV_OK || empty) return st;
+    int dev = 0;
+    if ((st = current_device(&dev)) != WKV_OK) return st;
+    const size_t n = static_cast<size_t>(B) * T * D * sizeof(float);
+    const size_t n0 = static_cast<size_t>(B) * D * sizeof(float);
+    if ((st = check_buffer(a, n, 4, "a", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(b, n, 4, "b", dev)) != WKV_OK) return st;
+    if (h0 != nullptr && (st = check_buffer(h0, n0, 4, "h0", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(h, n, 4, "h", dev)) != WKV_OK) return st;
+    if (overlaps(h, n, a, n) || overlaps(h, n, b, n) || overlaps(h, n, h0, h0 ? n0 : 0))
+        return fail(WKV_ERR_INVALID_ARG, "h overlaps an input");
+    ScanOp::Args args{a, b, h, h0};
+    return dispatch<ScanOp>(args, B, T, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, stream, dev);
+}
+
+wkv_status wkv_device_status(cudaStream_t stream) {
+    t_err.clear();
+    int dev = 0;
+    wkv_status st = current_device(&dev);
+    if (st != WKV_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    std::lock_guard<std::mutex> lk(g_mu);
+    WsEntry *w = find_ws(dev, stream);
+    if (w == nullptr || w->base == nullptr) return WKV_OK;
+    int code = 0;
+    e = cudaMemcpy(&code, w->base + 16, sizeof code, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+    if (code != 0) {
+        e = cudaMemset(w->base + 16, 0, sizeof code);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+        return fail(static_cast<wkv_status>(code),
+                    "a device-side wait gave up; the affected outputs are NaN");
+    }
+    return WKV_OK;
+}
+
+const char *wkv_last_error(void) { return t_err.c_str(); }
+
+wkv_status wkv_release_workspaces(void) {
+    t_err.clear();
+    int dev = 0;
+    wkv_status st = current_device(&dev);
+    if (st != WKV_OK) return st;
+    std::lock_guard<std::mutex> lk(g_mu);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    for (auto it = g_ws.begin(); it != g_ws.end();) {
+        if ((*it)->device == dev) {
+            if ((*it)->base) cudaFree((*it)->base);
+            delete *it;
+            it = g_ws.erase(it);
+        } else {
+            ++it;
+        }
+    }
+    for (auto it = g_retired.begin(); it != g_retired.end();) {
+        if (it->first == dev) {
+            cudaFree(it->second);
+            it = g_retired.erase(it);
+        } else {
+            ++it;
+        }
+    }
+    return WKV_OK;
+}
+
+wkv_status wkv_set_tile_steps(int steps) {
+    t_err.clear();
+    if (steps != 8 && steps != 32 && steps != 64 && steps != 128 && steps != 256)
+        return fail(WKV_ERR_INVALID_ARG, "tile steps must be 8, 32, 64, 128 or 256");
+    g_tile_steps.store(steps);
+    return WKV_OK;
+}
+
+int wkv_get_tile_steps(void) { return g_tile_steps.load(); }
+
+}  // extern "C"

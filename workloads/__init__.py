@@ -132,6 +132,7 @@ class ScanInputs:
     a: np.ndarray   # [B, T, D] float32
     b: np.ndarray   # [B, T, D] float32
     h0: Optional[np.ndarray]   # [B, D] float32 or None (zeros)
+    h_tilde: Optional[np.ndarray] = None   # [B, T, D] float32, the candidate states
 
 
 def _draw_log_w(rng, spec_w, C):
@@ -180,4 +181,4 @@ def make_scan(spec, *, B=None, T=None, D=None, seed=None, with_h0=None) -> ScanI
     a = (1.0 - z).astype(np.float32)
     b = (z * h_tilde).astype(np.float32)
     h0 = rng.normal(0.0, 1.0, size=(spec.B, spec.D)).astype(np.float32) if spec.with_h0 else None
-    return ScanInputs(spec, a, b, h0)
+    return ScanInputs(spec, a, b, h0, h_tilde.astype(np.float32))
