@@ -388,6 +388,20 @@ def run_reference(args):
     return 0
 
 
+def max_over_ranks(dist, value, device):
+    """The largest `value` over all ranks (every rank gets it)."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(elements_per_rank, world, ms_per_step):
+    """Whole-job throughput: every rank processes its own copy of the
+    workload each step (weak scaling); the step time is the slowest rank's."""
+    return elements_per_rank * world / (ms_per_step / 1e3)
+
+
 def workload_config(spec, name):
     if isinstance(spec, workloads.ScanSpec):
         return {"workload": name, "op": "diag_scan", "B": spec.B, "T": spec.T, "D": spec.D,
@@ -463,12 +477,10 @@ def main(argv=None):
     wkv.wkv_device_status()   # raises if a device-side wait gave up
 
     if pg is not None:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(pg, total_ms, "cuda")
 
     ms_per_step = total_ms / args.steps
-    value = wl.elements * world / (ms_per_step / 1e3)
+    value = aggregate_rate(wl.elements, world, ms_per_step)
     launch_ms = statistics.mean(per)
     peak, peak_kind = read_peaks()
     achieved = wl.alg_bytes / (launch_ms / 1e3) / 1e9
@@ -478,10 +490,8 @@ def main(argv=None):
     if not args.no_e2e:
         e2e = e2e_leg(torch, wl, args.e2e_steps)
         if pg is not None:
-            t = torch.tensor([e2e["ms_per_step"]], device="cuda", dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(t.item())
-            e2e["value"] = wl.elements * world / (e2e["ms_per_step"] / 1e3)
+            e2e["ms_per_step"] = max_over_ranks(pg, e2e["ms_per_step"], "cuda")
+            e2e["value"] = aggregate_rate(wl.elements, world, e2e["ms_per_step"])
         wkv.wkv_device_status()
 
     cpu = None

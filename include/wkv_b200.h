@@ -114,7 +114,7 @@ WKV_API const char *wkv_last_error(void);
 WKV_API wkv_status wkv_release_workspaces(void);
 
 /* Tuning knob, process-wide: the number of steps one thread block stages per
- * tile (8, 32, 64, 128 or 256; default 256).  Results do not depend on it
+ * tile (8, 32, 64, 128 or 256; default 128).  Results do not depend on it
  * beyond rounding: it only moves the boundaries where chunk summaries are
  * combined.  WKV_ERR_INVALID_ARG for any other value. */
 WKV_API wkv_status wkv_set_tile_steps(int steps);

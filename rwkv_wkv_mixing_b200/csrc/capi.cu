@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdint>
@@ -15,6 +16,7 @@
 #include <vector>
 
 #include "chunked_scan.cuh"
+#include "persistent_scan.cuh"
 #include "wkv_b200.h"
 #include "wkv_ops.cuh"
 
@@ -65,7 +67,7 @@ const Driver &driver() {
 }
 
 // ---- tuning knob: tile length in steps ---------------------------------------
-std::atomic<int> g_tile_steps{256};
+std::atomic<int> g_tile_steps{128};
 
 // ---- argument checks ------------------------------------------------------------
 // `p` must be device (or managed) memory of device `dev` holding `bytes`.
@@ -230,56 +232,62 @@ bool tma_eligible(const void *const *ptrs, int n, size_t es, int64_t T, int64_t 
 }
 
 // ---- launch -------------------------------------------------------------------------
-constexpr long long kSpinLimit = 1ll << 21;  // ~0.1-1 s of polling
+constexpr long long kSpinLimit = 1ll << 21;  // look-back polls, ~0.1-1 s
 
-template <class Op, int LT, int NW>
-wkv_status launch_tiles(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
-                        CUtensorMapDataType dt, cudaStream_t stream, int dev) {
+int sm_count(int dev) {
+    static std::atomic<int> cache[64];
+    if (dev >= 0 && dev < 64 && cache[dev].load() > 0) return cache[dev].load();
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = 148;
+    }
+    if (dev >= 0 && dev < 64) cache[dev].store(n);
+    return n;
+}
+
+// Geometry, tensor maps and (for sequences longer than one tile) the
+// look-back workspace of one call; `cg` channels and `lt` steps per tile.
+struct Plan {
+    Geometry g;
+    CUtensorMap maps[3];
+    Workspace ws;
+};
+
+template <class Op>
+wkv_status make_plan(const typename Op::Args &args, int64_t B, int64_t T, int64_t C, int lt,
+                     CUtensorMapDataType dt, cudaStream_t stream, int dev, bool want_tma,
+                     Plan *p) {
     constexpr int CG = 32 * Op::CPT;
     using io_t = typename Op::io_t;
-    Geometry g;
+    Geometry &g = p->g;
     g.B = static_cast<int>(B);
     g.T = static_cast<int>(T);
     g.C = static_cast<int>(C);
     g.n_cg = static_cast<int>((C + CG - 1) / CG);
-    g.n_seg = static_cast<int>((T + LT - 1) / LT);
+    g.n_seg = static_cast<int>((T + lt - 1) / lt);
     const long long tiles_per_seg = B * static_cast<long long>(g.n_cg);
     const long long tiles = tiles_per_seg * g.n_seg;
     if (tiles > INT32_MAX) return fail(WKV_ERR_INVALID_ARG, "problem has too many tiles");
     g.tiles_per_seg = static_cast<int>(tiles_per_seg);
     g.tiles = static_cast<int>(tiles);
     g.spin_limit = kSpinLimit;
-
-    CUtensorMap maps[3];
-    std::memset(maps, 0, sizeof maps);
-    const void *ptrs[3] = {args.x0, args.x1, args.y};
-    g.use_tma = tma_eligible(ptrs, 3, sizeof(io_t), T, C) ? 1 : 0;
-    if (g.use_tma) {
+    std::memset(p->maps, 0, sizeof p->maps);
+    g.use_tma = 0;
+    if (want_tma) {
+        const void *ptrs[3] = {args.x0, args.x1, args.y};
+        g.use_tma = tma_eligible(ptrs, 3, sizeof(io_t), T, C) ? 1 : 0;
         for (int i = 0; i < 3 && g.use_tma; ++i)
-            if (!make_map(&maps[i], ptrs[i], dt, sizeof(io_t), B, T, C, CG, LT)) g.use_tma = 0;
+            if (!make_map(&p->maps[i], ptrs[i], dt, sizeof(io_t), B, T, C, CG, lt)) g.use_tma = 0;
     }
-
-    constexpr size_t smem = chunked_scan_smem_bytes<Op, LT, NW>();
-    auto kern = chunked_scan_kernel<Op, LT, NW>;
-    static std::atomic<uint64_t> configured{0};  // one bit per device
-    if (dev < 64 && !(configured.load() & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        configured.fetch_or(1ull << dev);
-    }
-
-    Workspace ws;
-    std::memset(&ws, 0, sizeof ws);
+    std::memset(&p->ws, 0, sizeof p->ws);
     if (g.n_seg > 1) {
         std::lock_guard<std::mutex> lk(g_mu);
         const WsLayout l = ws_layout(static_cast<size_t>(tiles), Op::NV * CG);
         WsEntry *e = nullptr;
         wkv_status st = ensure_ws(dev, stream, l.total, &e);
         if (st != WKV_OK) return st;
+        Workspace &ws = p->ws;
         ws.ticket = reinterpret_cast<unsigned int *>(e->base);
         ws.done = reinterpret_cast<unsigned int *>(e->base + 4);
         ws.epoch = reinterpret_cast<unsigned long long *>(e->base + 8);
@@ -288,9 +296,58 @@ wkv_status launch_tiles(const typename Op::Args &args, int64_t B, int64_t T, int
         ws.agg = reinterpret_cast<float *>(e->base + l.agg);
         ws.incl = reinterpret_cast<float *>(e->base + l.incl);
     }
+    return WKV_OK;
+}
+
+template <typename K>
+wkv_status configure_once(K kern, size_t smem, int dev, std::atomic<uint64_t> &done) {
+    if (dev < 64 && (done.load() & (1ull << dev))) return WKV_OK;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    if (dev < 64) done.fetch_or(1ull << dev);
+    return WKV_OK;
+}
+
+// one thread block per tile; any shape (element-wise copies when no tensor map)
+template <class Op, int LT, int NW>
+wkv_status launch_chunked(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
+                          CUtensorMapDataType dt, cudaStream_t stream, int dev) {
+    Plan p;
+    wkv_status st = make_plan<Op>(args, B, T, C, LT, dt, stream, dev, true, &p);
+    if (st != WKV_OK) return st;
+    constexpr size_t smem = chunked_scan_smem_bytes<Op, LT, NW>();
+    auto kern = chunked_scan_kernel<Op, LT, NW>;
+    static std::atomic<uint64_t> configured{0};
+    if ((st = configure_once(kern, smem, dev, configured)) != WKV_OK) return st;
     cudaGetLastError();  // clear a stale error so the check below is about this launch
-    kern<<<static_cast<unsigned>(tiles), NW * 32, smem, stream>>>(maps[0], maps[1], maps[2], args,
-                                                                 g, ws);
+    kern<<<static_cast<unsigned>(p.g.tiles), NW * 32, smem, stream>>>(p.maps[0], p.maps[1],
+                                                                       p.maps[2], args, p.g, p.ws);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
+// persistent pipeline, one block per SM; shapes a tensor map describes
+template <class Op, int LT, int NWG, int NC, int NSTAGE>
+wkv_status launch_persistent(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
+                             CUtensorMapDataType dt, cudaStream_t stream, int dev) {
+    using Cfg = PersistentCfg<Op, LT, NWG, NC, NSTAGE>;
+    Plan p;
+    wkv_status st = make_plan<Op>(args, B, T, C, LT, dt, stream, dev, true, &p);
+    if (st != WKV_OK) return st;
+    if (!p.g.use_tma)  // a tensor map could not be made after all
+        return launch_chunked<Op, LT, 8>(args, B, T, C, dt, stream, dev);
+    auto kern = persistent_scan_kernel<Op, LT, NWG, NC, NSTAGE>;
+    static std::atomic<uint64_t> configured{0};
+    if ((st = configure_once(kern, Cfg::kSmemBytes, dev, configured)) != WKV_OK) return st;
+    const int grid = std::min(p.g.tiles, sm_count(dev));
+    cudaGetLastError();
+    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(
+        p.maps[0], p.maps[1], p.maps[2], args, p.g, p.ws);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     return WKV_OK;
@@ -299,12 +356,20 @@ wkv_status launch_tiles(const typename Op::Args &args, int64_t B, int64_t T, int
 template <class Op>
 wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
                     CUtensorMapDataType dt, cudaStream_t stream, int dev) {
+    const void *ptrs[3] = {args.x0, args.x1, args.y};
+    const bool tma = tma_eligible(ptrs, 3, sizeof(typename Op::io_t), T, C);
     switch (g_tile_steps.load()) {
-        case 8: return launch_tiles<Op, 8, 8>(args, B, T, C, dt, stream, dev);
-        case 32: return launch_tiles<Op, 32, 8>(args, B, T, C, dt, stream, dev);
-        case 64: return launch_tiles<Op, 64, 8>(args, B, T, C, dt, stream, dev);
-        case 128: return launch_tiles<Op, 128, 8>(args, B, T, C, dt, stream, dev);
-        default: return launch_tiles<Op, 256, 8>(args, B, T, C, dt, stream, dev);
+        case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
+        case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
+        case 64:
+            return tma ? launch_persistent<Op, 64, 4, 2, 6>(args, B, T, C, dt, stream, dev)
+                       : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
+        case 256:
+            return tma ? launch_persistent<Op, 256, 8, 1, 3>(args, B, T, C, dt, stream, dev)
+                       : launch_chunked<Op, 256, 8>(args, B, T, C, dt, stream, dev);
+        default:
+            return tma ? launch_persistent<Op, 128, 4, 2, 6>(args, B, T, C, dt, stream, dev)
+                       : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
     }
 }
 

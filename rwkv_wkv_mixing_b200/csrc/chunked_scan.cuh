@@ -33,118 +33,9 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "scan_common.cuh"
 
 namespace wkvb {
-
-constexpr uint32_t kFlagAgg = 1u;   // tile aggregate published
-constexpr uint32_t kFlagIncl = 2u;  // state after the tile published
-constexpr int kStatusTimeout = 4;   // == WKV_ERR_TIMEOUT
-
-// Device pointers of one look-back workspace.  The three counters live in
-// the workspace itself, so a launch needs no per-launch host state (CUDA-graph
-// replays stay correct): blocks take tile tickets from `ticket`; the last
-// block to finish resets `ticket` and `done` and advances `epoch`, which tags
-// every flag this launch publishes so flags left by earlier launches never
-// read as ready.  Launches sharing a workspace must run one after another
-// (same stream).
-struct Workspace {
-    unsigned int *ticket;        // next tile ticket of the running launch
-    unsigned int *done;          // blocks of the running launch that finished
-    unsigned long long *epoch;   // launches completed on this workspace
-    int *status;                 // device status word, 0 or an error code
-    unsigned long long *flags;   // [tiles] (epoch << 2) | kFlag*
-    float *agg;                  // [tiles][NV][CG] tile aggregates
-    float *incl;                 // [tiles][NV][CG] states after each tile
-};
-
-struct Geometry {
-    int B, T, C;           // batch rows, steps, channels
-    int n_cg;              // channel groups per row, ceil(C / CG)
-    int n_seg;             // time segments per row, ceil(T / LT)
-    int tiles_per_seg;     // B * n_cg
-    int tiles;             // n_seg * tiles_per_seg == gridDim.x
-    int use_tma;           // 1: TMA tile copies; 0: element-wise copies
-    long long spin_limit;  // polls of a predecessor's flag before giving up
-};
-
-// ---- vector access to CPT consecutive channels in shared memory -----------
-template <typename io_t, int CPT>
-struct Vec;
-
-template <>
-struct Vec<float, 1> {
-    __device__ __forceinline__ static void load(const float *p, float (&x)[1]) { x[0] = *p; }
-    __device__ __forceinline__ static void store(float *p, const float (&x)[1]) { *p = x[0]; }
-};
-
-template <>
-struct Vec<float, 2> {
-    __device__ __forceinline__ static void load(const float *p, float (&x)[2]) {
-        float2 t = *reinterpret_cast<const float2 *>(p);
-        x[0] = t.x;
-        x[1] = t.y;
-    }
-    __device__ __forceinline__ static void store(float *p, const float (&x)[2]) {
-        *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
-    }
-};
-
-template <>
-struct Vec<__nv_bfloat16, 2> {
-    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&x)[2]) {
-        float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
-        x[0] = t.x;
-        x[1] = t.y;
-    }
-    // round to nearest even
-    __device__ __forceinline__ static void store(__nv_bfloat16 *p, const float (&x)[2]) {
-        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(x[0], x[1]);
-    }
-};
-
-template <typename io_t>
-__device__ __forceinline__ io_t io_zero();
-template <>
-__device__ __forceinline__ float io_zero<float>() { return 0.f; }
-template <>
-__device__ __forceinline__ __nv_bfloat16 io_zero<__nv_bfloat16>() {
-    return __float2bfloat16_rn(0.f);
-}
-
-// ---- publishing a per-tile value for the look-back -------------------------
-template <class Op, int CG>
-__device__ __forceinline__ void publish(float *base, unsigned long long *flags, int tile,
-                                        const typename Op::State (&val)[Op::CPT],
-                                        unsigned long long flag, int lane) {
-    float *dst = base + static_cast<size_t>(tile) * Op::NV * CG;
-#pragma unroll
-    for (int j = 0; j < Op::CPT; ++j)
-#pragma unroll
-        for (int q = 0; q < Op::NV; ++q)
-            st_relaxed_gpu(dst + q * CG + lane * Op::CPT + j, Op::get(val[j], q));
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release_gpu_u64(flags + tile, flag);
-}
-
-// Count this block as finished; the last block of the launch resets the
-// ticket counter and advances the epoch for the next launch.  Every block
-// has taken its ticket and finished all look-back reads by this point.
-__device__ __forceinline__ void finish_launch(const Workspace &ws, const Geometry &g,
-                                              bool chained, int tid) {
-    if (!chained) return;
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        const unsigned int prev = atomicAdd(ws.done, 1u);
-        if (prev == static_cast<unsigned int>(g.tiles) - 1u) {
-            atomicExch(ws.ticket, 0u);
-            atomicExch(ws.done, 0u);
-            atomicAdd(ws.epoch, 1ull);
-            __threadfence();
-        }
-    }
-}
 
 template <class Op, int LT, int NW>
 constexpr size_t chunked_scan_smem_bytes() {
@@ -153,7 +44,7 @@ constexpr size_t chunked_scan_smem_bytes() {
 }
 
 template <class Op, int LT, int NW>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, 3)
     chunked_scan_kernel(const __grid_constant__ CUtensorMap map_x0,
                         const __grid_constant__ CUtensorMap map_x1,
                         const __grid_constant__ CUtensorMap map_y,
@@ -201,7 +92,7 @@ __global__ void __launch_bounds__(NW * 32)
     __syncthreads();
     const int tile = s_tile;
     if (tile < 0) {
-        finish_launch(ws, g, chained, tid);
+        finish_launch(ws, chained, tid, static_cast<unsigned>(g.tiles));
         return;
     }
     const unsigned long long epoch = s_epoch;
@@ -251,30 +142,12 @@ __global__ void __launch_bounds__(NW * 32)
     // ---- pass 1: summary of this warp's sub-chunk ---------------------------
     const int s0 = warp * LS;
     const int nval = max(0, min(LS, g.T - (t0 + s0)));
-    const io_t *p0 = s_x0 + s0 * CG + lane * CPT;
+    io_t *p0 = s_x0 + s0 * CG + lane * CPT;
     const io_t *p1 = s_x1 + s0 * CG + lane * CPT;
+    typename Op::Scratch sc[CPT];
     {
         State st[CPT];
-#pragma unroll
-        for (int j = 0; j < CPT; ++j) st[j] = Op::identity();
-        if (nval == LS) {
-#pragma unroll 8
-            for (int i = 0; i < LS; ++i) {
-                float x0[CPT], x1[CPT];
-                Vec<io_t, CPT>::load(p0 + i * CG, x0);
-                Vec<io_t, CPT>::load(p1 + i * CG, x1);
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) Op::step1(st[j], x0[j], x1[j], prm[j]);
-            }
-        } else {
-            for (int i = 0; i < nval; ++i) {
-                float x0[CPT], x1[CPT];
-                Vec<io_t, CPT>::load(p0 + i * CG, x0);
-                Vec<io_t, CPT>::load(p1 + i * CG, x1);
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) Op::step1(st[j], x0[j], x1[j], prm[j]);
-            }
-        }
+        Op::template summarize<LS>(p0, p1, nval, prm, st, sc);
 #pragma unroll
         for (int j = 0; j < CPT; ++j)
 #pragma unroll
@@ -311,52 +184,7 @@ __global__ void __launch_bounds__(NW * 32)
                     publish<Op, CG>(ws.agg, ws.flags, tile, agg, (epoch << 2) | kFlagAgg, lane);
                 // decoupled look-back over the tiles before this one in time
                 State run[CPT];
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) run[j] = Op::identity();
-                float run_len = 0.f;
-                int pred = tile - g.tiles_per_seg;
-                bool failed = false;
-                while (true) {
-                    unsigned long long f = 0;
-                    if (lane == 0) {
-                        long long n = 0;
-                        while (true) {
-                            f = ld_acquire_gpu_u64(ws.flags + pred);
-                            if ((f >> 2) == epoch && (f & 3u) != 0u) break;
-                            if (++n > g.spin_limit) {
-                                f = 0;
-                                break;
-                            }
-                            __nanosleep(64);
-                        }
-                    }
-                    f = __shfl_sync(0xffffffffu, f, 0);
-                    if (f == 0) {
-                        failed = true;
-                        break;
-                    }
-                    // each lane acquires the flag itself before reading the data
-                    (void)ld_acquire_gpu_u64(ws.flags + pred);
-                    const bool inc = (f & 3u) == kFlagIncl;
-                    const float *src =
-                        (inc ? ws.incl : ws.agg) + static_cast<size_t>(pred) * NV * CG;
-#pragma unroll
-                    for (int j = 0; j < CPT; ++j) {
-                        float vals[NV];
-#pragma unroll
-                        for (int q = 0; q < NV; ++q)
-                            vals[q] = ld_relaxed_gpu(src + q * CG + lane * CPT + j);
-                        run[j] = Op::combine(Op::make(vals), run[j], run_len, prm[j]);
-                    }
-                    if (inc) break;
-                    run_len += static_cast<float>(LT);
-                    pred -= g.tiles_per_seg;
-                    if (pred < 0) {  // cannot happen: every first-segment tile publishes
-                        failed = true;
-                        break;
-                    }
-                }
-                if (failed) {
+                if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run)) {
                     if (lane == 0) atomicExch(ws.status, kStatusTimeout);
 #pragma unroll
                     for (int j = 0; j < CPT; ++j) run[j] = Op::nan_state();
@@ -395,27 +223,7 @@ __global__ void __launch_bounds__(NW * 32)
                 cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(LS), prm[j]);
             }
         }
-        io_t *q0 = s_x0 + s0 * CG + lane * CPT;
-        if (nval == LS) {
-#pragma unroll 8
-            for (int i = 0; i < LS; ++i) {
-                float x0[CPT], x1[CPT], y[CPT];
-                Vec<io_t, CPT>::load(p0 + i * CG, x0);
-                Vec<io_t, CPT>::load(p1 + i * CG, x1);
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) y[j] = Op::step2(cur[j], x0[j], x1[j], prm[j]);
-                Vec<io_t, CPT>::store(q0 + i * CG, y);
-            }
-        } else {
-            for (int i = 0; i < nval; ++i) {
-                float x0[CPT], x1[CPT], y[CPT];
-                Vec<io_t, CPT>::load(p0 + i * CG, x0);
-                Vec<io_t, CPT>::load(p1 + i * CG, x1);
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) y[j] = Op::step2(cur[j], x0[j], x1[j], prm[j]);
-                Vec<io_t, CPT>::store(q0 + i * CG, y);
-            }
-        }
+        Op::template sweep<LS>(cur, p0, p1, nval, prm, sc);
     }
 
     // ---- write the output tile ----------------------------------------------
@@ -436,7 +244,7 @@ __global__ void __launch_bounds__(NW * 32)
                 args.y[(static_cast<size_t>(b) * g.T + t) * g.C + c] = s_x0[i];
         }
     }
-    finish_launch(ws, g, chained, tid);
+    finish_launch(ws, chained, tid, static_cast<unsigned>(g.tiles));
 }
 
 }  // namespace wkvb

@@ -1,0 +1,307 @@
+// Persistent, warp-specialised chunked scan for sm_100a (shapes a TMA tensor
+// map can describe).
+//
+// One thread block per SM stays resident for the whole launch.  Warp 0 is the
+// producer: one lane takes tile tickets and streams each tile's two input
+// tensors (LT steps x CG channels) into a ring of NSTAGE shared-memory stages
+// with TMA tile loads, each stage guarded by a "full" and an "empty" mbarrier.
+// The remaining warps form NC consumer groups of NWG warps; group g handles
+// ring iterations g, g+NC, g+2NC, ...  For each tile a group runs the same
+// two passes and look-back as chunked_scan_kernel -- pass 1 summaries per
+// warp, the carry into the tile (aggregate, decoupled look-back, publication)
+// by the group's first warp, pass 2 writing outputs over the stage's first
+// tensor -- then one thread issues the TMA store of the outputs and releases
+// the stage of the group's previous tile once that tile's store has read it.
+//
+// So HBM sees every element once, loads for the next tiles are always in
+// flight while tiles are being computed, and no thread block is launched per
+// tile.  Every wait is bounded (global-timer deadline on mbarriers, poll
+// budget in the look-back); a wait that gives up records WKV_ERR_TIMEOUT in
+// the status word and makes every loop of the block finish.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "scan_common.cuh"
+
+namespace wkvb {
+
+constexpr unsigned long long kBarrierWaitNs = 4000000000ull;  // 4 s
+
+template <class Op, int LT, int NWG, int NC, int NSTAGE>
+struct PersistentCfg {
+    static constexpr int CPT = Op::CPT, NV = Op::NV, CG = 32 * CPT, LS = LT / NWG;
+    static constexpr int kThreads = (1 + NC * NWG) * 32;
+    static constexpr size_t kTileElems = static_cast<size_t>(LT) * CG;
+    static constexpr size_t kStageBytes = 2 * kTileElems * sizeof(typename Op::io_t);
+    static constexpr size_t kSmemBytes =
+        NSTAGE * kStageBytes + static_cast<size_t>(NC) * (NWG + 1) * NV * CG * sizeof(float);
+    static_assert(LT % NWG == 0, "tile length must split evenly over a group's warps");
+    static_assert(LT <= 256, "TMA box rows are limited to 256");
+    static_assert(NSTAGE >= 2 * NC, "each group may hold two stages");
+    static_assert(1 + NC <= 16, "named barrier ids");
+};
+
+// Wait for phase `parity` of `bar`; false if the block is aborting or the
+// deadline passed (which starts the abort).
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                           const Workspace &ws) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    for (unsigned n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kBarrierWaitNs) {
+                *abort_flag = 1;
+                if (ws.status != nullptr) atomicExch(ws.status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+template <class Op, int LT, int NWG, int NC, int NSTAGE>
+__global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThreads, 1)
+    persistent_scan_kernel(const __grid_constant__ CUtensorMap map_x0,
+                           const __grid_constant__ CUtensorMap map_x1,
+                           const __grid_constant__ CUtensorMap map_y,
+                           const typename Op::Args args, const Geometry g, const Workspace ws) {
+    using Cfg = PersistentCfg<Op, LT, NWG, NC, NSTAGE>;
+    using io_t = typename Op::io_t;
+    using State = typename Op::State;
+    using Param = typename Op::Param;
+    constexpr int CPT = Cfg::CPT, NV = Cfg::NV, CG = Cfg::CG, LS = Cfg::LS;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    io_t *s_stage = reinterpret_cast<io_t *>(smem);  // [NSTAGE][2][LT][CG]
+    float *s_sum = reinterpret_cast<float *>(smem + NSTAGE * Cfg::kStageBytes);  // [NC][NWG][NV][CG]
+    float *s_carry = s_sum + NC * NWG * NV * CG;                                   // [NC][NV][CG]
+    __shared__ __align__(8) uint64_t full_bar[NSTAGE];
+    __shared__ __align__(8) uint64_t empty_bar[NSTAGE];
+    __shared__ int s_meta[NSTAGE];      // tile id per stage, -1 = no more tiles
+    __shared__ int s_last_it[NSTAGE];   // last ring iteration loaded into each stage
+    __shared__ int s_gtile[NC];         // each group's current tile, as its leader saw it
+    __shared__ unsigned long long s_epoch;
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool chained = g.n_seg > 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+            s_last_it[s] = -1;
+        }
+        fence_mbar_init();
+        s_epoch = chained ? ld_relaxed_gpu_u64(ws.epoch) : 0ull;
+        s_abort = 0;
+    }
+    __syncthreads();
+    const unsigned long long epoch = s_epoch;
+    volatile int *abort_flag = &s_abort;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            prefetch_tensormap(&map_x0);
+            prefetch_tensormap(&map_x1);
+            prefetch_tensormap(&map_y);
+            int sentinels = 0;
+            int next_static = static_cast<int>(blockIdx.x);
+            for (int it = 0; sentinels < NC; ++it) {
+                const int s = it % NSTAGE;
+                if (!wait_phase(&empty_bar[s], ((it / NSTAGE) & 1) ^ 1, abort_flag, ws)) break;
+                int tile = -1;
+                if (sentinels == 0) {
+                    if (chained) {
+                        // tickets go out in the order blocks ask for them, so a
+                        // tile only ever waits for tiles already being worked on
+                        const unsigned t = atomicAdd(ws.ticket, 1u);
+                        tile = t < static_cast<unsigned>(g.tiles) ? static_cast<int>(t) : -1;
+                    } else {
+                        tile = next_static < g.tiles ? next_static : -1;
+                        next_static += static_cast<int>(gridDim.x);
+                    }
+                }
+                s_meta[s] = tile;
+                if (tile < 0) {
+                    ++sentinels;
+                    mbar_arrive(&full_bar[s]);
+                } else {
+                    const int seg = tile / g.tiles_per_seg;
+                    const int rem = tile - seg * g.tiles_per_seg;
+                    const int b = rem / g.n_cg;
+                    const int c0 = (rem - b * g.n_cg) * CG;
+                    io_t *dst = s_stage + static_cast<size_t>(s) * 2 * Cfg::kTileElems;
+                    s_last_it[s] = it;
+                    mbar_arrive_expect_tx(&full_bar[s], static_cast<uint32_t>(Cfg::kStageBytes));
+                    tma_load_3d(dst, &map_x0, &full_bar[s], c0, seg * LT, b);
+                    tma_load_3d(dst + Cfg::kTileElems, &map_x1, &full_bar[s], c0, seg * LT, b);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- consumer group ----------------
+        const int cw = warp - 1;
+        const int grp = cw / NWG, wg = cw - grp * NWG;
+        const int gtid = wg * 32 + lane;
+        const int bar_id = 1 + grp;
+        float *g_sum = s_sum + grp * NWG * NV * CG;
+        float *g_carry = s_carry + grp * NV * CG;
+        int prev_s = -1;
+        for (int it = grp;; it += NC) {
+            const int s = it % NSTAGE;
+            const uint32_t parity = (it / NSTAGE) & 1;
+            // the group leader alone decides whether the stage arrived, so the
+            // whole group leaves (or stays in) the loop together
+            if (gtid == 0)
+                s_gtile[grp] = wait_phase(&full_bar[s], parity, abort_flag, ws) ? s_meta[s] : -2;
+            named_bar_sync(bar_id, NWG * 32);
+            const int tile = s_gtile[grp];
+            if (tile < 0) break;
+            // the phase has completed; observing it makes the TMA writes visible
+            // to this thread (the stage cannot be refilled before this group
+            // releases it, so the phase stays complete)
+            for (int n = 0; n < (1 << 20) && !mbar_try_wait(&full_bar[s], parity); ++n) {
+            }
+            const int seg = tile / g.tiles_per_seg;
+            const int rem = tile - seg * g.tiles_per_seg;
+            const int b = rem / g.n_cg;
+            const int t0 = seg * LT;
+            const int c0 = (rem - b * g.n_cg) * CG;
+            io_t *s_x0 = s_stage + static_cast<size_t>(s) * 2 * Cfg::kTileElems;
+            const io_t *s_x1 = s_x0 + Cfg::kTileElems;
+
+            Param prm[CPT];
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) prm[j] = Op::param(args, c0 + lane * CPT + j, g.C);
+
+            // pass 1
+            const int s0 = wg * LS;
+            const int nval = max(0, min(LS, g.T - (t0 + s0)));
+            io_t *p0 = s_x0 + s0 * CG + lane * CPT;
+            const io_t *p1 = s_x1 + s0 * CG + lane * CPT;
+            typename Op::Scratch sc[CPT];
+            {
+                State st[CPT];
+                Op::template summarize<LS>(p0, p1, nval, prm, st, sc);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j)
+#pragma unroll
+                    for (int q = 0; q < NV; ++q)
+                        g_sum[(wg * NV + q) * CG + lane * CPT + j] = Op::get(st[j], q);
+            }
+            named_bar_sync(bar_id, NWG * 32);
+
+            // carry into the tile (the group's first warp)
+            if (wg == 0) {
+                State agg[CPT], X[CPT];
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    agg[j] = Op::identity();
+                    for (int w = 0; w < NWG; ++w) {
+                        float vals[NV];
+#pragma unroll
+                        for (int q = 0; q < NV; ++q) vals[q] = g_sum[(w * NV + q) * CG + lane * CPT + j];
+                        const int len = max(0, min(LS, g.T - (t0 + w * LS)));
+                        agg[j] = Op::combine(agg[j], Op::make(vals), static_cast<float>(len), prm[j]);
+                    }
+                    X[j] = Op::carry0(args, b, c0 + lane * CPT + j, g.C);
+                }
+                if (chained) {
+                    const bool last = seg == g.n_seg - 1;
+                    if (seg == 0) {
+                        State inc[CPT];
+#pragma unroll
+                        for (int j = 0; j < CPT; ++j)
+                            inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
+                        publish<Op, CG>(ws.incl, ws.flags, tile, inc, (epoch << 2) | kFlagIncl, lane);
+                    } else {
+                        if (!last)
+                            publish<Op, CG>(ws.agg, ws.flags, tile, agg, (epoch << 2) | kFlagAgg, lane);
+                        State run[CPT];
+                        if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run)) {
+                            if (lane == 0) atomicExch(ws.status, kStatusTimeout);
+#pragma unroll
+                            for (int j = 0; j < CPT; ++j) run[j] = Op::nan_state();
+                        }
+#pragma unroll
+                        for (int j = 0; j < CPT; ++j) X[j] = run[j];
+                        if (!last) {
+                            State inc[CPT];
+#pragma unroll
+                            for (int j = 0; j < CPT; ++j)
+                                inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
+                            publish<Op, CG>(ws.incl, ws.flags, tile, inc, (epoch << 2) | kFlagIncl,
+                                            lane);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < CPT; ++j)
+#pragma unroll
+                    for (int q = 0; q < NV; ++q) g_carry[q * CG + lane * CPT + j] = Op::get(X[j], q);
+            }
+            named_bar_sync(bar_id, NWG * 32);
+
+            // pass 2
+            if (nval > 0) {
+                State cur[CPT];
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    float vals[NV];
+#pragma unroll
+                    for (int q = 0; q < NV; ++q) vals[q] = g_carry[q * CG + lane * CPT + j];
+                    cur[j] = Op::make(vals);
+                    for (int w = 0; w < wg; ++w) {  // earlier sub-chunks are all full
+#pragma unroll
+                        for (int q = 0; q < NV; ++q) vals[q] = g_sum[(w * NV + q) * CG + lane * CPT + j];
+                        cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(LS), prm[j]);
+                    }
+                }
+                Op::template sweep<LS>(cur, p0, p1, nval, prm, sc);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(bar_id, NWG * 32);
+
+            // store the outputs; release the previous tile's stage once its
+            // store has read it
+            if (gtid == 0) {
+                tma_store_3d(&map_y, s_x0, c0, t0, b);
+                bulk_commit();
+                if (prev_s >= 0) {
+                    bulk_wait_read_all_but_one();
+                    mbar_arrive(&empty_bar[prev_s]);
+                }
+                prev_s = s;
+            }
+        }
+        if (gtid == 0 && prev_s >= 0) {
+            bulk_wait_read_all();
+            mbar_arrive(&empty_bar[prev_s]);
+        }
+        __syncwarp();
+    }
+
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) {
+        // an aborted block must not exit with tile loads still landing in its
+        // shared memory: wait (bounded) for the last load of every stage
+        for (int s = 0; s < NSTAGE; ++s) {
+            const int it = s_last_it[s];
+            if (it < 0) continue;
+            const unsigned long long t0 = global_timer_ns();
+            while (!mbar_try_wait(&full_bar[s], (it / NSTAGE) & 1)) {
+                if (global_timer_ns() - t0 > kBarrierWaitNs) break;
+            }
+        }
+    }
+    finish_launch(ws, chained, static_cast<int>(threadIdx.x), gridDim.x);
+}
+
+}  // namespace wkvb

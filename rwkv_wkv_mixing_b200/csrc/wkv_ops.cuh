@@ -1,43 +1,101 @@
 // Op policies for chunked_scan_kernel: the RWKV-4 WKV operator and the
 // per-channel diagonal linear scan.
+//
+// An Op supplies, for the CPT channels one thread owns:
+//   summarize(p0, p1, n, ...)  pass 1: the summary of an n-step sub-chunk
+//                              (rows p0[i*CG], p1[i*CG]) from the empty state
+//   sweep(carry, ...)          pass 2: outputs of the sub-chunk from the state
+//                              before it, written over p0's rows
+//   combine(l, r, r_len)       the state l followed by a chunk of r_len steps
+//                              whose summary is r
 #pragma once
 
 #include <cuda_bf16.h>
 
-#include "chunked_scan.cuh"
 #include "ptx.cuh"
 
 namespace wkvb {
 
 constexpr float kLog2e = 1.4426950408889634f;
-// log2-scale of "no tokens yet"; finite so that differences of two sentinels
-// stay finite, and 2^(sentinel - anything real) flushes to zero
+// log-scale of "no tokens yet": finite, so differences of two such values
+// stay finite, and e^(kNoScale - anything real) is exactly zero
 constexpr float kNoScale = -1e30f;
 
+// ---- shared-memory access to CPT consecutive channels ---------------------
+template <typename io_t, int CPT>
+struct Vec;
+
+template <>
+struct Vec<float, 1> {
+    __device__ __forceinline__ static void load(const float *p, float (&x)[1]) { x[0] = *p; }
+    __device__ __forceinline__ static void store(float *p, const float (&x)[1]) { *p = x[0]; }
+};
+
+template <>
+struct Vec<float, 2> {
+    __device__ __forceinline__ static void load(const float *p, float (&x)[2]) {
+        float2 t = *reinterpret_cast<const float2 *>(p);
+        x[0] = t.x;
+        x[1] = t.y;
+    }
+    __device__ __forceinline__ static void store(float *p, const float (&x)[2]) {
+        *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+    }
+};
+
+template <>
+struct Vec<__nv_bfloat16, 2> {
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&x)[2]) {
+        float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+        x[0] = t.x;
+        x[1] = t.y;
+    }
+    // round to nearest even
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, const float (&x)[2]) {
+        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(x[0], x[1]);
+    }
+};
+
+// The output (a + e v) / (b + e) written as v + (a - b v) / (b + e): the same
+// quotient, but exact whenever the past does not move the answer -- an empty
+// past (a = b = 0, so y_0 = v_0 bit for bit) or a constant power-of-two v
+// (a = v b exactly) -- and the approximate reciprocal only perturbs the
+// correction term, whose size is |y - v|.
+__device__ __forceinline__ float wkv_output(float a, float b, float e, float v) {
+    return v + fmaf(-b, v, a) * rcp_approx(b + e);
+}
+
 // ---------------------------------------------------------------------------
-// WKV, eq. (14) of "RWKV：基于RNN的LLM" (section 二.1, Time-mixing block).
+// WKV, eq. (14) of "RWKV：基于RNN的LLM" (section 二.1, Time-mixing block):
+//   y_t = (num_t + e^{u + k_t} v_t) / (den_t + e^{u + k_t}),
+//   num_t = sum_{i<t} e^{-(t-1-i) w + k_i} v_i,  den_t = same without v_i.
 //
-// State before step t: the past sums
-//   num_t = sum_{i<t} e^{-(t-1-i) w + k_i} v_i,  den_t = sum_{i<t} e^{-(t-1-i) w + k_i},
-// kept as (a, b, p) with (num, den) = (a, b) * 2^p.  All exponents are in
-// log2 units (k, u, w pre-multiplied by log2 e), and p is the largest exponent
-// folded in so far, so every 2^x evaluated has x <= 0 and b >= 1 once a token
-// has been added.  Outputs:
-//   y_t = (num_t + e^{u + k_t} v_t) / (den_t + e^{u + k_t});
-// state update:
-//   (num, den)_{t+1} = e^{-w} (num, den)_t + e^{k_t} (v_t, 1).
-// A chunk of L steps maps a state S to e^{-L w} S + (chunk summary), which is
-// `combine`.
+// State: (a, b, p) with (num, den) = (a, b) * e^p, p in natural-log units.
+// Stepping the state: (num, den)_{t+1} = e^{-w} (num, den)_t + e^{k_t} (v_t, 1).
+//
+// Pass 1 (summary of a sub-chunk ending at step `end`, from the empty state):
+// p = m = max_i (k_i - (end-i) w), then a = sum_i e^{k_i - (end-i) w - m} v_i,
+// b = the same without v_i: every exponent is <= 0 and the largest term is 1.
+//
+// Pass 2 (outputs of a sub-chunk from the state before it): one reference
+// M = max(p_in, max_i k_i) for the whole sub-chunk, state scaled to e^M, so
+// each step is  e = e^{k_t - M} (<= 1),  y = (a + e U v) / (b + e U),
+// a <- a D + e v,  b <- b D + e  with per-channel constants U = e^u,
+// D = e^{-w}.  The loop-carried dependency is one FMA.  This is exact
+// arithmetic reordered; it is used when a bound shows every denominator stays
+// above 2^-100 (so nothing that matters is flushed to zero) and U is below
+// 2^64.  Otherwise the sub-chunk takes the per-step max-stabilised update,
+// whose every exponent is <= 0 for any finite input.
 // ---------------------------------------------------------------------------
 template <typename IO, int CPT_>
 struct WkvOp {
     using io_t = IO;
     static constexpr int CPT = CPT_;
+    static constexpr int CG = 32 * CPT;
     static constexpr int NV = 3;
-    static constexpr bool kExactDiv = sizeof(IO) == 4;
     struct Param {
-        float uu;  // u * log2 e
-        float ww;  // w * log2 e
+        float u, w;  // bonus and decay (natural units)
+        float U, D;  // e^u, e^{-w}
     };
     struct State {
         float a, b, p;
@@ -48,12 +106,18 @@ struct WkvOp {
         IO *y;         // y [B, T, C]
         const float *w, *u;  // [C]
     };
+    // per-thread facts pass 1 leaves for pass 2 of the same sub-chunk
+    struct Scratch {
+        float kmax, kmin;
+    };
 
     __device__ __forceinline__ static Param param(const Args &args, int c, int C) {
-        Param q{0.f, 0.f};
+        Param q{0.f, 0.f, 1.f, 1.f};
         if (c < C) {
-            q.uu = args.u[c] * kLog2e;
-            q.ww = args.w[c] * kLog2e;
+            q.u = args.u[c];
+            q.w = args.w[c];
+            q.U = expf(q.u);
+            q.D = expf(-q.w);
         }
         return q;
     }
@@ -70,54 +134,175 @@ struct WkvOp {
     }
     __device__ __forceinline__ static State make(const float (&v)[NV]) { return {v[0], v[1], v[2]}; }
 
-    // state l, then a chunk whose summary is r and whose length is r_len steps
     __device__ __forceinline__ static State combine(const State &l, const State &r, float r_len,
                                                     const Param &q) {
-        const float pd = l.p - r_len * q.ww;
+        const float pd = fmaf(-r_len, q.w, l.p);
         const float m = fmaxf(pd, r.p);
-        const float fl = ex2_approx(pd - m), fr = ex2_approx(r.p - m);
+        const float fl = expf(pd - m), fr = expf(r.p - m);
         return {fmaf(l.a, fl, r.a * fr), fmaf(l.b, fl, r.b * fr), m};
     }
 
-    // state update with token (k, v)
-    __device__ __forceinline__ static void step1(State &s, float k, float v, const Param &q) {
-        const float kk = k * kLog2e;
-        const float pd = s.p - q.ww;
-        const float d = pd - kk;
-        const float e = ex2_approx(-fabsf(d));
-        const bool old_wins = d >= 0.f;
-        const float fo = old_wins ? 1.f : e, fn = old_wins ? e : 1.f;
-        s.a = fmaf(s.a, fo, fn * v);
-        s.b = fmaf(s.b, fo, fn);
-        s.p = fmaxf(pd, kk);
+    // ---- pass 1 ------------------------------------------------------------
+    template <int LS>
+    __device__ __forceinline__ static void summarize(const IO *p0, const IO *p1, int n,
+                                                     const Param (&q)[CPT], State (&out)[CPT],
+                                                     Scratch (&sc)[CPT]) {
+        float m[CPT], kx[CPT], kn[CPT], a[CPT], b[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            m[j] = kNoScale;
+            kx[j] = kNoScale;
+            kn[j] = -kNoScale;
+            a[j] = 0.f;
+            b[j] = 0.f;
+        }
+        if (n == LS) {
+#pragma unroll 8
+            for (int i = 0; i < LS; ++i) {
+                float k[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, k);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    m[j] = fmaxf(m[j], fmaf(static_cast<float>(i - (LS - 1)), q[j].w, k[j]));
+                    kx[j] = fmaxf(kx[j], k[j]);
+                    kn[j] = fminf(kn[j], k[j]);
+                }
+            }
+#pragma unroll 8
+            for (int i = 0; i < LS; ++i) {
+                float k[CPT], v[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, k);
+                Vec<IO, CPT>::load(p1 + i * CG, v);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    const float x = fmaf(static_cast<float>(i - (LS - 1)), q[j].w, k[j]);
+                    const float e = ex2_approx((x - m[j]) * kLog2e);
+                    a[j] = fmaf(e, v[j], a[j]);
+                    b[j] += e;
+                }
+            }
+        } else {
+            for (int i = 0; i < n; ++i) {
+                float k[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, k);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    m[j] = fmaxf(m[j], fmaf(static_cast<float>(i - (n - 1)), q[j].w, k[j]));
+                    kx[j] = fmaxf(kx[j], k[j]);
+                    kn[j] = fminf(kn[j], k[j]);
+                }
+            }
+            for (int i = 0; i < n; ++i) {
+                float k[CPT], v[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, k);
+                Vec<IO, CPT>::load(p1 + i * CG, v);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    const float x = fmaf(static_cast<float>(i - (n - 1)), q[j].w, k[j]);
+                    const float e = ex2_approx((x - m[j]) * kLog2e);
+                    a[j] = fmaf(e, v[j], a[j]);
+                    b[j] += e;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            out[j] = {a[j], b[j], m[j]};
+            sc[j] = {kx[j], kn[j]};
+        }
     }
 
-    // output at this step, then the state update
-    __device__ __forceinline__ static float step2(State &s, float k, float v, const Param &q) {
-        const float x = fmaf(k, kLog2e, q.uu);
+    // ---- pass 2 ------------------------------------------------------------
+    // exact per-step update (max-stabilised), one channel
+    __device__ __forceinline__ static float step_exact(State &s, float k, float v,
+                                                       const Param &q) {
+        const float x = q.u + k;
         const float d = s.p - x;
-        const float e = ex2_approx(-fabsf(d));
+        const float e = ex2_approx(-fabsf(d) * kLog2e);
         const bool old_wins = d >= 0.f;
         const float fo = old_wins ? 1.f : e, fn = old_wins ? e : 1.f;
-        const float num = fmaf(s.a, fo, fn * v);
-        const float den = fmaf(s.b, fo, fn);
-        // fp32 outputs use the correctly rounded quotient, so a constant
-        // power-of-two v comes back exactly; bf16 outputs are rounded to 8
-        // significant bits afterwards, where one ulp of fp32 cannot matter
-        const float y = kExactDiv ? __fdiv_rn(num, den) : num * rcp_approx(den);
-        step1(s, k, v, q);
+        // (fo a + fn v) / (fo b + fn) with fo, fn as the state's and the token's weights
+        const float y = wkv_output(fo * s.a, fo * s.b, fn, v);
+        const float pd = s.p - q.w;
+        const float d2 = pd - k;
+        const float e2 = ex2_approx(-fabsf(d2) * kLog2e);
+        const bool old2 = d2 >= 0.f;
+        const float go = old2 ? 1.f : e2, gn = old2 ? e2 : 1.f;
+        s.a = fmaf(s.a, go, gn * v);
+        s.b = fmaf(s.b, go, gn);
+        s.p = fmaxf(pd, k);
         return y;
+    }
+
+    template <int LS>
+    __device__ __forceinline__ static void sweep(const State (&carry)[CPT], IO *p0, const IO *p1,
+                                                 int n, const Param (&q)[CPT],
+                                                 const Scratch (&sc)[CPT]) {
+        // reference per channel, and whether the fixed-reference form is safe
+        float M[CPT], A[CPT], Bs[CPT];
+        bool fast = true;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            M[j] = fmaxf(carry[j].p, sc[j].kmax);
+            const float s = expf(carry[j].p - M[j]);
+            A[j] = carry[j].a * s;
+            Bs[j] = carry[j].b * s;
+            // den_t >= e^{u + k_t - M}, and den_t >= b_in e^{p_in - M - t w}
+            const bool by_token = sc[j].kmin + q[j].u - M[j] >= -69.f;
+            const bool by_carry =
+                carry[j].b >= 1.f && carry[j].p - M[j] - static_cast<float>(n) * q[j].w >= -69.f;
+            fast = fast && (by_token || by_carry) && q[j].u <= 44.f;
+        }
+        if (fast) {
+            if (n == LS) {
+#pragma unroll 8
+                for (int i = 0; i < LS; ++i) fast_step(p0 + i * CG, p1 + i * CG, M, A, Bs, q);
+            } else {
+                for (int i = 0; i < n; ++i) fast_step(p0 + i * CG, p1 + i * CG, M, A, Bs, q);
+            }
+        } else {
+            State s[CPT];
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) s[j] = carry[j];
+            for (int i = 0; i < n; ++i) {
+                float k[CPT], v[CPT], y[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, k);
+                Vec<IO, CPT>::load(p1 + i * CG, v);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) y[j] = step_exact(s[j], k[j], v[j], q[j]);
+                Vec<IO, CPT>::store(p0 + i * CG, y);
+            }
+        }
+    }
+
+    __device__ __forceinline__ static void fast_step(IO *pk, const IO *pv, const float (&M)[CPT],
+                                                     float (&A)[CPT], float (&Bs)[CPT],
+                                                     const Param (&q)[CPT]) {
+        float k[CPT], v[CPT], y[CPT];
+        Vec<IO, CPT>::load(pk, k);
+        Vec<IO, CPT>::load(pv, v);
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const float e = ex2_approx((k[j] - M[j]) * kLog2e);
+            const float eu = e * q[j].U;
+            y[j] = wkv_output(A[j], Bs[j], eu, v[j]);
+            A[j] = fmaf(A[j], q[j].D, e * v[j]);
+            Bs[j] = fmaf(Bs[j], q[j].D, e);
+        }
+        Vec<IO, CPT>::store(pk, y);
     }
 };
 
 // ---------------------------------------------------------------------------
 // Diagonal linear scan h_t = a_t h_{t-1} + b_t ("Were RNNs All We Needed?",
 // model-architecture section).  Chunk summary: (A, H) = (product of the a's,
-// state produced from h = 0); state h followed by chunk (A, H) gives A h + H.
+// state produced from h = 0); the state h followed by a chunk (A, H) is
+// A h + H.
 // ---------------------------------------------------------------------------
 struct ScanOp {
     using io_t = float;
     static constexpr int CPT = 1;
+    static constexpr int CG = 32;
     static constexpr int NV = 2;
     struct Param {};
     struct State {
@@ -129,6 +314,7 @@ struct ScanOp {
         float *y;         // h [B, T, D]
         const float *h0;  // [B, D] or nullptr
     };
+    struct Scratch {};
 
     __device__ __forceinline__ static Param param(const Args &, int, int) { return {}; }
     __device__ __forceinline__ static State identity() { return {1.f, 0.f}; }
@@ -147,13 +333,46 @@ struct ScanOp {
                                                     const Param &) {
         return {l.A * r.A, fmaf(r.A, l.H, r.H)};
     }
-    __device__ __forceinline__ static void step1(State &s, float a, float b, const Param &) {
-        s.H = fmaf(a, s.H, b);
-        s.A *= a;
+
+    template <int LS>
+    __device__ __forceinline__ static void summarize(const float *p0, const float *p1, int n,
+                                                     const Param (&)[1], State (&out)[1],
+                                                     Scratch (&)[1]) {
+        float A = 1.f, H = 0.f;
+        if (n == LS) {
+#pragma unroll
+            for (int i = 0; i < LS; ++i) {
+                const float a = p0[i * CG], b = p1[i * CG];
+                H = fmaf(a, H, b);
+                A *= a;
+            }
+        } else {
+            for (int i = 0; i < n; ++i) {
+                const float a = p0[i * CG], b = p1[i * CG];
+                H = fmaf(a, H, b);
+                A *= a;
+            }
+        }
+        out[0] = {A, H};
     }
-    __device__ __forceinline__ static float step2(State &s, float a, float b, const Param &) {
-        s.H = fmaf(a, s.H, b);
-        return s.H;
+
+    template <int LS>
+    __device__ __forceinline__ static void sweep(const State (&carry)[1], float *p0,
+                                                 const float *p1, int n, const Param (&)[1],
+                                                 const Scratch (&)[1]) {
+        float H = carry[0].H;
+        if (n == LS) {
+#pragma unroll
+            for (int i = 0; i < LS; ++i) {
+                H = fmaf(p0[i * CG], H, p1[i * CG]);
+                p0[i * CG] = H;
+            }
+        } else {
+            for (int i = 0; i < n; ++i) {
+                H = fmaf(p0[i * CG], H, p1[i * CG]);
+                p0[i * CG] = H;
+            }
+        }
     }
 };
 

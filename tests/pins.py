@@ -225,7 +225,7 @@ def scan_worked_example(fn, tol=1e-12):
     return [f"worked example: {msg}"] if msg else []
 
 
-def scan_closed_forms(fn, tol=1e-10):
+def scan_closed_forms(fn, tol=1e-10, exact_tol=0.0):
     out = []
     rng = np.random.default_rng(11)
     B, T, D = 2, 50, 3
@@ -235,7 +235,7 @@ def scan_closed_forms(fn, tol=1e-10):
     msg = _close(fn(np.ones((B, T, D)), b, h0), h0[:, None, :] + np.cumsum(b, axis=1), tol)
     if msg: out.append(f"a=1 cumsum: {msg}")
     # a = 0: h = b
-    msg = _close(fn(np.zeros((B, T, D)), b, h0), b, 0.0)
+    msg = _close(fn(np.zeros((B, T, D)), b, h0), b, exact_tol)
     if msg: out.append(f"a=0: {msg}")
     # b = 0: h_t = h0 * prod_{j<=t} a_j
     a = rng.uniform(0.5, 1.2, (B, T, D))
