@@ -362,13 +362,13 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
         case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
         case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
         case 64:
-            return tma ? launch_persistent<Op, 64, 4, 2, 6>(args, B, T, C, dt, stream, dev)
+            return tma ? launch_persistent<Op, 64, 4, 6, 12>(args, B, T, C, dt, stream, dev)
                        : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
         case 256:
-            return tma ? launch_persistent<Op, 256, 8, 1, 3>(args, B, T, C, dt, stream, dev)
+            return tma ? launch_persistent<Op, 256, 8, 2, 3>(args, B, T, C, dt, stream, dev)
                        : launch_chunked<Op, 256, 8>(args, B, T, C, dt, stream, dev);
         default:
-            return tma ? launch_persistent<Op, 128, 4, 2, 6>(args, B, T, C, dt, stream, dev)
+            return tma ? launch_persistent<Op, 128, 4, 4, 6>(args, B, T, C, dt, stream, dev)
                        : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
     }
 }

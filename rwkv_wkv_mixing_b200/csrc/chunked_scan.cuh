@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(NW * 32, 3)
                 cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(LS), prm[j]);
             }
         }
-        Op::template sweep<LS>(cur, p0, p1, nval, prm, sc);
+        Op::template sweep<LS>(cur, p0, p1, nval, prm, sc, p0, CG, true);
     }
 
     // ---- write the output tile ----------------------------------------------

@@ -10,14 +10,17 @@
 // two passes and look-back as chunked_scan_kernel -- pass 1 summaries per
 // warp, the carry into the tile (aggregate, decoupled look-back, publication)
 // by the group's first warp, pass 2 writing outputs over the stage's first
-// tensor -- then one thread issues the TMA store of the outputs and releases
-// the stage of the group's previous tile once that tile's store has read it.
+// tensor -- then one thread issues the TMA store of the outputs, waits until
+// the store has read the stage, and releases it to the producer.  Outputs
+// leave through the async proxy, so the look-back's release fences never wait
+// behind a warp's own output stores.
 //
-// So HBM sees every element once, loads for the next tiles are always in
-// flight while tiles are being computed, and no thread block is launched per
-// tile.  Every wait is bounded (global-timer deadline on mbarriers, poll
-// budget in the look-back); a wait that gives up records WKV_ERR_TIMEOUT in
-// the status word and makes every loop of the block finish.
+// So HBM sees every element once, loads for the next tiles are in flight
+// while tiles are being computed, several tiles per SM hide the look-back
+// latency, and no thread block is launched per tile.  Every wait is bounded
+// (global-timer deadline on mbarriers, poll budget in the look-back); a wait
+// that gives up records WKV_ERR_TIMEOUT in the status word and makes every
+// loop of the block finish.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -40,7 +43,8 @@ struct PersistentCfg {
         NSTAGE * kStageBytes + static_cast<size_t>(NC) * (NWG + 1) * NV * CG * sizeof(float);
     static_assert(LT % NWG == 0, "tile length must split evenly over a group's warps");
     static_assert(LT <= 256, "TMA box rows are limited to 256");
-    static_assert(NSTAGE >= 2 * NC, "each group may hold two stages");
+    static_assert(NSTAGE > NC, "one stage per group plus at least one being loaded");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
     static_assert(1 + NC <= 16, "named barrier ids");
 };
 
@@ -153,7 +157,6 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
         const int bar_id = 1 + grp;
         float *g_sum = s_sum + grp * NWG * NV * CG;
         float *g_carry = s_carry + grp * NV * CG;
-        int prev_s = -1;
         for (int it = grp;; it += NC) {
             const int s = it % NSTAGE;
             const uint32_t parity = (it / NSTAGE) & 1;
@@ -249,7 +252,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             }
             named_bar_sync(bar_id, NWG * 32);
 
-            // pass 2
+            // pass 2: outputs over the stage's first tensor
             if (nval > 0) {
                 State cur[CPT];
 #pragma unroll
@@ -264,26 +267,19 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                         cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(LS), prm[j]);
                     }
                 }
-                Op::template sweep<LS>(cur, p0, p1, nval, prm, sc);
+                Op::template sweep<LS>(cur, p0, p1, nval, prm, sc, p0, CG, true);
             }
             fence_proxy_async_smem();
             named_bar_sync(bar_id, NWG * 32);
 
-            // store the outputs; release the previous tile's stage once its
-            // store has read it
+            // store the tile (rows >= T and channels >= C are clipped), then
+            // hand the stage back once the store has read it
             if (gtid == 0) {
                 tma_store_3d(&map_y, s_x0, c0, t0, b);
                 bulk_commit();
-                if (prev_s >= 0) {
-                    bulk_wait_read_all_but_one();
-                    mbar_arrive(&empty_bar[prev_s]);
-                }
-                prev_s = s;
+                bulk_wait_read_all();
+                mbar_arrive(&empty_bar[s]);
             }
-        }
-        if (gtid == 0 && prev_s >= 0) {
-            bulk_wait_read_all();
-            mbar_arrive(&empty_bar[prev_s]);
         }
         __syncwarp();
     }

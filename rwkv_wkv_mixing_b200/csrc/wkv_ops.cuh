@@ -5,7 +5,7 @@
 //   summarize(p0, p1, n, ...)  pass 1: the summary of an n-step sub-chunk
 //                              (rows p0[i*CG], p1[i*CG]) from the empty state
 //   sweep(carry, ...)          pass 2: outputs of the sub-chunk from the state
-//                              before it, written over p0's rows
+//                              before it, to out[i*ostride] (shared or global)
 //   combine(l, r, r_len)       the state l followed by a chunk of r_len steps
 //                              whose summary is r
 #pragma once
@@ -234,10 +234,13 @@ struct WkvOp {
         return y;
     }
 
+    // outputs go to out[i * ostride] (shared or global memory); when `valid`
+    // is false this thread's channels are past C and nothing is stored
     template <int LS>
-    __device__ __forceinline__ static void sweep(const State (&carry)[CPT], IO *p0, const IO *p1,
-                                                 int n, const Param (&q)[CPT],
-                                                 const Scratch (&sc)[CPT]) {
+    __device__ __forceinline__ static void sweep(const State (&carry)[CPT], const IO *p0,
+                                                 const IO *p1, int n, const Param (&q)[CPT],
+                                                 const Scratch (&sc)[CPT], IO *out, size_t ostride,
+                                                 bool valid) {
         // reference per channel, and whether the fixed-reference form is safe
         float M[CPT], A[CPT], Bs[CPT];
         bool fast = true;
@@ -256,9 +259,11 @@ struct WkvOp {
         if (fast) {
             if (n == LS) {
 #pragma unroll 8
-                for (int i = 0; i < LS; ++i) fast_step(p0 + i * CG, p1 + i * CG, M, A, Bs, q);
+                for (int i = 0; i < LS; ++i)
+                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, A, Bs, q);
             } else {
-                for (int i = 0; i < n; ++i) fast_step(p0 + i * CG, p1 + i * CG, M, A, Bs, q);
+                for (int i = 0; i < n; ++i)
+                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, A, Bs, q);
             }
         } else {
             State s[CPT];
@@ -270,14 +275,14 @@ struct WkvOp {
                 Vec<IO, CPT>::load(p1 + i * CG, v);
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) y[j] = step_exact(s[j], k[j], v[j], q[j]);
-                Vec<IO, CPT>::store(p0 + i * CG, y);
+                if (valid) Vec<IO, CPT>::store(out + i * ostride, y);
             }
         }
     }
 
-    __device__ __forceinline__ static void fast_step(IO *pk, const IO *pv, const float (&M)[CPT],
-                                                     float (&A)[CPT], float (&Bs)[CPT],
-                                                     const Param (&q)[CPT]) {
+    __device__ __forceinline__ static void fast_step(const IO *pk, const IO *pv, IO *py, bool valid,
+                                                     const float (&M)[CPT], float (&A)[CPT],
+                                                     float (&Bs)[CPT], const Param (&q)[CPT]) {
         float k[CPT], v[CPT], y[CPT];
         Vec<IO, CPT>::load(pk, k);
         Vec<IO, CPT>::load(pv, v);
@@ -289,7 +294,7 @@ struct WkvOp {
             A[j] = fmaf(A[j], q[j].D, e * v[j]);
             Bs[j] = fmaf(Bs[j], q[j].D, e);
         }
-        Vec<IO, CPT>::store(pk, y);
+        if (valid) Vec<IO, CPT>::store(py, y);
     }
 };
 
@@ -357,20 +362,21 @@ struct ScanOp {
     }
 
     template <int LS>
-    __device__ __forceinline__ static void sweep(const State (&carry)[1], float *p0,
+    __device__ __forceinline__ static void sweep(const State (&carry)[1], const float *p0,
                                                  const float *p1, int n, const Param (&)[1],
-                                                 const Scratch (&)[1]) {
+                                                 const Scratch (&)[1], float *out, size_t ostride,
+                                                 bool valid) {
         float H = carry[0].H;
         if (n == LS) {
-#pragma unroll
+#pragma unroll 8
             for (int i = 0; i < LS; ++i) {
                 H = fmaf(p0[i * CG], H, p1[i * CG]);
-                p0[i * CG] = H;
+                if (valid) out[i * ostride] = H;
             }
         } else {
             for (int i = 0; i < n; ++i) {
                 H = fmaf(p0[i * CG], H, p1[i * CG]);
-                p0[i * CG] = H;
+                if (valid) out[i * ostride] = H;
             }
         }
     }
