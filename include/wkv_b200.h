@@ -101,6 +101,35 @@ WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,
                      const float *a, const float *b, const float *h0, float *h,
                      cudaStream_t stream);
 
+/* WKV forward, fp32, without allocating any device memory.  The pages this
+ * library follows have no counterpart of this entry point: it exists for
+ * callers that cannot call cudaMalloc -- code running inside an engine that
+ * has already reserved the GPU's memory for its own pool, plugin interfaces
+ * that hand an operator nothing but its input and output buffers, and
+ * latency-critical paths that must not pay for an allocation or for the
+ * device-wide synchronisation cudaMalloc / cudaFree can cause.
+ *
+ * Same operation, arguments, layout and host-side checks as wkv_forward.
+ * Instead of a workspace, the state passed between thread blocks lives in one
+ * fixed 16 MiB device array; every GPU that uses this entry point holds it
+ * from its first call until the process exits.  A problem whose scratch would
+ * not fit -- more than 21,619 tiles, i.e. B * ceil(C/32) * ceil(T/128) >
+ * 21,619 (sequences of at most 128 steps need no scratch) -- is rejected with
+ * WKV_ERR_INVALID_ARG before anything runs; use wkv_forward for it.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and sets kernel
+ * attributes; make that first call before any stream capture.
+ * Every call on a device shares the one array and first clears (cudaMemsetAsync
+ * on `stream`) the counters and flags that must start at zero, so calls whose
+ * work overlaps on the GPU -- on different streams, or from several host
+ * threads -- race and give wrong results: serialise them.  A device-side wait
+ * that gives up leaves NaN in the affected outputs; wkv_device_status does not
+ * report it for this entry point. */
+WKV_API wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C,
+                                       const float *w, const float *u,
+                                       const float *k, const float *v, float *y,
+                                       cudaStream_t stream);
+
 /* Synchronise `stream`, then return and clear the device status word of that
  * stream's workspace: WKV_OK, or WKV_ERR_TIMEOUT if a device-side wait gave up
  * since the last query.  WKV_ERR_CUDA if the synchronisation itself failed. */

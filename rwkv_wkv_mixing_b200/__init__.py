@@ -30,13 +30,14 @@ STATUS_NAMES = {0: "WKV_OK", 1: "WKV_ERR_INVALID_ARG", 2: "WKV_ERR_ALIGNMENT",
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m rwkv_wkv_mixing_b200.build` (nvcc, sm_100a)")
+                      "`python rwkv_wkv_mixing_b200/build.py` (nvcc, sm_100a)")
 
 _i64, _p, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
 lib = ctypes.CDLL(LIB_PATH)
 _SIGS = {
     "wkv_forward": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_bf16": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_noalloc": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "diag_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "wkv_device_status": ([_p], _i32),
     "wkv_last_error": ([], ctypes.c_char_p),
@@ -117,6 +118,15 @@ def wkv_forward_bf16(w, u, k, v, y=None, stream=None):
     return _wkv("wkv_forward_bf16", torch.bfloat16, w, u, k, v, y, stream)
 
 
+def wkv_forward_noalloc(w, u, k, v, y=None, stream=None):
+    """WKV forward, fp32, with the library allocating no device memory: its
+    scratch is a fixed 16 MiB device array shared by every call on a device
+    (serialise calls; problems needing more scratch raise WkvError).  For
+    callers that cannot allocate; `y` should then be passed in."""
+    import torch
+    return _wkv("wkv_forward_noalloc", torch.float32, w, u, k, v, y, stream)
+
+
 def diag_scan(a, b, h0=None, h=None, stream=None):
     """h_t = a_t * h_{t-1} + b_t per channel, h_{-1} = h0 (zeros if None)."""
     import torch
@@ -162,6 +172,6 @@ def wkv_get_tile_steps() -> int:
     return int(lib.wkv_get_tile_steps())
 
 
-__all__ = ["wkv_forward", "wkv_forward_bf16", "diag_scan", "wkv_device_status",
+__all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan", "wkv_device_status",
            "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
            "wkv_get_tile_steps", "WkvError", "lib", "LIB_PATH"]

@@ -1,6 +1,6 @@
 """Build libwkv_b200.so in-tree with nvcc for sm_100a.
 
-    python -m rwkv_wkv_mixing_b200.build [--verbose]
+    python rwkv_wkv_mixing_b200/build.py [--verbose]
 
 No GPU is needed: nvcc cross-compiles.  The CUDA runtime is linked
 statically and the driver API is reached through cudaGetDriverEntryPoint, so
@@ -19,8 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libwkv_b200.so")
-SOURCES = ["capi.cu"]
-HEADERS = ["chunked_scan.cuh", "wkv_ops.cuh", "ptx.cuh"]
+SOURCES = ["capi.cu", "noalloc.cu"]
+HEADERS = ["chunked_scan.cuh", "persistent_scan.cuh", "scan_common.cuh", "wkv_ops.cuh", "ptx.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -23,8 +23,15 @@
 using namespace wkvb;
 
 namespace {
-
 thread_local std::string t_err;
+}
+
+namespace wkvb {
+// lets the library's other translation units set the wkv_last_error() message
+void set_last_error(const char *msg) { t_err = msg; }
+}  // namespace wkvb
+
+namespace {
 
 wkv_status fail(wkv_status st, const char *fmt, ...) {
     char buf[512];
