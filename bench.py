@@ -70,6 +70,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--launch", default="graph", choices=["graph", "direct"],
+                    help="replay the K steps from CUDA graphs (default) or call directly")
     return ap.parse_args(argv)
 
 
@@ -227,7 +229,6 @@ class DeviceWorkload:
             b = x1 if i == 0 else x1.clone()
             self.sets.append((a, b, torch.empty_like(a)))
         self.stream = torch.cuda.current_stream()
-        self.sh = self.stream.cuda_stream
 
     def _to_dev(self, arr, dev):
         t = self.torch.from_numpy(np.ascontiguousarray(arr))
@@ -236,13 +237,16 @@ class DeviceWorkload:
         return t.to(dev)
 
     def call(self, x0, x1, y):
+        """One C-ABI call on torch's current stream (the capture stream while a
+        graph is being captured)."""
         lib = self.lib
+        sh = self.torch.cuda.current_stream().cuda_stream
         if self.is_scan:
             return lib.diag_scan(self.B, self.T, self.C, x0.data_ptr(), x1.data_ptr(), None,
-                                 y.data_ptr(), self.sh)
+                                 y.data_ptr(), sh)
         fn = lib.wkv_forward_bf16 if self.dtype == "bf16" else lib.wkv_forward
         return fn(self.B, self.T, self.C, self.params[0].data_ptr(), self.params[1].data_ptr(),
-                  x0.data_ptr(), x1.data_ptr(), y.data_ptr(), self.sh)
+                  x0.data_ptr(), x1.data_ptr(), y.data_ptr(), sh)
 
     def step(self, i):
         st = self.call(*self.sets[i % self.n_sets])
@@ -251,21 +255,88 @@ class DeviceWorkload:
 
 
 def time_steps(torch, wl, K):
-    """K steps back to back; events around the whole region and around every
-    launch (all on the launching stream)."""
+    """K steps launched directly, back to back; events around the whole region
+    and around every launch.  When the host is slower than the GPU these
+    per-launch events also see host time, so `time_steps_graph` is the
+    default."""
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(wl.stream)
+    stream = torch.cuda.current_stream()
+    start.record(stream)
     for i in range(K):
-        ev[i][0].record(wl.stream)
+        ev[i][0].record(stream)
         wl.step(i)
-        ev[i][1].record(wl.stream)
-    end.record(wl.stream)
+        ev[i][1].record(stream)
+    end.record(stream)
     end.synchronize()
-    total_ms = start.elapsed_time(end)
-    per = [a.elapsed_time(b) for a, b in ev]
-    return total_ms, per
+    return start.elapsed_time(end), [a.elapsed_time(b) for a, b in ev]
+
+
+class StepGraphs:
+    """Steps captured into CUDA graphs (each step one C-ABI call), so K steps
+    replay back to back on the device with no host work between them.  Events
+    on the launching stream bracket every replay; a launch's duration is its
+    replay's duration over the steps in it."""
+
+    def __init__(self, torch, wl, K, chunk=128):
+        self.torch, self.wl, self.K = torch, wl, K
+        self.G = min(K, chunk)
+        self.reps, self.tail = divmod(K, self.G)
+        self.side = torch.cuda.Stream()
+        self.graph = self._capture(self.G)
+        self.tail_graph = self._capture(self.tail) if self.tail else None
+
+    def _capture(self, n):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        # the library keeps one look-back workspace per stream and cannot
+        # allocate it during capture: size it with plain calls first
+        torch.cuda.synchronize()
+        with torch.cuda.stream(self.side):
+            for i in range(3):
+                self.wl.step(i)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=self.side):
+            for i in range(n):
+                self.wl.step(i)
+        torch.cuda.synchronize()
+        return g
+
+    def warm(self):
+        self.graph.replay()
+        if self.tail_graph is not None:
+            self.tail_graph.replay()
+        self.torch.cuda.synchronize()
+
+    def run(self):
+        """Replay K steps; total ms and the mean launch ms of every replay."""
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        mk = lambda: torch.cuda.Event(enable_timing=True)   # noqa: E731
+        marks = [mk() for _ in range(self.reps + 2)]
+        marks[0].record(stream)
+        for r in range(self.reps):
+            self.graph.replay()
+            marks[r + 1].record(stream)
+        if self.tail_graph is not None:
+            self.tail_graph.replay()
+        marks[-1].record(stream)
+        marks[-1].synchronize()
+        per = [marks[r].elapsed_time(marks[r + 1]) / self.G for r in range(self.reps)]
+        return marks[0].elapsed_time(marks[-1]), per
+
+
+def host_overhead_us(torch, wl, n=200):
+    """Host time of one C-ABI call (argument checks, tensor maps, launch),
+    measured while the GPU is busy so calls never wait on the device."""
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(n):
+        wl.step(i)
+    dt = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    return dt / n * 1e6
 
 
 def e2e_leg(torch, wl, steps):
@@ -466,9 +537,18 @@ def main(argv=None):
                 wl.step(i); i += 1
             torch.cuda.synchronize()
 
+    graphs = None
+    if args.launch == "graph":
+        graphs = StepGraphs(torch, wl, args.steps)
+        graphs.warm()
+    host_us = host_overhead_us(torch, wl)
+
     barrier()
     t_timed0 = time.time()
-    total_ms, per = time_steps(torch, wl, args.steps)
+    if graphs is not None:
+        total_ms, per = graphs.run()
+    else:
+        total_ms, per = time_steps(torch, wl, args.steps)
     barrier()
     t_timed1 = time.time()
     if sampler is not None:
@@ -481,6 +561,8 @@ def main(argv=None):
 
     ms_per_step = total_ms / args.steps
     value = aggregate_rate(wl.elements, world, ms_per_step)
+    if not per:
+        per = [total_ms / args.steps]
     launch_ms = statistics.mean(per)
     peak, peak_kind = read_peaks()
     achieved = wl.alg_bytes / (launch_ms / 1e3) / 1e9
@@ -505,6 +587,8 @@ def main(argv=None):
                        f"({wl.n_sets * 3 * wl.es * wl.elements / 1e6:.0f} MB > L2 "
                        f"{l2 / 1e6:.0f} MB)"),
                 "tile_steps": wkv.wkv_get_tile_steps(),
+                "launch": args.launch + (" (K steps replayed from captured graphs)"
+                                         if args.launch == "graph" else ""),
                 "gpu": props.name, "sms": props.multi_processor_count})
     line = {
         "metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world,
@@ -522,6 +606,7 @@ def main(argv=None):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps,
+        "host_us_per_call": host_us,
         "clocks": sampler.summary(t_timed0, t_timed1) if sampler is not None else None,
     }
     if rank == 0:

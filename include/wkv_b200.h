@@ -113,14 +113,14 @@ WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,
  * Instead of a workspace, the state passed between thread blocks lives in one
  * fixed 16 MiB device array; every GPU that uses this entry point holds it
  * from its first call until the process exits.  A problem whose scratch would
- * not fit -- more than 21,619 tiles, i.e. B * ceil(C/32) * ceil(T/128) >
- * 21,619 (sequences of at most 128 steps need no scratch) -- is rejected with
+ * not fit -- more than 32,767 tiles, i.e. B * ceil(C/32) * ceil(T/128) >
+ * 32,767 (sequences of at most 128 steps need no scratch) -- is rejected with
  * WKV_ERR_INVALID_ARG before anything runs; use wkv_forward for it.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and sets kernel
  * attributes; make that first call before any stream capture.
  * Every call on a device shares the one array and first clears (cudaMemsetAsync
- * on `stream`) the counters and flags that must start at zero, so calls whose
+ * on `stream`) the counters and records that must start at zero, so calls whose
  * work overlaps on the GPU -- on different streams, or from several host
  * threads -- race and give wrong results: serialise them.  A device-side wait
  * that gives up leaves NaN in the affected outputs; wkv_device_status does not

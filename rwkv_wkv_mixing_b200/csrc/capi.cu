@@ -151,17 +151,9 @@ constexpr size_t kWsHeader = 256;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-struct WsLayout {
-    size_t flags, agg, incl, total;
-};
-
-WsLayout ws_layout(size_t tiles, size_t floats_per_tile) {
-    WsLayout l;
-    l.flags = kWsHeader;
-    l.agg = round_up(l.flags + tiles * sizeof(unsigned long long), 256);
-    l.incl = round_up(l.agg + tiles * floats_per_tile * sizeof(float), 256);
-    l.total = round_up(l.incl + tiles * floats_per_tile * sizeof(float), 256);
-    return l;
+// header, then one 16-byte record per (tile, channel)
+size_t ws_bytes(size_t tiles, size_t channels_per_tile) {
+    return round_up(kWsHeader + tiles * channels_per_tile * sizeof(uint4), 256);
 }
 
 WsEntry *find_ws(int dev, cudaStream_t stream) {
@@ -290,18 +282,15 @@ wkv_status make_plan(const typename Op::Args &args, int64_t B, int64_t T, int64_
     std::memset(&p->ws, 0, sizeof p->ws);
     if (g.n_seg > 1) {
         std::lock_guard<std::mutex> lk(g_mu);
-        const WsLayout l = ws_layout(static_cast<size_t>(tiles), Op::NV * CG);
         WsEntry *e = nullptr;
-        wkv_status st = ensure_ws(dev, stream, l.total, &e);
+        wkv_status st = ensure_ws(dev, stream, ws_bytes(static_cast<size_t>(tiles), CG), &e);
         if (st != WKV_OK) return st;
         Workspace &ws = p->ws;
         ws.ticket = reinterpret_cast<unsigned int *>(e->base);
         ws.done = reinterpret_cast<unsigned int *>(e->base + 4);
         ws.epoch = reinterpret_cast<unsigned long long *>(e->base + 8);
         ws.status = reinterpret_cast<int *>(e->base + 16);
-        ws.flags = reinterpret_cast<unsigned long long *>(e->base + l.flags);
-        ws.agg = reinterpret_cast<float *>(e->base + l.agg);
-        ws.incl = reinterpret_cast<float *>(e->base + l.incl);
+        ws.records = reinterpret_cast<uint4 *>(e->base + kWsHeader);
     }
     return WKV_OK;
 }

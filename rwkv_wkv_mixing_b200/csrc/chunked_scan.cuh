@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(NW * 32, 3)
             // every tile this block waits for belongs to a block that is
             // already resident: the look-back always makes progress.
             tile = static_cast<int>(atomicAdd(ws.ticket, 1u));
-            epoch = ld_relaxed_gpu_u64(ws.epoch);
+            epoch = epoch_of(ws);
             if (tile >= g.tiles) {  // counters corrupted: report, do no work
                 atomicExch(ws.status, kStatusTimeout);
                 tile = -1;
@@ -161,11 +161,17 @@ __global__ void __launch_bounds__(NW * 32, 3)
         State agg[CPT], X[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
+            // fold the warps' summaries in time order; each slot is
+            // overwritten with its warp's exclusive prefix (the fold of the
+            // sub-chunks before it) for pass 2
             agg[j] = Op::identity();
             for (int s = 0; s < NW; ++s) {
                 float vals[NV];
+                float *slot = s_sum + s * NV * CG + lane * CPT + j;
 #pragma unroll
-                for (int q = 0; q < NV; ++q) vals[q] = s_sum[(s * NV + q) * CG + lane * CPT + j];
+                for (int q = 0; q < NV; ++q) vals[q] = slot[q * CG];
+#pragma unroll
+                for (int q = 0; q < NV; ++q) slot[q * CG] = Op::get(agg[j], q);
                 const int len = max(0, min(LS, g.T - (t0 + s * LS)));
                 agg[j] = Op::combine(agg[j], Op::make(vals), static_cast<float>(len), prm[j]);
             }
@@ -178,14 +184,14 @@ __global__ void __launch_bounds__(NW * 32, 3)
 #pragma unroll
                 for (int j = 0; j < CPT; ++j)
                     inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                publish<Op, CG>(ws.incl, ws.flags, tile, inc, (epoch << 2) | kFlagIncl, lane);
+                publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
             } else {
                 if (!last)
-                    publish<Op, CG>(ws.agg, ws.flags, tile, agg, (epoch << 2) | kFlagAgg, lane);
+                    publish<Op, CG>(ws, tile, agg, kFlagAgg, epoch, lane);
                 // decoupled look-back over the tiles before this one in time
                 State run[CPT];
                 if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run)) {
-                    if (lane == 0) atomicExch(ws.status, kStatusTimeout);
+                    atomicExch(ws.status, kStatusTimeout);  // this lane gave up
 #pragma unroll
                     for (int j = 0; j < CPT; ++j) run[j] = Op::nan_state();
                 }
@@ -196,8 +202,7 @@ __global__ void __launch_bounds__(NW * 32, 3)
 #pragma unroll
                     for (int j = 0; j < CPT; ++j)
                         inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                    publish<Op, CG>(ws.incl, ws.flags, tile, inc, (epoch << 2) | kFlagIncl,
-                                    lane);
+                    publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
                 }
             }
         }
@@ -217,10 +222,10 @@ __global__ void __launch_bounds__(NW * 32, 3)
 #pragma unroll
             for (int q = 0; q < NV; ++q) vals[q] = s_carry[q * CG + lane * CPT + j];
             cur[j] = Op::make(vals);
-            for (int s = 0; s < warp; ++s) {  // earlier sub-chunks are all full
+            if (warp > 0) {  // the sub-chunks before this warp's, all full
 #pragma unroll
-                for (int q = 0; q < NV; ++q) vals[q] = s_sum[(s * NV + q) * CG + lane * CPT + j];
-                cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(LS), prm[j]);
+                for (int q = 0; q < NV; ++q) vals[q] = s_sum[(warp * NV + q) * CG + lane * CPT + j];
+                cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(warp * LS), prm[j]);
             }
         }
         Op::template sweep<LS>(cur, p0, p1, nval, prm, sc, p0, CG, true);

@@ -34,6 +34,7 @@ constexpr size_t kScratchBytes = static_cast<size_t>(16) << 20;  // 16 MiB per d
 constexpr int kMaxDevices = 64;
 constexpr int kTileSteps = 128;  // tile length of both kernel variants used here
 constexpr size_t kHeader = 256;  // [0] ticket, [4] done, [8] epoch, [16] status
+constexpr size_t kMaxTiles = (kScratchBytes - kHeader) / (32 * sizeof(uint4));  // 32767
 
 // the scratch; host code must not pass this name to a kernel (it is a host
 // stand-in), only the device address cudaGetSymbolAddress returns
@@ -158,23 +159,18 @@ extern "C" wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const
         return fail(WKV_ERR_INVALID_ARG, "each of B, T, C must be below 2^31");
     if (static_cast<unsigned __int128>(B) * T * C >= (static_cast<unsigned __int128>(1) << 62))
         return fail(WKV_ERR_INVALID_ARG, "B*T*C must be below 2^62");
-    // tiles of 32 channels x kTileSteps steps, and the scratch they need
+    // tiles of 32 channels x kTileSteps steps, and the scratch they need: a
+    // header and one 16-byte record per (tile, channel)
     const long long n_cg = (C + 31) / 32, n_seg = (T + kTileSteps - 1) / kTileSteps;
     const long long tiles = B * n_cg * n_seg;
-    const size_t flags_bytes = (static_cast<size_t>(tiles) * 8 + 255) / 256 * 256;
-    const size_t per_tile_floats = static_cast<size_t>(Op::NV) * 32;
-    const size_t need = n_seg > 1 ? kHeader + flags_bytes + 2 * static_cast<size_t>(tiles) *
-                                                                per_tile_floats * sizeof(float)
-                                  : 0;
+    const size_t need = n_seg > 1 ? kHeader + static_cast<size_t>(tiles) * 32 * sizeof(uint4) : 0;
     if (tiles > INT32_MAX || need > kScratchBytes)
         return fail(WKV_ERR_INVALID_ARG,
                     "wkv_forward_noalloc: B=%lld T=%lld C=%lld needs %zu bytes of scratch, more "
                     "than its fixed %zu-byte device array (at most %zu tiles of 32 channels x %d "
                     "steps); use wkv_forward",
                     static_cast<long long>(B), static_cast<long long>(T),
-                    static_cast<long long>(C), need, kScratchBytes,
-                    (kScratchBytes - kHeader - 256) / (8 + 2 * per_tile_floats * sizeof(float)),
-                    kTileSteps);
+                    static_cast<long long>(C), need, kScratchBytes, kMaxTiles, kTileSteps);
 
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -209,18 +205,17 @@ extern "C" wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const
     Workspace ws;
     std::memset(&ws, 0, sizeof ws);
     if (need > 0) {
-        // the array keeps the last call's contents: start counters, status and
-        // this call's flags from zero (a memset, not an allocation)
+        // the array keeps the last call's contents: start the counters, the
+        // status word and this call's records from zero (a memset, not an
+        // allocation), so nothing a previous call left behind can be read
         unsigned char *base = slot.scratch;
-        e = cudaMemsetAsync(base, 0, kHeader + flags_bytes, stream);
+        e = cudaMemsetAsync(base, 0, need, stream);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scratch)");
         ws.ticket = reinterpret_cast<unsigned int *>(base);
         ws.done = reinterpret_cast<unsigned int *>(base + 4);
         ws.epoch = reinterpret_cast<unsigned long long *>(base + 8);
         ws.status = reinterpret_cast<int *>(base + 16);
-        ws.flags = reinterpret_cast<unsigned long long *>(base + kHeader);
-        ws.agg = reinterpret_cast<float *>(base + kHeader + flags_bytes);
-        ws.incl = ws.agg + static_cast<size_t>(tiles) * per_tile_floats;
+        ws.records = reinterpret_cast<uint4 *>(base + kHeader);
     }
 
     CUtensorMap maps[3];

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             s_last_it[s] = -1;
         }
         fence_mbar_init();
-        s_epoch = chained ? ld_relaxed_gpu_u64(ws.epoch) : 0ull;
+        s_epoch = chained ? epoch_of(ws) : 0ull;
         s_abort = 0;
     }
     __syncthreads();
@@ -206,11 +206,17 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                 State agg[CPT], X[CPT];
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) {
+                    // fold the warps' summaries in time order; each slot is
+                    // overwritten with its warp's exclusive prefix (the fold of
+                    // the sub-chunks before it) for pass 2
                     agg[j] = Op::identity();
                     for (int w = 0; w < NWG; ++w) {
                         float vals[NV];
+                        float *slot = g_sum + w * NV * CG + lane * CPT + j;
 #pragma unroll
-                        for (int q = 0; q < NV; ++q) vals[q] = g_sum[(w * NV + q) * CG + lane * CPT + j];
+                        for (int q = 0; q < NV; ++q) vals[q] = slot[q * CG];
+#pragma unroll
+                        for (int q = 0; q < NV; ++q) slot[q * CG] = Op::get(agg[j], q);
                         const int len = max(0, min(LS, g.T - (t0 + w * LS)));
                         agg[j] = Op::combine(agg[j], Op::make(vals), static_cast<float>(len), prm[j]);
                     }
@@ -223,13 +229,13 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
 #pragma unroll
                         for (int j = 0; j < CPT; ++j)
                             inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                        publish<Op, CG>(ws.incl, ws.flags, tile, inc, (epoch << 2) | kFlagIncl, lane);
+                        publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
                     } else {
                         if (!last)
-                            publish<Op, CG>(ws.agg, ws.flags, tile, agg, (epoch << 2) | kFlagAgg, lane);
+                            publish<Op, CG>(ws, tile, agg, kFlagAgg, epoch, lane);
                         State run[CPT];
                         if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run)) {
-                            if (lane == 0) atomicExch(ws.status, kStatusTimeout);
+                            atomicExch(ws.status, kStatusTimeout);  // this lane gave up
 #pragma unroll
                             for (int j = 0; j < CPT; ++j) run[j] = Op::nan_state();
                         }
@@ -240,8 +246,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
 #pragma unroll
                             for (int j = 0; j < CPT; ++j)
                                 inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                            publish<Op, CG>(ws.incl, ws.flags, tile, inc, (epoch << 2) | kFlagIncl,
-                                            lane);
+                            publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
                         }
                     }
                 }
@@ -261,10 +266,10 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
 #pragma unroll
                     for (int q = 0; q < NV; ++q) vals[q] = g_carry[q * CG + lane * CPT + j];
                     cur[j] = Op::make(vals);
-                    for (int w = 0; w < wg; ++w) {  // earlier sub-chunks are all full
+                    if (wg > 0) {  // the sub-chunks before this warp's, all full
 #pragma unroll
-                        for (int q = 0; q < NV; ++q) vals[q] = g_sum[(w * NV + q) * CG + lane * CPT + j];
-                        cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(LS), prm[j]);
+                        for (int q = 0; q < NV; ++q) vals[q] = g_sum[(wg * NV + q) * CG + lane * CPT + j];
+                        cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(wg * LS), prm[j]);
                     }
                 }
                 Op::template sweep<LS>(cur, p0, p1, nval, prm, sc, p0, CG, true);

@@ -119,6 +119,23 @@ __device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned 
     return v;
 }
 
+// 16-byte record accesses: one aligned vector access each, so a reader sees a
+// record either entirely before or entirely after a writer's store
+__device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const uint4 *p) {
+    uint4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu_v4(uint4 *p, uint4 v) {
+    asm volatile("st.relaxed.gpu.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ float ld_relaxed_gpu(const float *p) {
     float v;
     asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");

@@ -7,6 +7,14 @@
 // state) as soon as it has it, looks back over its predecessors for the state
 // before itself, and publishes the state after itself (Merrill & Garland,
 // "Single-pass Parallel Prefix Scan with Decoupled Look-back").
+//
+// What is published is one 16-byte record per (tile, channel): two state
+// floats and a 64-bit tag, written and read with single aligned vector
+// accesses.  The tag says whether the record holds the aggregate or the state
+// after the tile, carries the launch's epoch (so records left by earlier
+// launches never read as current) and 16 bits the operation may use to
+// complete its state.  A record is self-contained: no fence orders it against
+// anything else, and one load both polls and reads it.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -16,25 +24,22 @@
 
 namespace wkvb {
 
-constexpr uint32_t kFlagAgg = 1u;   // tile aggregate published
-constexpr uint32_t kFlagIncl = 2u;  // state after the tile published
+constexpr uint32_t kFlagAgg = 1u;   // record holds the tile aggregate
+constexpr uint32_t kFlagIncl = 2u;  // record holds the state after the tile
 constexpr int kStatusTimeout = 4;   // == WKV_ERR_TIMEOUT
+constexpr int kEpochBits = 46;      // tag: epoch(46) | op bits(16) | flag(2)
 
-// Device pointers of one look-back workspace.  The three counters live in
-// the workspace itself, so a launch needs no per-launch host state (CUDA-graph
+// Device pointers of one look-back workspace.  The counters live in the
+// workspace itself, so a launch needs no per-launch host state (CUDA-graph
 // replays stay correct): blocks take tile tickets from `ticket`; the last
-// block to finish resets `ticket` and `done` and advances `epoch`, which tags
-// every flag this launch publishes so flags left by earlier launches never
-// read as ready.  Launches sharing a workspace must run one after another
-// (same stream).
+// block to finish resets `ticket` and `done` and advances `epoch`.  Launches
+// sharing a workspace must run one after another (same stream).
 struct Workspace {
     unsigned int *ticket;        // next tile ticket of the running launch
     unsigned int *done;          // blocks of the running launch that finished
     unsigned long long *epoch;   // launches completed on this workspace
     int *status;                 // device status word, 0 or an error code
-    unsigned long long *flags;   // [tiles] (epoch << 2) | kFlag*
-    float *agg;                  // [tiles][NV][CG] tile aggregates
-    float *incl;                 // [tiles][NV][CG] states after each tile
+    uint4 *records;              // [tiles][CG] published states
 };
 
 struct Geometry {
@@ -42,9 +47,9 @@ struct Geometry {
     int n_cg;              // channel groups per row, ceil(C / CG)
     int n_seg;             // time segments per row, ceil(T / LT)
     int tiles_per_seg;     // B * n_cg
-    int tiles;             // n_seg * tiles_per_seg == gridDim.x
+    int tiles;             // n_seg * tiles_per_seg
     int use_tma;           // 1: TMA tile copies; 0: element-wise copies
-    long long spin_limit;  // polls of a predecessor's flag before giving up
+    long long spin_limit;  // polls of one predecessor record before giving up
 };
 
 template <typename io_t>
@@ -56,20 +61,31 @@ __device__ __forceinline__ __nv_bfloat16 io_zero<__nv_bfloat16>() {
     return __float2bfloat16_rn(0.f);
 }
 
-// ---- publishing a per-tile value for the look-back -------------------------
+__device__ __forceinline__ unsigned long long epoch_of(const Workspace &ws) {
+    return ld_relaxed_gpu_u64(ws.epoch) & ((1ull << kEpochBits) - 1ull);
+}
+
+// Publish this lane's CPT channels of `tile` with the given flag.
 template <class Op, int CG>
-__device__ __forceinline__ void publish(float *base, unsigned long long *flags, int tile,
-                                        const typename Op::State (&val)[Op::CPT],
-                                        unsigned long long flag, int lane) {
-    float *dst = base + static_cast<size_t>(tile) * Op::NV * CG;
+__device__ __forceinline__ void publish(const Workspace &ws, int tile,
+                                        const typename Op::State (&val)[Op::CPT], uint32_t flag,
+                                        unsigned long long epoch, int lane) {
+    uint4 *dst = ws.records + static_cast<size_t>(tile) * CG + lane * Op::CPT;
 #pragma unroll
-    for (int j = 0; j < Op::CPT; ++j)
-#pragma unroll
-        for (int q = 0; q < Op::NV; ++q)
-            st_relaxed_gpu(dst + q * CG + lane * Op::CPT + j, Op::get(val[j], q));
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release_gpu_u64(flags + tile, flag);
+    for (int j = 0; j < Op::CPT; ++j) {
+        float x, y;
+        uint32_t bits16;
+        Op::pack(val[j], x, y, bits16);
+        const unsigned long long tag =
+            (epoch << 18) | (static_cast<unsigned long long>(bits16 & 0xffffu) << 2) | flag;
+        st_relaxed_gpu_v4(dst + j, make_uint4(__float_as_uint(x), __float_as_uint(y),
+                                              static_cast<uint32_t>(tag),
+                                              static_cast<uint32_t>(tag >> 32)));
+    }
+}
+
+__device__ __forceinline__ unsigned long long record_tag(uint4 r) {
+    return (static_cast<unsigned long long>(r.w) << 32) | r.z;
 }
 
 // Count this block as finished; the last of the `blocks` increments a
@@ -92,93 +108,67 @@ __device__ __forceinline__ void finish_launch(const Workspace &ws, bool chained,
     }
 }
 
-// Decoupled look-back for one tile, run by one warp.  The tiles before this
-// one in time are tile - S, tile - 2S, ... (S = tiles per time segment).
-// Lanes poll the flags of a window of 32 predecessors at once; the window is
-// folded (newest first, lanes now acting as channels) up to the nearest
-// predecessor that has published the state after itself, or entirely when
-// all 32 have published only their aggregates, in which case the next window
-// follows.  Returns false if a flag never appeared within the poll budget.
+// Decoupled look-back for one tile, each lane for its own CPT channels.  The
+// tiles before this one in time are tile - S, tile - 2S, ... (S = tiles per
+// time segment).  A lane folds its channel's records newest first -- a tile
+// aggregate moves the fold one tile further back, a state-after-tile ends it
+// -- prefetching several hops' records with independent loads.  Lanes may
+// stop at different hops; each ends with the state before this tile.
+// Returns false (in every lane that gave up) if a record never appeared
+// within the poll budget.
 template <class Op, int LT>
 __device__ __forceinline__ bool lookback(const Workspace &ws, const Geometry &g, int tile,
                                          unsigned long long epoch,
                                          const typename Op::Param (&prm)[Op::CPT], int lane,
                                          typename Op::State (&run)[Op::CPT]) {
-    constexpr int CPT = Op::CPT, NV = Op::NV, CG = 32 * CPT;
-    const int S = g.tiles_per_seg;
+    constexpr int CPT = Op::CPT, CG = 32 * CPT, HB = 4;  // hops per batch of loads
+    const long long S = g.tiles_per_seg;
+    bool ok = true;
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) run[j] = Op::identity();
-    float run_len = 0.f;
-    int base = tile;
-    while (true) {
-        const long long q = static_cast<long long>(base) - static_cast<long long>(lane + 1) * S;
-        const bool exists = q >= 0;  // this lane's predecessor in time
-        unsigned long long f = 0;
-        bool rdy = false;
-        int last = -1;        // fold lanes 0..last
-        bool found = false;   // lane `last` holds a state-after-tile
-        long long polls = 0;
-        while (true) {
-            if (exists && !rdy) {
-                f = ld_acquire_gpu_u64(ws.flags + q);
-                rdy = (f >> 2) == epoch && (f & 3u) != 0u;
+    for (int j = 0; j < CPT; ++j) {
+        run[j] = Op::identity();
+        float run_len = 0.f;
+        long long base = tile;
+        bool done = false;
+        while (!done && ok) {
+            uint4 rec[HB];
+#pragma unroll
+            for (int i = 0; i < HB; ++i) {
+                const long long q = base - (i + 1) * S;
+                rec[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (q >= 0)
+                    rec[i] = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
             }
-            const unsigned rdym = __ballot_sync(0xffffffffu, rdy);
-            const unsigned incm = __ballot_sync(0xffffffffu, rdy && (f & 3u) == kFlagIncl);
-            const unsigned exm = __ballot_sync(0xffffffffu, exists);
-            if (incm != 0u) {
-                const int h = __ffs(incm) - 1;
-                const unsigned need = h == 31 ? 0xffffffffu : ((1u << (h + 1)) - 1u);
-                if ((rdym & need) == need) {
-                    last = h;
-                    found = true;
+#pragma unroll
+            for (int i = 0; i < HB; ++i) {
+                if (done || !ok) break;
+                const long long q = base - (i + 1) * S;
+                if (q < 0) {  // cannot happen: first-segment tiles always end the fold
+                    ok = false;
                     break;
                 }
-            } else if (exm == 0xffffffffu && rdym == 0xffffffffu) {
-                last = 31;  // 32 aggregates, none final yet: fold them, look further
-                break;
-            }
-            if (++polls > g.spin_limit) return false;
-            __nanosleep(32);
-        }
-        // every lane fences after its own acquire, so data published before
-        // any of the observed flags is visible to the whole warp
-        __syncwarp();
-        __threadfence();
-        // fold the window newest-first; the loads of several hops are issued
-        // together so a window costs a few memory latencies, not one per hop
-        constexpr int HB = 8 / CPT;  // hops per batch of loads
-        for (int h0 = 0; h0 <= last; h0 += HB) {
-            float vals[HB][CPT][NV];
-#pragma unroll
-            for (int hh = 0; hh < HB; ++hh) {
-                const int h = h0 + hh;
-                const unsigned long long fh = __shfl_sync(0xffffffffu, f, h & 31);
-                if (h <= last) {
-                    const long long qh =
-                        static_cast<long long>(base) - static_cast<long long>(h + 1) * S;
-                    const float *src = ((fh & 3u) == kFlagIncl ? ws.incl : ws.agg) +
-                                       static_cast<size_t>(qh) * NV * CG;
-#pragma unroll
-                    for (int j = 0; j < CPT; ++j)
-#pragma unroll
-                        for (int v = 0; v < NV; ++v)
-                            vals[hh][j][v] = ld_relaxed_gpu(src + v * CG + lane * CPT + j);
+                uint4 r = rec[i];
+                long long polls = 0;
+                while (((record_tag(r) >> 18) != epoch) || (record_tag(r) & 3u) == 0u) {
+                    if (++polls > g.spin_limit) {
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(32);
+                    r = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
                 }
+                if (!ok) break;
+                const unsigned long long tag = record_tag(r);
+                const typename Op::State val = Op::unpack(
+                    __uint_as_float(r.x), __uint_as_float(r.y), static_cast<uint32_t>(tag >> 2) & 0xffffu);
+                run[j] = Op::combine(val, run[j], run_len, prm[j]);
+                run_len += static_cast<float>(LT);
+                done = (tag & 3u) == kFlagIncl;
             }
-#pragma unroll
-            for (int hh = 0; hh < HB; ++hh) {
-                if (h0 + hh <= last) {
-#pragma unroll
-                    for (int j = 0; j < CPT; ++j)
-                        run[j] = Op::combine(Op::make(vals[hh][j]), run[j], run_len, prm[j]);
-                    run_len += static_cast<float>(LT);
-                }
-            }
+            base -= HB * S;
         }
-        if (found) return true;
-        base -= 32 * S;  // all 32 existed, so base - 32 S >= 0
     }
+    return ok;
 }
 
 }  // namespace wkvb

@@ -134,6 +134,22 @@ struct WkvOp {
     }
     __device__ __forceinline__ static State make(const float (&v)[NV]) { return {v[0], v[1], v[2]}; }
 
+    // a published state in two floats: rescaled to the integer log-scale
+    // ceil(p), which travels in the record's 16 spare tag bits (published
+    // states are never empty, so p is finite; |p| beyond 32767 is clamped,
+    // inputs that large are outside the operator's domain anyway)
+    __device__ __forceinline__ static void pack(const State &s, float &x, float &y,
+                                                uint32_t &bits16) {
+        const float pi = fminf(fmaxf(ceilf(s.p), -32768.f), 32767.f);
+        const float f = expf(s.p - pi);
+        x = s.a * f;
+        y = s.b * f;
+        bits16 = static_cast<uint32_t>(static_cast<int>(pi) + 32768);
+    }
+    __device__ __forceinline__ static State unpack(float x, float y, uint32_t bits16) {
+        return {x, y, static_cast<float>(static_cast<int>(bits16) - 32768)};
+    }
+
     __device__ __forceinline__ static State combine(const State &l, const State &r, float r_len,
                                                     const Param &q) {
         const float pd = fmaf(-r_len, q.w, l.p);
@@ -334,6 +350,13 @@ struct ScanOp {
     }
     __device__ __forceinline__ static float get(const State &s, int q) { return q == 0 ? s.A : s.H; }
     __device__ __forceinline__ static State make(const float (&v)[NV]) { return {v[0], v[1]}; }
+    __device__ __forceinline__ static void pack(const State &s, float &x, float &y,
+                                                uint32_t &bits16) {
+        x = s.A;
+        y = s.H;
+        bits16 = 0u;
+    }
+    __device__ __forceinline__ static State unpack(float x, float y, uint32_t) { return {x, y}; }
     __device__ __forceinline__ static State combine(const State &l, const State &r, float,
                                                     const Param &) {
         return {l.A * r.A, fmaf(r.A, l.H, r.H)};

@@ -56,7 +56,7 @@ def test_noalloc_matches_allocating_entry_point_twice(lib, B, T, C):
 
 
 def test_noalloc_rejects_a_problem_beyond_its_scratch(lib):
-    # 1 x 4096 x 40960: 1280 channel groups x 32 tiles in time = 40960 tiles > 21619
+    # 1 x 4096 x 40960: 1280 channel groups x 32 tiles in time = 40960 tiles > 32767
     B, T, C = 1, 4096, 40960
     k = torch.zeros(B, T, C, device="cuda")
     w = torch.zeros(C, device="cuda")
