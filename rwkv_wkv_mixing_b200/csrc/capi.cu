@@ -341,10 +341,24 @@ wkv_status launch_persistent(const typename Op::Args &args, int64_t B, int64_t T
     static std::atomic<uint64_t> configured{0};
     if ((st = configure_once(kern, Cfg::kSmemBytes, dev, configured)) != WKV_OK) return st;
     const int grid = std::min(p.g.tiles, sm_count(dev));
+    // programmatic dependent launch: this grid's blocks may be scheduled while
+    // the previous grid in the stream drains; the kernel reads no global
+    // memory before griddepcontrol.wait
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     cudaGetLastError();
-    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(
-        p.maps[0], p.maps[1], p.maps[2], args, p.g, p.ws);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err =
+        cudaLaunchKernelEx(&cfg, kern, p.maps[0], p.maps[1], p.maps[2], args, p.g, p.ws);
+    if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     return WKV_OK;
 }

@@ -67,6 +67,29 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volat
     }
 }
 
+// Wait until `bar` has completed the phase that delivers ring iteration `it`
+// into its stage.  Stages are shared by consumer groups, so a fast group can
+// start waiting while the barrier still runs a phase two fills back, whose
+// parity is the same as the one wanted; the stage's fill stamp (written by
+// the producer before it arms the phase) tells the phases apart.
+__device__ __forceinline__ bool wait_fill(uint64_t *bar, const int *fill_it, int it,
+                                          uint32_t parity, volatile int *abort_flag,
+                                          const Workspace &ws) {
+    const volatile int *stamp = fill_it;
+    const unsigned long long t0 = global_timer_ns();
+    for (unsigned n = 0;; ++n) {
+        if (*stamp == it && mbar_try_wait(bar, parity)) return true;
+        if ((n & 63u) == 63u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kBarrierWaitNs) {
+                *abort_flag = 1;
+                if (ws.status != nullptr) atomicExch(ws.status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
 template <class Op, int LT, int NWG, int NC, int NSTAGE>
 __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThreads, 1)
     persistent_scan_kernel(const __grid_constant__ CUtensorMap map_x0,
@@ -86,6 +109,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
     __shared__ __align__(8) uint64_t full_bar[NSTAGE];
     __shared__ __align__(8) uint64_t empty_bar[NSTAGE];
     __shared__ int s_meta[NSTAGE];      // tile id per stage, -1 = no more tiles
+    __shared__ int s_fill_it[NSTAGE];   // ring iteration the stage was last filled for
     __shared__ int s_last_it[NSTAGE];   // last ring iteration loaded into each stage
     __shared__ int s_gtile[NC];         // each group's current tile, as its leader saw it
     __shared__ unsigned long long s_epoch;
@@ -99,11 +123,16 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
             s_last_it[s] = -1;
+            s_fill_it[s] = -1;
         }
         fence_mbar_init();
-        s_epoch = chained ? epoch_of(ws) : 0ull;
         s_abort = 0;
     }
+    // everything above touched only shared memory; with a programmatic
+    // dependency on the previous grid in the stream, nothing global is read
+    // before that grid has finished
+    grid_dependency_wait();
+    if (threadIdx.x == 0) s_epoch = chained ? epoch_of(ws) : 0ull;
     __syncthreads();
     const unsigned long long epoch = s_epoch;
     volatile int *abort_flag = &s_abort;
@@ -132,6 +161,10 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                     }
                 }
                 s_meta[s] = tile;
+                // stamped before the arrive that releases it: a consumer only
+                // accepts a completed phase of this stage when the stamp
+                // names its own iteration
+                *static_cast<volatile int *>(&s_fill_it[s]) = it;
                 if (tile < 0) {
                     ++sentinels;
                     mbar_arrive(&full_bar[s]);
@@ -163,7 +196,9 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             // the group leader alone decides whether the stage arrived, so the
             // whole group leaves (or stays in) the loop together
             if (gtid == 0)
-                s_gtile[grp] = wait_phase(&full_bar[s], parity, abort_flag, ws) ? s_meta[s] : -2;
+                s_gtile[grp] = wait_fill(&full_bar[s], &s_fill_it[s], it, parity, abort_flag, ws)
+                                   ? s_meta[s]
+                                   : -2;
             named_bar_sync(bar_id, NWG * 32);
             const int tile = s_gtile[grp];
             if (tile < 0) break;
@@ -302,6 +337,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             }
         }
     }
+    allow_dependent_launch();
     finish_launch(ws, chained, static_cast<int>(threadIdx.x), gridDim.x);
 }
 

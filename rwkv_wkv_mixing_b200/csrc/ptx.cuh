@@ -47,6 +47,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// ---- programmatic dependent launch ----------------------------------------------
+// wait until the grids this one depends on have completed and their memory
+// is visible (a no-op when launched without a programmatic dependency)
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// let the next grid in the stream start launching its blocks
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- named barriers and timers ----------------------------------------------
 // non-.aligned form: threads of one warp may arrive at different times
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -390,3 +390,37 @@ def test_persistent_and_blockwise_kernels_agree(m):
         m.wkv_set_tile_steps(old)
     for steps, got in outs.items():
         assert_close(got, want, 2e-2 * np.abs(x.v).max(), f"bf16 tile steps {steps}")
+
+
+# ---------------------------------------------------------------------------
+# many launches queued back to back: the persistent pipeline's stage hand-off
+# and the look-back counters must hold up launch after launch
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("op", ["wkv", "wkv_bf16", "scan"])
+def test_many_back_to_back_launches(m, op):
+    n_out, n_launch = 32, 256
+    if op == "scan":
+        x = workloads.make_scan("scan_mingru", B=8, T=2048, D=256, seed=71)
+        a, b = dev(x.a), dev(x.b)
+        want = torch.from_numpy(oracle.scan_rnn(x.a, x.b, None)).to("cuda")
+        tol = 1e-5 * float(want.abs().max())
+        outs = [torch.empty_like(a) for _ in range(n_out)]
+        for i in range(n_launch):
+            m.diag_scan(a, b, None, h=outs[i % n_out])
+    else:
+        name = "wkv_3b_bf16" if op == "wkv_bf16" else "wkv_169m"
+        x = workloads.make_wkv(name, B=4, T=2048, C=256, seed=72)
+        w, u = dev(x.w), dev(x.u)
+        if op == "wkv_bf16":
+            k, v = bf16_dev(x.k_bits), bf16_dev(x.v_bits)
+            fn, tol = m.wkv_forward_bf16, 2e-2 * float(np.abs(x.v).max())
+        else:
+            k, v = dev(x.k), dev(x.v)
+            fn, tol = m.wkv_forward, wkv_tol(2048, float(np.abs(x.v).max()))
+        want = torch.from_numpy(oracle.wkv_rnn(x.w, x.u, x.k, x.v)).to("cuda")
+        outs = [torch.empty_like(k) for _ in range(n_out)]
+        for i in range(n_launch):
+            fn(w, u, k, v, y=outs[i % n_out])
+    m.wkv_device_status()
+    worst = max(float((o.double() - want).abs().max()) for o in outs)
+    assert worst <= tol, f"{op}: worst max err over {n_out} outputs {worst} > {tol}"
