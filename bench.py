@@ -66,7 +66,7 @@ def parse_args(argv=None):
                     help="untimed steps before the timed region, so clocks settle")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="budget of the CPU-oracle baseline (rank 0, N=1)")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -340,40 +340,49 @@ def host_overhead_us(torch, wl, n=200):
 
 
 def e2e_leg(torch, wl, steps):
-    """Through the C ABI with host buffers: pinned host inputs are copied to
-    the device, the library runs, the result is copied back, every step."""
+    """Through the C ABI with host buffers: every step is one call of the
+    library's host-buffer entry point on pinned host memory, which uploads the
+    step's inputs, computes and downloads the result (overlapped in chunks)
+    and returns when the result is on the host.  Timed with CUDA events on the
+    current stream around the synchronous calls."""
+    lib = wl.lib
     hx0 = torch.from_numpy(np.ascontiguousarray(wl.host["x0"])).pin_memory()
     hx1 = torch.from_numpy(np.ascontiguousarray(wl.host["x1"])).pin_memory()
-    if wl.dtype == "bf16":
-        hx0, hx1 = hx0.view(torch.bfloat16), hx1.view(torch.bfloat16)
     hy = torch.empty_like(hx0).pin_memory()
     hp = [p.cpu().pin_memory() for p in wl.params]
-    dx0, dx1, dy = wl.sets[0]
+    if wl.is_scan:
+        api = "diag_scan_host"
+        call = lambda: lib.diag_scan_host(wl.B, wl.T, wl.C, hx0.data_ptr(), hx1.data_ptr(),  # noqa: E731
+                                          None, hy.data_ptr())
+    else:
+        api = "wkv_forward_bf16_host" if wl.dtype == "bf16" else "wkv_forward_host"
+        fn = getattr(lib, api)
+        call = lambda: fn(wl.B, wl.T, wl.C, hp[0].data_ptr(), hp[1].data_ptr(),  # noqa: E731
+                          hx0.data_ptr(), hx1.data_ptr(), hy.data_ptr())
 
     def one():
-        for h, d in zip(hp, wl.params):
-            d.copy_(h, non_blocking=True)
-        dx0.copy_(hx0, non_blocking=True)
-        dx1.copy_(hx1, non_blocking=True)
-        st = wl.call(dx0, dx1, dy)
+        st = call()
         if st != 0:
-            raise RuntimeError("library call failed")
-        hy.copy_(dy, non_blocking=True)
+            raise RuntimeError(f"{api} failed: {st}: {lib.wkv_last_error().decode()}")
 
-    for _ in range(3):
+    for _ in range(2):
         one()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(wl.stream)
+    stream = torch.cuda.current_stream()
+    t0 = time.perf_counter()
+    a.record(stream)
     for _ in range(steps):
         one()
-    b.record(wl.stream)
+    b.record(stream)
     b.synchronize()
+    wall_ms = (time.perf_counter() - t0) / steps * 1e3
     ms = a.elapsed_time(b) / steps
     h2d = hx0.numel() * hx0.element_size() * 2 + wl.param_bytes
     d2h = hy.numel() * hy.element_size()
     return {"value": wl.elements / (ms / 1e3), "unit": "elem/s", "ms_per_step": ms,
-            "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "wall_ms_per_step": wall_ms, "steps": steps, "api": api,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "host_buffers": "pinned"}
 
 

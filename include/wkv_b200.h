@@ -130,6 +130,28 @@ WKV_API wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C,
                                        const float *k, const float *v, float *y,
                                        cudaStream_t stream);
 
+/* The same three operations on HOST buffers (every pointer, w/u/h0 included,
+ * is host memory; NULL h0 = zeros).  The call copies the inputs to the
+ * device, runs the kernel and copies the outputs back, and returns when they
+ * are in the output buffer (synchronous; no stream argument).  The work is cut
+ * into up to 8 independent chunks -- batch rows, or 64-channel-aligned channel
+ * slices when B is 1 -- pipelined over three internal streams so the uploads of
+ * one chunk overlap the compute and download of another.  Page-locked host
+ * memory (cudaHostAlloc / cudaHostRegister) gives full overlap; pageable memory
+ * works but its copies are staged by the driver.  The library allocates device
+ * staging (three chunks of inputs, outputs and parameters) on first use and
+ * grows it on demand.  Calls are serialised across host threads.  Returns
+ * WKV_ERR_TIMEOUT if a device-side wait gave up during the call. */
+WKV_API wkv_status wkv_forward_host(int64_t B, int64_t T, int64_t C,
+                                    const float *w, const float *u,
+                                    const float *k, const float *v, float *y);
+WKV_API wkv_status wkv_forward_bf16_host(int64_t B, int64_t T, int64_t C,
+                                         const float *w, const float *u,
+                                         const wkv_bf16_t *k, const wkv_bf16_t *v,
+                                         wkv_bf16_t *y);
+WKV_API wkv_status diag_scan_host(int64_t B, int64_t T, int64_t D,
+                                  const float *a, const float *b, const float *h0, float *h);
+
 /* Synchronise `stream`, then return and clear the device status word of that
  * stream's workspace: WKV_OK, or WKV_ERR_TIMEOUT if a device-side wait gave up
  * since the last query.  WKV_ERR_CUDA if the synchronisation itself failed. */
@@ -148,6 +170,16 @@ WKV_API wkv_status wkv_release_workspaces(void);
  * combined.  WKV_ERR_INVALID_ARG for any other value. */
 WKV_API wkv_status wkv_set_tile_steps(int steps);
 WKV_API int wkv_get_tile_steps(void);
+
+/* Test hook for failure detection, process-wide, for later launches of the
+ * allocating entry points.  skip_tile >= 0: that tile (in the launch's
+ * ticket numbering) never publishes its state, so the bounded look-back waits
+ * of the tiles after it in time run out; spin_limit > 0 replaces the number
+ * of polls a wait makes before giving up (0 restores the default, about a
+ * second).  The outcome is WKV_ERR_TIMEOUT from wkv_device_status and NaN in
+ * the affected outputs; the context stays usable.  (-1, 0) turns it off.
+ * WKV_ERR_INVALID_ARG for skip_tile < -1 or spin_limit < 0. */
+WKV_API wkv_status wkv_set_fault_injection(int skip_tile, long long spin_limit);
 
 #ifdef __cplusplus
 }

@@ -10,6 +10,7 @@ raises if the library has not been built.
     y = wkv_forward(w, u, k, v)            # fp32 [B,T,C] k, v; [C] w, u
     y = wkv_forward_bf16(w, u, k, v)       # bf16 k, v -> bf16 y, fp32 state
     h = diag_scan(a, b, h0=None)           # fp32 [B,T,D]; h0 [B,D] or None
+    y = wkv_forward_host(w, u, k, v)       # the same on CPU tensors, copies overlapped
 """
 from __future__ import annotations
 
@@ -39,11 +40,15 @@ _SIGS = {
     "wkv_forward_bf16": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_noalloc": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "diag_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_bf16_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
+    "diag_scan_host": ([_i64, _i64, _i64, _p, _p, _p, _p], _i32),
     "wkv_device_status": ([_p], _i32),
     "wkv_last_error": ([], ctypes.c_char_p),
     "wkv_release_workspaces": ([], _i32),
     "wkv_set_tile_steps": ([_i32], _i32),
     "wkv_get_tile_steps": ([], _i32),
+    "wkv_set_fault_injection": ([_i32, _i64], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -151,6 +156,79 @@ def diag_scan(a, b, h0=None, h=None, stream=None):
     return h
 
 
+def _need_host(t, name, dtype, ndim):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a CPU tensor (pinned for overlapped copies)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _wkv_host(fn_name, io_dtype, w, u, k, v, y):
+    import torch
+    _need_host(k, "k", io_dtype, 3)
+    _need_host(v, "v", io_dtype, 3)
+    _need_host(w, "w", torch.float32, 1)
+    _need_host(u, "u", torch.float32, 1)
+    if k.shape != v.shape:
+        raise ValueError("k and v must have one shape")
+    B, T, C = k.shape
+    if w.shape[0] != C or u.shape[0] != C:
+        raise ValueError("w and u must be [C]")
+    if y is None:
+        y = torch.empty_like(k, pin_memory=k.is_pinned())
+    else:
+        _need_host(y, "y", io_dtype, 3)
+        if y.shape != k.shape:
+            raise ValueError("y must have the shape of k")
+    _check(getattr(lib, fn_name)(B, T, C, w.data_ptr(), u.data_ptr(), k.data_ptr(),
+                                 v.data_ptr(), y.data_ptr()), fn_name)
+    return y
+
+
+def wkv_forward_host(w, u, k, v, y=None):
+    """WKV forward, fp32, on host (CPU) tensors: uploads, computes and
+    downloads in an overlapped pipeline; returns when y holds the result."""
+    import torch
+    return _wkv_host("wkv_forward_host", torch.float32, w, u, k, v, y)
+
+
+def wkv_forward_bf16_host(w, u, k, v, y=None):
+    """WKV forward, bf16 k/v/y on host tensors (fp32 w, u)."""
+    import torch
+    return _wkv_host("wkv_forward_bf16_host", torch.bfloat16, w, u, k, v, y)
+
+
+def diag_scan_host(a, b, h0=None, h=None):
+    """Diagonal scan on host (CPU) tensors, pipelined; returns h."""
+    import torch
+    _need_host(a, "a", torch.float32, 3)
+    _need_host(b, "b", torch.float32, 3)
+    if a.shape != b.shape:
+        raise ValueError("a and b must have one shape")
+    B, T, D = a.shape
+    if h0 is not None:
+        _need_host(h0, "h0", torch.float32, 2)
+        if tuple(h0.shape) != (B, D):
+            raise ValueError("h0 must be [B, D]")
+    if h is None:
+        h = torch.empty_like(a, pin_memory=a.is_pinned())
+    else:
+        _need_host(h, "h", torch.float32, 3)
+        if h.shape != a.shape:
+            raise ValueError("h must have the shape of a")
+    _check(lib.diag_scan_host(B, T, D, a.data_ptr(), b.data_ptr(),
+                              None if h0 is None else h0.data_ptr(), h.data_ptr()),
+           "diag_scan_host")
+    return h
+
+
 def wkv_device_status(stream=None):
     """Synchronise the stream; raise WkvError if a device-side wait gave up."""
     _check(lib.wkv_device_status(_stream_handle(stream)), "wkv_device_status")
@@ -172,6 +250,14 @@ def wkv_get_tile_steps() -> int:
     return int(lib.wkv_get_tile_steps())
 
 
-__all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan", "wkv_device_status",
+def wkv_set_fault_injection(skip_tile: int = -1, spin_limit: int = 0):
+    """Test hook: make tile `skip_tile` never publish (its successors' bounded
+    waits run out after `spin_limit` polls); (-1, 0) turns it off."""
+    _check(lib.wkv_set_fault_injection(int(skip_tile), int(spin_limit)),
+           "wkv_set_fault_injection")
+
+
+__all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan",
+           "wkv_forward_host", "wkv_forward_bf16_host", "diag_scan_host", "wkv_device_status",
            "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
            "wkv_get_tile_steps", "WkvError", "lib", "LIB_PATH"]

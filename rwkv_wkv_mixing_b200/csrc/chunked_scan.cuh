@@ -184,10 +184,10 @@ __global__ void __launch_bounds__(NW * 32, 3)
 #pragma unroll
                 for (int j = 0; j < CPT; ++j)
                     inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
+                publish<Op, CG>(ws, g, tile, inc, kFlagIncl, epoch, lane);
             } else {
                 if (!last)
-                    publish<Op, CG>(ws, tile, agg, kFlagAgg, epoch, lane);
+                    publish<Op, CG>(ws, g, tile, agg, kFlagAgg, epoch, lane);
                 // decoupled look-back over the tiles before this one in time
                 State run[CPT];
                 if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run)) {
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(NW * 32, 3)
 #pragma unroll
                     for (int j = 0; j < CPT; ++j)
                         inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                    publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
+                    publish<Op, CG>(ws, g, tile, inc, kFlagIncl, epoch, lane);
                 }
             }
         }

@@ -201,6 +201,7 @@ extern "C" wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const
     g.tiles_per_seg = static_cast<int>(B * n_cg);
     g.tiles = static_cast<int>(tiles);
     g.spin_limit = 1ll << 21;
+    g.skip_publish = -1;
 
     Workspace ws;
     std::memset(&ws, 0, sizeof ws);

@@ -264,10 +264,10 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
 #pragma unroll
                         for (int j = 0; j < CPT; ++j)
                             inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                        publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
+                        publish<Op, CG>(ws, g, tile, inc, kFlagIncl, epoch, lane);
                     } else {
                         if (!last)
-                            publish<Op, CG>(ws, tile, agg, kFlagAgg, epoch, lane);
+                            publish<Op, CG>(ws, g, tile, agg, kFlagAgg, epoch, lane);
                         State run[CPT];
                         if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run)) {
                             atomicExch(ws.status, kStatusTimeout);  // this lane gave up
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
 #pragma unroll
                             for (int j = 0; j < CPT; ++j)
                                 inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                            publish<Op, CG>(ws, tile, inc, kFlagIncl, epoch, lane);
+                            publish<Op, CG>(ws, g, tile, inc, kFlagIncl, epoch, lane);
                         }
                     }
                 }

@@ -50,6 +50,7 @@ struct Geometry {
     int tiles;             // n_seg * tiles_per_seg
     int use_tma;           // 1: TMA tile copies; 0: element-wise copies
     long long spin_limit;  // polls of one predecessor record before giving up
+    int skip_publish;      // test hook: this tile publishes nothing (-1: none)
 };
 
 template <typename io_t>
@@ -65,11 +66,14 @@ __device__ __forceinline__ unsigned long long epoch_of(const Workspace &ws) {
     return ld_relaxed_gpu_u64(ws.epoch) & ((1ull << kEpochBits) - 1ull);
 }
 
-// Publish this lane's CPT channels of `tile` with the given flag.
+// Publish this lane's CPT channels of `tile` with the given flag.  (The
+// fault-injection test hook can name one tile that never publishes, so that
+// the look-back waits behind it run out.)
 template <class Op, int CG>
-__device__ __forceinline__ void publish(const Workspace &ws, int tile,
+__device__ __forceinline__ void publish(const Workspace &ws, const Geometry &g, int tile,
                                         const typename Op::State (&val)[Op::CPT], uint32_t flag,
                                         unsigned long long epoch, int lane) {
+    if (tile == g.skip_publish) return;
     uint4 *dst = ws.records + static_cast<size_t>(tile) * CG + lane * Op::CPT;
 #pragma unroll
     for (int j = 0; j < Op::CPT; ++j) {

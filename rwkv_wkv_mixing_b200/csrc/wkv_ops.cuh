@@ -159,11 +159,22 @@ struct WkvOp {
     }
 
     // ---- pass 1 ------------------------------------------------------------
+    // Exponent argument (x - r) in log2 units for ex2.  fp32 keeps the
+    // subtraction exact before scaling, so the error is a few ulp of |x - r|
+    // (small for the terms that matter); bf16 folds both into one FMA, whose
+    // error of about 2^-24 (|x| + |r|) is far below bf16 rounding.
+    __device__ __forceinline__ static float exp_arg(float x, float r, float r2) {
+        if constexpr (sizeof(IO) == 2)
+            return fmaf(x, kLog2e, -r2);
+        else
+            return (x - r) * kLog2e;
+    }
+
     template <int LS>
     __device__ __forceinline__ static void summarize(const IO *p0, const IO *p1, int n,
                                                      const Param (&q)[CPT], State (&out)[CPT],
                                                      Scratch (&sc)[CPT]) {
-        float m[CPT], kx[CPT], kn[CPT], a[CPT], b[CPT];
+        float m[CPT], m2[CPT], kx[CPT], kn[CPT], a[CPT], b[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
             m[j] = kNoScale;
@@ -184,6 +195,8 @@ struct WkvOp {
                     kn[j] = fminf(kn[j], k[j]);
                 }
             }
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) m2[j] = m[j] * kLog2e;
 #pragma unroll 8
             for (int i = 0; i < LS; ++i) {
                 float k[CPT], v[CPT];
@@ -192,7 +205,7 @@ struct WkvOp {
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) {
                     const float x = fmaf(static_cast<float>(i - (LS - 1)), q[j].w, k[j]);
-                    const float e = ex2_approx((x - m[j]) * kLog2e);
+                    const float e = ex2_approx(exp_arg(x, m[j], m2[j]));
                     a[j] = fmaf(e, v[j], a[j]);
                     b[j] += e;
                 }
@@ -208,6 +221,8 @@ struct WkvOp {
                     kn[j] = fminf(kn[j], k[j]);
                 }
             }
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) m2[j] = m[j] * kLog2e;
             for (int i = 0; i < n; ++i) {
                 float k[CPT], v[CPT];
                 Vec<IO, CPT>::load(p0 + i * CG, k);
@@ -215,7 +230,7 @@ struct WkvOp {
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) {
                     const float x = fmaf(static_cast<float>(i - (n - 1)), q[j].w, k[j]);
-                    const float e = ex2_approx((x - m[j]) * kLog2e);
+                    const float e = ex2_approx(exp_arg(x, m[j], m2[j]));
                     a[j] = fmaf(e, v[j], a[j]);
                     b[j] += e;
                 }
@@ -258,11 +273,12 @@ struct WkvOp {
                                                  const Scratch (&sc)[CPT], IO *out, size_t ostride,
                                                  bool valid) {
         // reference per channel, and whether the fixed-reference form is safe
-        float M[CPT], A[CPT], Bs[CPT];
+        float M[CPT], M2[CPT], A[CPT], Bs[CPT];
         bool fast = true;
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
             M[j] = fmaxf(carry[j].p, sc[j].kmax);
+            M2[j] = M[j] * kLog2e;
             const float s = expf(carry[j].p - M[j]);
             A[j] = carry[j].a * s;
             Bs[j] = carry[j].b * s;
@@ -276,10 +292,10 @@ struct WkvOp {
             if (n == LS) {
 #pragma unroll 8
                 for (int i = 0; i < LS; ++i)
-                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, A, Bs, q);
+                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, M2, A, Bs, q);
             } else {
                 for (int i = 0; i < n; ++i)
-                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, A, Bs, q);
+                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, M2, A, Bs, q);
             }
         } else {
             State s[CPT];
@@ -297,14 +313,15 @@ struct WkvOp {
     }
 
     __device__ __forceinline__ static void fast_step(const IO *pk, const IO *pv, IO *py, bool valid,
-                                                     const float (&M)[CPT], float (&A)[CPT],
-                                                     float (&Bs)[CPT], const Param (&q)[CPT]) {
+                                                     const float (&M)[CPT], const float (&M2)[CPT],
+                                                     float (&A)[CPT], float (&Bs)[CPT],
+                                                     const Param (&q)[CPT]) {
         float k[CPT], v[CPT], y[CPT];
         Vec<IO, CPT>::load(pk, k);
         Vec<IO, CPT>::load(pv, v);
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
-            const float e = ex2_approx((k[j] - M[j]) * kLog2e);
+            const float e = ex2_approx(exp_arg(k[j], M[j], M2[j]));
             const float eu = e * q[j].U;
             y[j] = wkv_output(A[j], Bs[j], eu, v[j]);
             A[j] = fmaf(A[j], q[j].D, e * v[j]);

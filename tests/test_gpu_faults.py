@@ -1,0 +1,61 @@
+"""Failure detection on the GPU without faulting it.
+
+A test hook makes one tile never publish its state, so the look-back waits of
+the tiles after it in time run out.  Every wait in the kernels is bounded: the
+waits give up after a short poll budget, the launch finishes, the affected
+outputs are NaN (and only those), wkv_device_status reports WKV_ERR_TIMEOUT,
+and the next call on the same context is correct again.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture
+def m(cuda_dev):
+    import rwkv_wkv_mixing_b200 as mod
+    yield mod
+    mod.wkv_set_fault_injection(-1, 0)
+    mod.wkv_set_tile_steps(128)
+
+
+@pytest.mark.parametrize("steps", [128, 32])   # persistent pipeline, block per tile
+def test_a_tile_that_never_publishes_times_out_cleanly(m, steps):
+    B, T, C = 1, 1024, 64            # two 32-channel groups -> two chains in time
+    x = workloads.make_wkv("wkv_169m", B=B, T=T, C=C, seed=101)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to("cuda")   # noqa: E731
+    w, u, k, v = d(x.w), d(x.u), d(x.k), d(x.v)
+    want = oracle.wkv_rnn(x.w, x.u, x.k, x.v)
+    tol = 1e-5 * float(np.abs(x.v).max())
+    m.wkv_set_tile_steps(steps)
+    m.wkv_device_status()             # start from a clean status word
+
+    # tiles are numbered segment-major, 2 per segment: tile 4 = segment 2 of
+    # channel group 0; it computes its own outputs but never publishes
+    m.wkv_set_fault_injection(4, 4096)
+    y = m.wkv_forward(w, u, k, v)
+    with pytest.raises(m.WkvError) as err:
+        m.wkv_device_status()
+    assert err.value.status == m.WKV_ERR_TIMEOUT
+    got = y.double().cpu().numpy()
+    cut = 3 * steps                   # first step of segment 3
+    assert np.isnan(got[:, cut:, :32]).all(), "outputs behind the silent tile must be NaN"
+    assert np.abs(got[:, :cut, :] - want[:, :cut, :]).max() <= tol
+    assert np.abs(got[:, :, 32:] - want[:, :, 32:]).max() <= tol
+
+    # the context is still usable: the same call without the fault is correct
+    m.wkv_set_fault_injection(-1, 0)
+    y = m.wkv_forward(w, u, k, v)
+    m.wkv_device_status()
+    assert np.abs(y.double().cpu().numpy() - want).max() <= tol
+
+
+def test_fault_injection_arguments_are_checked(m):
+    assert m.lib.wkv_set_fault_injection(-2, 0) == m.WKV_ERR_INVALID_ARG
+    assert m.lib.wkv_set_fault_injection(0, -1) == m.WKV_ERR_INVALID_ARG
+    assert m.lib.wkv_set_fault_injection(-1, 0) == m.WKV_OK

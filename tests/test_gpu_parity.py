@@ -424,3 +424,44 @@ def test_many_back_to_back_launches(m, op):
     m.wkv_device_status()
     worst = max(float((o.double() - want).abs().max()) for o in outs)
     assert worst <= tol, f"{op}: worst max err over {n_out} outputs {worst} > {tol}"
+
+
+# ---------------------------------------------------------------------------
+# host-buffer entry points (chunked, overlapped copy / compute pipeline)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,T,C,pinned", [(8, 700, 96, True),     # chunks of batch rows
+                                          (1, 1500, 512, True),   # channel slices, 2-D copies
+                                          (3, 300, 40, False),    # pageable memory
+                                          (1, 50, 33, True)])     # one chunk
+def test_wkv_host_entry_point(m, B, T, C, pinned):
+    x = workloads.make_wkv("wkv_169m", B=B, T=T, C=C, seed=B + T + C)
+    h = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory() if pinned \
+        else torch.from_numpy(np.ascontiguousarray(a))   # noqa: E731
+    y = m.wkv_forward_host(h(x.w), h(x.u), h(x.k), h(x.v))
+    want = oracle.wkv_rnn(x.w, x.u, x.k, x.v)
+    assert_close(y.double().numpy(), want, wkv_tol(T, np.abs(x.v).max()), f"host {B}x{T}x{C}")
+
+
+def test_wkv_bf16_host_entry_point(m):
+    x = workloads.make_wkv("wkv_3b_bf16", B=1, T=900, C=384, seed=81)
+    kb = torch.from_numpy(x.k_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    vb = torch.from_numpy(x.v_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y = m.wkv_forward_bf16_host(torch.from_numpy(x.w), torch.from_numpy(x.u), kb, vb)
+    want = oracle.wkv_rnn(x.w, x.u, x.k, x.v)
+    assert_close(y.float().double().numpy(), want, 2e-2 * np.abs(x.v).max(), "bf16 host")
+
+
+@pytest.mark.parametrize("B,T,D", [(16, 600, 64), (1, 700, 256)])
+def test_scan_host_entry_point(m, B, T, D):
+    x = workloads.make_scan("scan_mingru", B=B, T=T, D=D, seed=91, with_h0=True)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()   # noqa: E731
+    hh = m.diag_scan_host(t(x.a), t(x.b), t(x.h0))
+    want = oracle.scan_rnn(x.a, x.b, x.h0)
+    assert_close(hh.double().numpy(), want, 1e-5 * np.abs(want).max(), "scan host")
+
+
+def test_host_entry_point_rejects_device_memory(m):
+    k = torch.zeros(1, 4, 4, device="cuda")
+    w = torch.zeros(4)
+    assert m.lib.wkv_forward_host(1, 4, 4, w.data_ptr(), w.data_ptr(), k.data_ptr(),
+                                  k.data_ptr(), k.data_ptr()) == m.WKV_ERR_INVALID_ARG
