@@ -17,6 +17,10 @@ Pieces (all float64; each cites the page it follows):
 * ``wkv_rnn``             -- the RNN-mode state update (RWKV evolution
   article, section RWKV-V4), max-stabilised; the full-tensor oracle and the
   timed CPU baseline (C code, OpenMP over channels).
+* ``wkv_direct_state`` / ``wkv_rnn_state`` -- the same two forms starting
+  from a given state (the past sums before step 0, RNN mode) and returning
+  the state after the last step; ``wkv_direct_points(..., s_in=)`` likewise.
+  A state is [B, 3, C]: planes a, b, p with (num, den) = (a, b) e^p.
 * ``wkv_slru_ratio_np``   -- the "RWKV = ratio of two SLRUs" form from the
   review of "Resurrecting Recurrent Neural Networks for Long Sequences"
   (section on the RWKV variant), unstabilised; |k| small only.
@@ -47,6 +51,7 @@ _lib = None
 __all__ = [
     "build", "max_threads", "wkv_direct", "wkv_direct_points", "wkv_direct_np",
     "wkv_rnn", "wkv_slru_ratio_np", "scan_rnn", "scan_direct_points",
+    "wkv_direct_state", "wkv_rnn_state", "state_mean_logden",
 ]
 
 
@@ -73,6 +78,10 @@ def _get():
                 "oracle_wkv_direct": [i64, i64, i64, p, p, p, p, p, ctypes.c_int],
                 "oracle_wkv_direct_points": [i64, i64, i64, p, p, p, p, i64, p, p, ctypes.c_int],
                 "oracle_wkv_rnn": [i64, i64, i64, p, p, p, p, p, ctypes.c_int],
+                "oracle_wkv_direct_s": [i64, i64, i64, p, p, p, p, p, p, p, ctypes.c_int],
+                "oracle_wkv_direct_points_s": [i64, i64, i64, p, p, p, p, p, i64, p, p,
+                                               ctypes.c_int],
+                "oracle_wkv_rnn_s": [i64, i64, i64, p, p, p, p, p, p, p, ctypes.c_int],
                 "oracle_scan_rnn": [i64, i64, i64, p, p, p, p, ctypes.c_int],
                 "oracle_scan_direct_points": [i64, i64, i64, p, p, p, i64, p, p, ctypes.c_int],
             }.items():
@@ -114,16 +123,66 @@ def wkv_direct(w, u, k, v, nthreads: int = 0) -> np.ndarray:
     return y
 
 
-def wkv_direct_points(w, u, k, v, points, nthreads: int = 0) -> np.ndarray:
-    """Eq. (14) at the flat output indices ``points`` (b*T*C + t*C + c)."""
+def _state_arg(s, B, C):
+    if s is None:
+        return None
+    s = _f64(s)
+    if s.shape != (B, 3, C):
+        raise ValueError("a state must be [B, 3, C]")
+    return s
+
+
+def _optr(x):
+    return None if x is None else _ptr(x)
+
+
+def wkv_direct_points(w, u, k, v, points, nthreads: int = 0, s_in=None) -> np.ndarray:
+    """Eq. (14) at the flat output indices ``points`` (b*T*C + t*C + c),
+    from the state ``s_in`` ([B, 3, C]) or the empty past."""
     B, T, C, w, u, k, v = _wkv_args(w, u, k, v)
+    s_in = _state_arg(s_in, B, C)
     pts = np.ascontiguousarray(points, dtype=np.int64).reshape(-1)
     if pts.size and (pts.min() < 0 or pts.max() >= B * T * C):
         raise IndexError("point out of range")
     out = np.empty(pts.size, dtype=np.float64)
-    _get().oracle_wkv_direct_points(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v),
-                                    pts.size, _ptr(pts), _ptr(out), nthreads)
+    _get().oracle_wkv_direct_points_s(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v),
+                                      _optr(s_in), pts.size, _ptr(pts), _ptr(out), nthreads)
     return out
+
+
+def wkv_direct_state(w, u, k, v, s_in=None, nthreads: int = 0):
+    """Eq. (14) at every output from the state ``s_in`` (None: empty past);
+    returns (y, s_out), s_out the past sums after the last step with p the
+    largest logit.  O(T^2) per channel."""
+    B, T, C, w, u, k, v = _wkv_args(w, u, k, v)
+    s_in = _state_arg(s_in, B, C)
+    y = np.empty((B, T, C), dtype=np.float64)
+    s_out = np.empty((B, 3, C), dtype=np.float64)
+    _get().oracle_wkv_direct_s(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _optr(s_in),
+                               _ptr(y), _ptr(s_out), nthreads)
+    return y, s_out
+
+
+def wkv_rnn_state(w, u, k, v, s_in=None, nthreads: int = 0):
+    """RNN-mode recurrence from the state ``s_in`` (None: empty past);
+    returns (y, s_out)."""
+    B, T, C, w, u, k, v = _wkv_args(w, u, k, v)
+    s_in = _state_arg(s_in, B, C)
+    y = np.empty((B, T, C), dtype=np.float64)
+    s_out = np.empty((B, 3, C), dtype=np.float64)
+    _get().oracle_wkv_rnn_s(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _optr(s_in),
+                            _ptr(y), _ptr(s_out), nthreads)
+    return y, s_out
+
+
+def state_mean_logden(s):
+    """What a state (a, b, p) fixes whatever its scaling: the mean a / b of
+    the past values and ln den = p + ln b.  Two states are the same state
+    exactly when both agree."""
+    s = np.asarray(s, dtype=np.float64)
+    a, b, p = s[:, 0], s[:, 1], s[:, 2]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return a / b, p + np.log(b)
 
 
 def wkv_rnn(w, u, k, v, nthreads: int = 0) -> np.ndarray:

@@ -25,7 +25,9 @@
  *               section: the scan form v_t = a_t (.) v_{t-1} + b_t.
  *
  * Layout: k, v, y, a, b, h are [B, T, C] row-major with C fastest; w, u are
- * [C]; h0 is [B, C] or NULL (zeros).  Inputs and results are float64 (the
+ * [C]; h0 is [B, C] or NULL (zeros).  A WKV state is [B, 3, C]: planes a, b,
+ * p per batch row, standing for the past sums (num, den) = (a, b) e^p; NULL
+ * or a = b = 0 is the empty past.  Inputs and results are float64 (the
  * caller widens the float32 / bf16 values the GPU path reads, exactly).
  */
 #include <math.h>
@@ -45,33 +47,67 @@ int oracle_max_threads(void) { return omp_get_max_threads(); }
  *     l_i = -(t-1-i) w_c + k_i   for i < t,      l_t = u_c + k_t.
  * Each point is an O(t) direct sum; the common factor e^{-m}, m = max l,
  * is taken out of numerator and denominator so no term overflows.
+ *
+ * A state before step 0 (RNN mode, [RWKV-EVO] section RWKV-V4; sequential
+ * decoding, [RWKV-LLM] section 三) is the pair of past sums (num_0, den_0).  Step t
+ * sees it decayed t times, so it adds e^{-t w} (num_0, den_0) to the sums:
+ * one more term with logit -t w + p and weights (a, b) in place of (v_i, 1).
  * ------------------------------------------------------------------------ */
-static double wkv_direct_one(int64_t T, int64_t C, double w, double u,
-                             const double *k, const double *v, int64_t t) {
-    /* k, v point at channel c of batch row b (stride C between steps) */
-    double m = u + k[t * C];
+static int state_empty(const double *s, int64_t C) {
+    /* s points at (a, b, p) of one channel, planes C apart */
+    return !s || (s[0] == 0.0 && s[C] == 0.0) || (isinf(s[2 * C]) && s[2 * C] < 0);
+}
+
+/* sums over i < t (and the state) of e^{l_i - m} (v_i, 1), with m the largest
+ * logit among them and `extra` (a logit the caller adds itself) */
+static void past_sums(int64_t C, double w, const double *k, const double *v,
+                      const double *s, int64_t t, double extra,
+                      double *m_out, double *num, double *den) {
+    int has_s = !state_empty(s, C);
+    double m = extra;
     for (int64_t i = 0; i < t; ++i) {
         double l = -(double)(t - 1 - i) * w + k[i * C];
         if (l > m) m = l;
     }
-    double e_t = exp(u + k[t * C] - m);
-    double num = e_t * v[t * C];
-    double den = e_t;
+    double ls = has_s ? -(double)t * w + s[2 * C] : -INFINITY;
+    if (ls > m) m = ls;
+    double n = 0.0, d = 0.0;
     for (int64_t i = 0; i < t; ++i) {
         double e = exp(-(double)(t - 1 - i) * w + k[i * C] - m);
-        num += e * v[i * C];
-        den += e;
+        n += e * v[i * C];
+        d += e;
     }
-    (void)T;
-    return num / den;
+    if (has_s) {
+        double e = exp(ls - m);
+        n += e * s[0];
+        d += e * s[C];
+    }
+    *m_out = m;
+    *num = n;
+    *den = d;
+}
+
+static double wkv_direct_one(int64_t C, double w, double u, const double *k,
+                             const double *v, const double *s, int64_t t) {
+    /* k, v point at channel c of batch row b (stride C between steps);
+     * s at that channel's state or NULL */
+    double lt = u + k[t * C];
+    double m, num, den;
+    past_sums(C, w, k, v, s, t, lt, &m, &num, &den);
+    double e_t = exp(lt - m);
+    return (num + e_t * v[t * C]) / (den + e_t);
+}
+
+static const double *state_at(const double *s, int64_t b, int64_t c, int64_t C) {
+    return s ? s + b * 3 * C + c : NULL;
 }
 
 /* points[j] is the flat index b*T*C + t*C + c of the j-th requested output */
-void oracle_wkv_direct_points(int64_t B, int64_t T, int64_t C,
-                              const double *w, const double *u,
-                              const double *k, const double *v,
-                              int64_t n, const int64_t *points, double *out,
-                              int nthreads) {
+void oracle_wkv_direct_points_s(int64_t B, int64_t T, int64_t C,
+                                const double *w, const double *u,
+                                const double *k, const double *v, const double *s_in,
+                                int64_t n, const int64_t *points, double *out,
+                                int nthreads) {
     (void)B;
 #pragma omp parallel for schedule(dynamic, 16) num_threads(pick_threads(nthreads))
     for (int64_t j = 0; j < n; ++j) {
@@ -81,22 +117,49 @@ void oracle_wkv_direct_points(int64_t B, int64_t T, int64_t C,
         int64_t c = f % C;
         const double *kb = k + b * T * C + c;
         const double *vb = v + b * T * C + c;
-        out[j] = wkv_direct_one(T, C, w[c], u[c], kb, vb, t);
+        out[j] = wkv_direct_one(C, w[c], u[c], kb, vb, state_at(s_in, b, c, C), t);
     }
 }
 
-/* every output by the definition: O(T^2) per channel, small inputs only */
-void oracle_wkv_direct(int64_t B, int64_t T, int64_t C,
-                       const double *w, const double *u,
-                       const double *k, const double *v, double *y, int nthreads) {
+void oracle_wkv_direct_points(int64_t B, int64_t T, int64_t C,
+                              const double *w, const double *u,
+                              const double *k, const double *v,
+                              int64_t n, const int64_t *points, double *out,
+                              int nthreads) {
+    oracle_wkv_direct_points_s(B, T, C, w, u, k, v, NULL, n, points, out, nthreads);
+}
+
+/* every output by the definition: O(T^2) per channel, small inputs only;
+ * s_out (if not NULL) gets the past sums after the last step, the same
+ * definition at t = T without a current token, as (a, b, p) with p the
+ * largest logit */
+void oracle_wkv_direct_s(int64_t B, int64_t T, int64_t C,
+                         const double *w, const double *u,
+                         const double *k, const double *v, const double *s_in,
+                         double *y, double *s_out, int nthreads) {
 #pragma omp parallel for schedule(dynamic, 1) num_threads(pick_threads(nthreads))
     for (int64_t bc = 0; bc < B * C; ++bc) {
         int64_t b = bc / C, c = bc % C;
         const double *kb = k + b * T * C + c;
         const double *vb = v + b * T * C + c;
+        const double *sb = state_at(s_in, b, c, C);
         for (int64_t t = 0; t < T; ++t)
-            y[b * T * C + t * C + c] = wkv_direct_one(T, C, w[c], u[c], kb, vb, t);
+            y[b * T * C + t * C + c] = wkv_direct_one(C, w[c], u[c], kb, vb, sb, t);
+        if (s_out) {
+            double m, num, den;
+            past_sums(C, w[c], kb, vb, sb, T, -INFINITY, &m, &num, &den);
+            double *so = s_out + b * 3 * C + c;
+            so[0] = num;
+            so[C] = den;
+            so[2 * C] = m;
+        }
     }
+}
+
+void oracle_wkv_direct(int64_t B, int64_t T, int64_t C,
+                       const double *w, const double *u,
+                       const double *k, const double *v, double *y, int nthreads) {
+    oracle_wkv_direct_s(B, T, C, w, u, k, v, NULL, y, NULL, nthreads);
 }
 
 /* ------------------------------------------------------------------------
@@ -108,16 +171,24 @@ void oracle_wkv_direct(int64_t B, int64_t T, int64_t C,
  *     y_t = (num_t + e^{u+k_t} v_t) / (den_t + e^{u+k_t}).
  * The pair is stored as (a, b) = (num, den) * e^{-p}; p is the largest
  * exponent seen so far, so every exp() below has a non-positive argument.
- * Starting state: empty sums (a = b = 0, p = -inf).
+ * Starting state: s_in, or empty sums (a = b = 0, p = -inf) when it is NULL;
+ * the state after the last step goes to s_out when it is not NULL.
  * ------------------------------------------------------------------------ */
-void oracle_wkv_rnn(int64_t B, int64_t T, int64_t C,
-                    const double *w, const double *u,
-                    const double *k, const double *v, double *y, int nthreads) {
+void oracle_wkv_rnn_s(int64_t B, int64_t T, int64_t C,
+                      const double *w, const double *u,
+                      const double *k, const double *v, const double *s_in,
+                      double *y, double *s_out, int nthreads) {
 #pragma omp parallel for schedule(static) num_threads(pick_threads(nthreads))
     for (int64_t bc = 0; bc < B * C; ++bc) {
         int64_t b = bc / C, c = bc % C;
         double wc = w[c], uc = u[c];
         double a = 0.0, d = 0.0, p = -INFINITY;
+        const double *sb = state_at(s_in, b, c, C);
+        if (!state_empty(sb, C)) {
+            a = sb[0];
+            d = sb[C];
+            p = sb[2 * C];
+        }
         for (int64_t t = 0; t < T; ++t) {
             int64_t o = b * T * C + t * C + c;
             double kt = k[o], vt = v[o];
@@ -134,7 +205,19 @@ void oracle_wkv_rnn(int64_t B, int64_t T, int64_t C,
             d = f_old * d + f_new;
             p = q2;
         }
+        if (s_out) {
+            double *so = s_out + b * 3 * C + c;
+            so[0] = a;
+            so[C] = d;
+            so[2 * C] = p;
+        }
     }
+}
+
+void oracle_wkv_rnn(int64_t B, int64_t T, int64_t C,
+                    const double *w, const double *u,
+                    const double *k, const double *v, double *y, int nthreads) {
+    oracle_wkv_rnn_s(B, T, C, w, u, k, v, NULL, y, NULL, nthreads);
 }
 
 /* ------------------------------------------------------------------------

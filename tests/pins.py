@@ -213,6 +213,147 @@ def run_wkv_pins(fn):
 
 
 # ---------------------------------------------------------------------------
+# WKV with a state in and out.  An implementation here is
+#     fn(w, u, k, v, s_in) -> (y, s_out)
+# with states [B, 3, C] (planes a, b, p: past sums (num, den) = (a, b) e^p) and
+# s_in None for the empty past.  A state is compared by what fixes it: the
+# mean a / b and ln den = p + ln b.
+# ---------------------------------------------------------------------------
+def _state_parts(s):
+    s = np.asarray(s, dtype=np.float64)
+    a, b, p = s[:, 0], s[:, 1], s[:, 2]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return a / b, p + np.log(b)
+
+
+def _close_state(got, want, tol):
+    gm, gl = _state_parts(got)
+    wm, wl = _state_parts(want)
+    return _close(gm, wm, tol) or _close(gl, wl, tol)
+
+
+def _state_from(num, den):
+    """A [1, 3, C] state holding the past sums num, den (den > 0)."""
+    num = np.asarray(num, dtype=np.float64).reshape(1, -1)
+    den = np.asarray(den, dtype=np.float64).reshape(1, -1)
+    return np.stack([num / den, np.ones_like(den), np.log(den)], axis=1)
+
+
+def wkv_state_worked_example(fn, tol=1e-12):
+    g = read_golden("wkv_state_worked_example.txt")
+    w = np.array([-np.log(float(g["w_exp_neg"][0]))])
+    u = np.array([np.log(float(g["u_exp"][0]))])
+    s_in = np.array([[[float(g["state_a"][0])], [float(g["state_b"][0])],
+                      [np.log(float(g["state_p_exp"][0]))]]])
+    k = np.log(np.array([float(x) for x in g["k_exp"]]))[None, :, None]
+    v = np.array([float(x) for x in g["v"]])[None, :, None]
+    y, s_out = fn(w, u, k, v, s_in)
+    out = []
+    msg = _close(y, np.array([float(x) for x in g["y"]])[None, :, None], tol)
+    if msg: out.append(f"state worked example, y: {msg}")
+    msg = _close_state(s_out, _state_from(float(g["num_out"][0]), float(g["den_out"][0])), tol)
+    if msg: out.append(f"state worked example, state out: {msg}")
+    return out
+
+
+def wkv_state_empty(fn, tol=0.0):
+    """No state, the explicit empty state (a = b = 0) and the no-state
+    forms agree, outputs and state out."""
+    w, u, k, v = _rand_wkv(11, B=2, T=20, C=3)
+    y0, s0 = fn(w, u, k, v, None)
+    out = []
+    for p_fill in (-np.inf, 0.0, 7.5):
+        s_in = np.zeros((2, 3, 3)); s_in[:, 2] = p_fill
+        y1, s1 = fn(w, u, k, v, s_in)
+        msg = _close(y1, y0, tol) or _close_state(s1, s0, max(tol, 1e-15))
+        if msg: out.append(f"empty state (p = {p_fill}): {msg}")
+    return out
+
+
+def wkv_state_chaining(fn, tol=1e-12):
+    """Splitting the steps into calls that hand the state on gives the
+    outputs and final state of one call (several split points, T = 1 calls
+    included: RNN-mode decoding)."""
+    w, u, k, v = _rand_wkv(12, B=2, T=40, C=4)
+    y, s = fn(w, u, k, v, None)
+    out = []
+    for cuts in ([17], [1, 2, 3, 39], [10, 20, 30], list(range(1, 40))):
+        ys, st, prev = [], None, 0
+        for c in cuts + [40]:
+            yy, st = fn(w, u, k[:, prev:c], v[:, prev:c], st)
+            ys.append(yy)
+            prev = c
+        msg = _close(np.concatenate(ys, axis=1), y, tol) or _close_state(st, s, tol)
+        if msg: out.append(f"chaining at {cuts[:4]}: {msg}")
+    return out
+
+
+def wkv_state_virtual_token(fn, tol=1e-12):
+    """The state after one token (k0, v0) is (num, den) = (e^{k0} v0, e^{k0});
+    starting there equals running that token first and dropping its output."""
+    w, u, k, v = _rand_wkv(13, B=1, T=25, C=3)
+    y_full, s_full = fn(w, u, k, v, None)
+    s_in = _state_from(np.exp(k[0, 0]) * v[0, 0], np.exp(k[0, 0]))
+    y, s = fn(w, u, k[:, 1:], v[:, 1:], s_in)
+    msg = _close(y, y_full[:, 1:], tol) or _close_state(s, s_full, tol)
+    return [f"state as a virtual token: {msg}"] if msg else []
+
+
+def wkv_state_scaling(fn, tol=1e-12):
+    """(a, b, p) and (a e^s, b e^s, p - s) are one state: same outputs and
+    same state out."""
+    w, u, k, v = _rand_wkv(14, B=2, T=16, C=3)
+    rng = np.random.default_rng(14)
+    s_in = np.stack([rng.normal(0, 1, (2, 3)), np.exp(rng.normal(0, 1, (2, 3))),
+                     rng.normal(0, 2, (2, 3))], axis=1)
+    y0, s0 = fn(w, u, k, v, s_in)
+    out = []
+    for sh in (-3.0, 0.5, 12.0):
+        s2 = s_in.copy(); s2[:, 0] *= np.exp(sh); s2[:, 1] *= np.exp(sh); s2[:, 2] -= sh
+        y1, s1 = fn(w, u, k, v, s2)
+        msg = _close(y1, y0, tol) or _close_state(s1, s0, tol)
+        if msg: out.append(f"state rescaling by e^{sh}: {msg}")
+    return out
+
+
+def wkv_state_decay_only(fn, tol=1e-12):
+    """With k = -inf-like keys (-60) and u = 0 the tokens add nothing next to
+    a unit state: the state's mean passes straight through to every output
+    and the state out is the state in decayed t times (ln den drops by T w)."""
+    C, T = 3, 6
+    w = np.array([0.1, 0.7, 2.0]); u = np.zeros(C)
+    k = np.full((1, T, C), -60.0); v = np.ones((1, T, C))
+    s_in = np.stack([np.array([[0.25, -1.5, 2.0]]), np.ones((1, C)), np.array([[3.0, 0.0, -2.0]])], axis=1)
+    # token weight e^{-60} against a state weight of at least e^{-2 - 5 * 2}:
+    # the tokens move the results by about e^{-48}, far below tol
+    y, s = fn(w, u, k, v, s_in)
+    out = []
+    msg = _close(y, np.broadcast_to(np.array([0.25, -1.5, 2.0]), (1, T, C)), tol)
+    if msg: out.append(f"decay only, y: {msg}")
+    want = np.stack([np.array([[0.25, -1.5, 2.0]]), np.ones((1, C)),
+                     np.array([[3.0, 0.0, -2.0]]) - T * w[None]], axis=1)
+    msg = _close_state(s, want, tol)
+    if msg: out.append(f"decay only, state: {msg}")
+    return out
+
+
+WKV_STATE_PINS = [wkv_state_worked_example, wkv_state_empty, wkv_state_chaining,
+                  wkv_state_virtual_token, wkv_state_scaling, wkv_state_decay_only]
+
+
+def run_wkv_state_pins(fn):
+    """The state pins, plus every stateless pin on fn(..., None)[0]."""
+    fails = []
+    for pin in WKV_STATE_PINS:
+        try:
+            fails += pin(fn)
+        except Exception as e:  # a mutant may crash a pin; that counts as caught
+            fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
+    fails += run_wkv_pins(lambda w, u, k, v: fn(w, u, k, v, None)[0])
+    return fails
+
+
+# ---------------------------------------------------------------------------
 # diagonal scan pins
 # ---------------------------------------------------------------------------
 def scan_worked_example(fn, tol=1e-12):

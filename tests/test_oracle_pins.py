@@ -196,6 +196,89 @@ def test_planted_mistake_in_c_oracle_is_caught(name, tmp_path):
     assert pins.run_wkv_pins(mut) != []
 
 
+# --- WKV with a state in and out -------------------------------------------
+def st_direct(w, u, k, v, s):
+    return oracle.wkv_direct_state(w, u, k, v, s)
+
+
+def st_rnn(w, u, k, v, s):
+    return oracle.wkv_rnn_state(w, u, k, v, s)
+
+
+def st_points(w, u, k, v, s):
+    k = np.asarray(k)
+    y = oracle.wkv_direct_points(w, u, k, v, np.arange(k.size), s_in=s).reshape(k.shape)
+    return y, oracle.wkv_direct_state(w, u, k, v, s)[1]
+
+
+@pytest.mark.parametrize("fn", [st_direct, st_rnn, st_points], ids=["direct", "rnn", "points"])
+def test_wkv_state_oracle_passes_pins(fn):
+    assert pins.run_wkv_state_pins(fn) == []
+
+
+def test_wkv_state_forms_agree_on_random_states():
+    rng = np.random.default_rng(21)
+    B, T, C = 3, 70, 6
+    w, u, k, v = (np.exp(rng.uniform(-3, 1, C)), rng.normal(0, 0.5, C),
+                  rng.normal(0, 2, (B, T, C)), rng.normal(0, 1, (B, T, C)))
+    s_in = np.stack([rng.normal(0, 1, (B, C)), np.exp(rng.normal(0, 1, (B, C))),
+                     rng.normal(0, 3, (B, C))], axis=1)
+    y1, s1 = oracle.wkv_direct_state(w, u, k, v, s_in)
+    y2, s2 = oracle.wkv_rnn_state(w, u, k, v, s_in)
+    assert np.max(np.abs(y1 - y2)) < 1e-13
+    for x1, x2 in zip(oracle.state_mean_logden(s1), oracle.state_mean_logden(s2)):
+        assert np.max(np.abs(x1 - x2)) < 1e-12
+
+
+C_STATE_MUTANTS = {
+    # (anchor, replacement, C function the mutant is called through)
+    "state_not_decayed": ("double ls = has_s ? -(double)t * w + s[2 * C] : -INFINITY;",
+                          "double ls = has_s ? s[2 * C] : -INFINITY;", "direct"),
+    "state_decayed_once_more": ("double ls = has_s ? -(double)t * w + s[2 * C] : -INFINITY;",
+                                "double ls = has_s ? -(double)(t + 1) * w + s[2 * C] : -INFINITY;",
+                                "direct"),
+    "state_b_weights_num": ("n += e * s[0];", "n += e * s[C];", "direct"),
+    "state_out_one_step_short": ("past_sums(C, w[c], kb, vb, sb, T, -INFINITY, &m, &num, &den);",
+                                 "past_sums(C, w[c], kb, vb, sb, T - 1, -INFINITY, &m, &num, &den);",
+                                 "direct"),
+    "rnn_state_planes_swapped": ("a = sb[0];\n            d = sb[C];",
+                                 "a = sb[C];\n            d = sb[0];", "rnn"),
+    "rnn_state_out_decayed": ("so[2 * C] = p;\n        }\n    }\n}\n\nvoid oracle_wkv_rnn(",
+                              "so[2 * C] = p - wc;\n        }\n    }\n}\n\nvoid oracle_wkv_rnn(", "rnn"),
+}
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+@pytest.mark.parametrize("name", sorted(C_STATE_MUTANTS))
+def test_planted_mistake_in_state_oracle_is_caught(name, tmp_path):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "wkv_oracle.c")).read()
+    old, new, which = C_STATE_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation anchor for {name} not found"
+    mpath = tmp_path / "mut.c"
+    mpath.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-o", str(so),
+                           str(mpath), "-lm"])
+    lib = ctypes.CDLL(str(so))
+    i64, p = ctypes.c_int64, ctypes.c_void_p
+    cfn = getattr(lib, "oracle_wkv_direct_s" if which == "direct" else "oracle_wkv_rnn_s")
+    cfn.argtypes = [i64, i64, i64, p, p, p, p, p, p, p, ctypes.c_int]
+    cfn.restype = None
+
+    def mut(w, u, k, v, s_in):
+        k = np.ascontiguousarray(k, float); v = np.ascontiguousarray(v, float)
+        w = np.ascontiguousarray(w, float).reshape(-1); u = np.ascontiguousarray(u, float).reshape(-1)
+        B, T, C = k.shape
+        sp = None if s_in is None else np.ascontiguousarray(s_in, float)
+        y = np.empty(k.shape); s_out = np.empty((B, 3, C))
+        cfn(B, T, C, *(x.ctypes.data_as(p) for x in (w, u, k, v)),
+            None if sp is None else sp.ctypes.data_as(p), y.ctypes.data_as(p),
+            s_out.ctypes.data_as(p), 1)
+        return y, s_out
+
+    assert pins.run_wkv_state_pins(mut) != []
+
+
 # --- diagonal scan ---------------------------------------------------------
 def scan_rnn(a, b, h0):
     return oracle.scan_rnn(a, b, h0)
