@@ -218,16 +218,22 @@ class DeviceWorkload:
         self.inputs = x
         self.B, self.T, self.C = B, T, C
         self.elements = B * T * C
-        self.alg_bytes = 3 * self.es * self.elements + self.param_bytes
-        set_bytes = 3 * self.es * self.elements
+        # a workload with a state reads it and writes it back (in place)
+        self.has_state = getattr(x, "s_in", None) is not None
+        self.state_bytes = 2 * 3 * 4 * B * C if self.has_state else 0
+        self.alg_bytes = 3 * self.es * self.elements + self.param_bytes + self.state_bytes
+        set_bytes = 3 * self.es * self.elements + self.state_bytes
+        self.set_bytes = set_bytes
         self.n_sets = 1 if set_bytes >= 3 * l2_bytes else int(np.ceil(3 * l2_bytes / set_bytes)) + 1
         x0 = self._to_dev(self.host["x0"], dev)
         x1 = self._to_dev(self.host["x1"], dev)
+        s0 = torch.from_numpy(x.s_in).to(dev) if self.has_state else None
         self.sets = []
         for i in range(self.n_sets):
             a = x0 if i == 0 else x0.clone()
             b = x1 if i == 0 else x1.clone()
-            self.sets.append((a, b, torch.empty_like(a)))
+            st = None if s0 is None else (s0 if i == 0 else s0.clone())
+            self.sets.append((a, b, torch.empty_like(a), st))
         self.stream = torch.cuda.current_stream()
 
     def _to_dev(self, arr, dev):
@@ -236,7 +242,7 @@ class DeviceWorkload:
             t = t.view(self.torch.bfloat16)
         return t.to(dev)
 
-    def call(self, x0, x1, y):
+    def call(self, x0, x1, y, st=None):
         """One C-ABI call on torch's current stream (the capture stream while a
         graph is being captured)."""
         lib = self.lib
@@ -244,9 +250,22 @@ class DeviceWorkload:
         if self.is_scan:
             return lib.diag_scan(self.B, self.T, self.C, x0.data_ptr(), x1.data_ptr(), None,
                                  y.data_ptr(), sh)
+        if st is not None:   # state in and out, updated in place
+            fn = lib.wkv_forward_bf16_state if self.dtype == "bf16" else lib.wkv_forward_state
+            return fn(self.B, self.T, self.C, self.params[0].data_ptr(),
+                      self.params[1].data_ptr(), x0.data_ptr(), x1.data_ptr(), y.data_ptr(),
+                      st.data_ptr(), st.data_ptr(), sh)
         fn = lib.wkv_forward_bf16 if self.dtype == "bf16" else lib.wkv_forward
         return fn(self.B, self.T, self.C, self.params[0].data_ptr(), self.params[1].data_ptr(),
                   x0.data_ptr(), x1.data_ptr(), y.data_ptr(), sh)
+
+    def kernel(self):
+        """The kernel a step launches (the library's dispatch rule)."""
+        if not self.is_scan and self.T <= 16:
+            return "wkv_serial_kernel"
+        if self.lib.wkv_get_tile_steps() in (8, 32):
+            return "chunked_scan_kernel"
+        return "persistent_scan_kernel"
 
     def step(self, i):
         st = self.call(*self.sets[i % self.n_sets])
@@ -350,7 +369,33 @@ def e2e_leg(torch, wl, steps):
     hx1 = torch.from_numpy(np.ascontiguousarray(wl.host["x1"])).pin_memory()
     hy = torch.empty_like(hx0).pin_memory()
     hp = [p.cpu().pin_memory() for p in wl.params]
-    if wl.is_scan:
+    hs = None
+    if wl.has_state:
+        # no host-buffer entry point takes a state: the user-side sequence is
+        # pinned copies in, the device call, copies out, on one stream
+        hs = torch.from_numpy(wl.inputs.s_in).pin_memory()
+        dx0, dx1, dy, ds = (torch.empty(t.shape, dtype=t.dtype, device="cuda")
+                            for t in (hx0, hx1, hy, hs))
+        if wl.dtype == "bf16":
+            dx0, dx1, dy = (t.view(torch.bfloat16) for t in (dx0, dx1, dy))
+        dp = wl.params
+        api = ("wkv_forward_bf16_state" if wl.dtype == "bf16" else "wkv_forward_state") + \
+            " with pinned copies on one stream"
+        fn = getattr(lib, "wkv_forward_bf16_state" if wl.dtype == "bf16" else "wkv_forward_state")
+
+        def call():
+            stream = torch.cuda.current_stream()
+            dx0.copy_(hx0.view(dx0.dtype) if wl.dtype == "bf16" else hx0, non_blocking=True)
+            dx1.copy_(hx1.view(dx1.dtype) if wl.dtype == "bf16" else hx1, non_blocking=True)
+            ds.copy_(hs, non_blocking=True)
+            st = fn(wl.B, wl.T, wl.C, dp[0].data_ptr(), dp[1].data_ptr(), dx0.data_ptr(),
+                    dx1.data_ptr(), dy.data_ptr(), ds.data_ptr(), ds.data_ptr(),
+                    stream.cuda_stream)
+            hy.copy_(dy.view(hy.dtype) if wl.dtype == "bf16" else dy, non_blocking=True)
+            hs.copy_(ds, non_blocking=True)
+            stream.synchronize()
+            return st
+    elif wl.is_scan:
         api = "diag_scan_host"
         call = lambda: lib.diag_scan_host(wl.B, wl.T, wl.C, hx0.data_ptr(), hx1.data_ptr(),  # noqa: E731
                                           None, hy.data_ptr())
@@ -378,8 +423,11 @@ def e2e_leg(torch, wl, steps):
     b.synchronize()
     wall_ms = (time.perf_counter() - t0) / steps * 1e3
     ms = a.elapsed_time(b) / steps
-    h2d = hx0.numel() * hx0.element_size() * 2 + wl.param_bytes
+    h2d = hx0.numel() * hx0.element_size() * 2 + (wl.param_bytes if hs is None else 0)
     d2h = hy.numel() * hy.element_size()
+    if hs is not None:   # the state travels both ways
+        h2d += hs.numel() * 4
+        d2h += hs.numel() * 4
     return {"value": wl.elements / (ms / 1e3), "unit": "elem/s", "ms_per_step": ms,
             "wall_ms_per_step": wall_ms, "steps": steps, "api": api,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -413,7 +461,11 @@ def oracle_runner(name, max_elements=None):
             chans = max(1, min(C, max_elements // T))
     k = np.ascontiguousarray(k[:rows, :, :chans]); v = np.ascontiguousarray(v[:rows, :, :chans])
     w, u = w[:chans], u[:chans]
-    fn = lambda: oracle.wkv_rnn(w, u, k, v)   # noqa: E731
+    if x.s_in is not None:
+        s_in = np.ascontiguousarray(x.s_in[:rows, :, :chans], dtype=np.float64)
+        fn = lambda: oracle.wkv_rnn_state(w, u, k, v, s_in)   # noqa: E731
+    else:
+        fn = lambda: oracle.wkv_rnn(w, u, k, v)   # noqa: E731
     return fn, rows * T * chans, f"{rows} of {B} batch rows x {chans} of {C} channels (all T={T})"
 
 
@@ -486,8 +538,9 @@ def workload_config(spec, name):
     if isinstance(spec, workloads.ScanSpec):
         return {"workload": name, "op": "diag_scan", "B": spec.B, "T": spec.T, "D": spec.D,
                 "io": "f32"}
-    return {"workload": name, "op": "wkv_forward" + ("_bf16" if spec.dtype == "bf16" else ""),
-            "B": spec.B, "T": spec.T, "C": spec.C, "io": spec.dtype}
+    op = "wkv_forward" + ("_bf16" if spec.dtype == "bf16" else "") + \
+        ("_state (state [B,3,C] fp32 read and written in place)" if spec.state else "")
+    return {"workload": name, "op": op, "B": spec.B, "T": spec.T, "C": spec.C, "io": spec.dtype}
 
 
 # ---------------------------------------------------------------------------
@@ -593,7 +646,7 @@ def main(argv=None):
     cfg = workload_config(spec, args.workload)
     cfg.update({"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                 "l2": (f"inputs rotate over {wl.n_sets} buffer sets "
-                       f"({wl.n_sets * 3 * wl.es * wl.elements / 1e6:.0f} MB > L2 "
+                       f"({wl.n_sets * wl.set_bytes / 1e6:.0f} MB > L2 "
                        f"{l2 / 1e6:.0f} MB)"),
                 "tile_steps": wkv.wkv_get_tile_steps(),
                 "launch": args.launch + (" (K steps replayed from captured graphs)"
@@ -611,7 +664,7 @@ def main(argv=None):
                      "traffic": traffic, "alg_bytes_per_launch": wl.alg_bytes,
                      "launch_ms_mean": launch_ms,
                      "launch_ms_median": statistics.median(per),
-                     "kernel": "chunked_scan_kernel"},
+                     "kernel": wl.kernel()},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps,

@@ -42,6 +42,11 @@
  *           grown when a larger problem needs it.  Make one call of each size
  *           before capturing a stream into a CUDA graph.  Calls on different
  *           streams use different workspaces and may run concurrently.
+ * Rounding  results match the operator to fp32 rounding; they are bitwise
+ *           reproducible from run to run when T spans at most two tiles
+ *           (256 steps).  Beyond that the carry between tiles may fold a
+ *           different, equivalent set of partial results, which can move the
+ *           last bits.
  * Errors    argument errors are detected on the host before anything is
  *           launched and return a non-zero wkv_status; wkv_last_error()
  *           then describes the problem (thread-local, valid until the next
@@ -94,6 +99,47 @@ WKV_API wkv_status wkv_forward_bf16(int64_t B, int64_t T, int64_t C,
                             const float *w, const float *u,
                             const wkv_bf16_t *k, const wkv_bf16_t *v, wkv_bf16_t *y,
                             cudaStream_t stream);
+
+/* WKV forward from a given state, with the state after the last step
+ * returned: streaming a sequence over several calls, and RNN-mode decoding
+ * one token per call (T = 1).  The RNN-mode reading of eq. (14) (RWKV
+ * evolution article, section RWKV-V4; "RWKV：基于RNN的LLM" section 三,
+ * sequential decoding): the state before step t is the pair of past sums
+ *
+ *     num_t = sum_{i<t} e^{-(t-1-i) w + k_i} v_i,   den_t = the same without v_i,
+ *
+ * and each step decays it by e^{-w} and adds e^{k_t} (v_t, 1), so a state
+ * handed in as the sums before step 0 enters step t weighted by e^{-t w}:
+ *
+ *     y_t = (e^{-t w} num_in + sum_{0<=i<t} ... + e^{u+k_t} v_t)
+ *         / (e^{-t w} den_in + sum_{0<=i<t} ... + e^{u+k_t}).
+ *
+ * State layout: s_in, s_out are [B, 3, C] float -- for batch row b the planes
+ * a, b, p of C floats each, standing for (num, den) = (a, b) * e^p (p in
+ * natural-log units; any scaling of one state is the same state).  s_in NULL,
+ * or a = b = 0, or p = -inf, is the empty past (then this is wkv_forward).
+ * A valid non-empty state has b > 0 and finite fields.  s_out NULL: no state
+ * out.  The library writes s_out with b > 0 and p the scale it computed in.
+ * Passing the s_out of one call as the s_in of the next continues the
+ * sequence (the outputs equal those of one call over all steps, within
+ * rounding).  s_out may be the same buffer as s_in (update in place); any
+ * other overlap between s_in, s_out and k, v, y, w, u is WKV_ERR_INVALID_ARG.
+ * Other arguments, checks and layout as wkv_forward / wkv_forward_bf16;
+ * s_in / s_out need 4-byte alignment.  Sequences of at most 16 steps (and
+ * wkv_forward's too) run on a kernel that keeps each channel's state in one
+ * thread's registers and needs no workspace. */
+WKV_API wkv_status wkv_forward_state(int64_t B, int64_t T, int64_t C,
+                                     const float *w, const float *u,
+                                     const float *k, const float *v, float *y,
+                                     const float *s_in, float *s_out,
+                                     cudaStream_t stream);
+
+/* wkv_forward_state with bfloat16 k/v/y (fp32 w, u and fp32 state). */
+WKV_API wkv_status wkv_forward_bf16_state(int64_t B, int64_t T, int64_t C,
+                                          const float *w, const float *u,
+                                          const wkv_bf16_t *k, const wkv_bf16_t *v,
+                                          wkv_bf16_t *y, const float *s_in, float *s_out,
+                                          cudaStream_t stream);
 
 /* Diagonal linear scan, fp32.  a, b, h: [B, T, D] float; h0: [B, D] float or
  * NULL (zero initial state).  Pointers must be 4-byte aligned. */

@@ -9,6 +9,7 @@ raises if the library has not been built.
 
     y = wkv_forward(w, u, k, v)            # fp32 [B,T,C] k, v; [C] w, u
     y = wkv_forward_bf16(w, u, k, v)       # bf16 k, v -> bf16 y, fp32 state
+    y, s = wkv_forward_state(w, u, k, v, s_in)   # + state [B,3,C] in and out
     h = diag_scan(a, b, h0=None)           # fp32 [B,T,D]; h0 [B,D] or None
     y = wkv_forward_host(w, u, k, v)       # the same on CPU tensors, copies overlapped
 """
@@ -39,6 +40,8 @@ _SIGS = {
     "wkv_forward": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_bf16": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_noalloc": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_state": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_bf16_state": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p], _i32),
     "diag_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_bf16_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
@@ -121,6 +124,53 @@ def wkv_forward_bf16(w, u, k, v, y=None, stream=None):
     """WKV forward, bf16 k/v/y with fp32 state and fp32 w, u."""
     import torch
     return _wkv("wkv_forward_bf16", torch.bfloat16, w, u, k, v, y, stream)
+
+
+def _wkv_state(fn_name, io_dtype, w, u, k, v, s_in, y, s_out, stream):
+    import torch
+    _need(k, "k", io_dtype, 3)
+    B, _, C = k.shape
+    for t, name in ((s_in, "s_in"), (s_out, "s_out")):
+        if t is not None:
+            _need(t, name, torch.float32, 3)
+            if tuple(t.shape) != (B, 3, C):
+                raise ValueError(f"{name} must be [B, 3, C] = {(B, 3, C)}")
+    if s_out is None:
+        s_out = torch.empty((B, 3, C), dtype=torch.float32, device=k.device)
+    _need(v, "v", io_dtype, 3)
+    _need(w, "w", torch.float32, 1)
+    _need(u, "u", torch.float32, 1)
+    if k.shape != v.shape:
+        raise ValueError("k and v must have one shape")
+    if w.shape[0] != C or u.shape[0] != C:
+        raise ValueError("w and u must be [C]")
+    if y is None:
+        y = torch.empty_like(k)
+    else:
+        _need(y, "y", io_dtype, 3)
+        if y.shape != k.shape:
+            raise ValueError("y must have the shape of k")
+    _check(getattr(lib, fn_name)(B, k.shape[1], C, w.data_ptr(), u.data_ptr(), k.data_ptr(),
+                                 v.data_ptr(), y.data_ptr(),
+                                 None if s_in is None else s_in.data_ptr(), s_out.data_ptr(),
+                                 _stream_handle(stream)), fn_name)
+    return y, s_out
+
+
+def wkv_forward_state(w, u, k, v, s_in=None, y=None, s_out=None, stream=None):
+    """WKV forward, fp32, from the state ``s_in`` ([B, 3, C] planes a, b, p:
+    past sums (num, den) = (a, b) e^p; None = empty past).  Returns
+    (y, s_out), s_out the state after the last step (``s_out=s_in`` updates
+    it in place; T = 1 is one RNN-mode decoding step)."""
+    import torch
+    return _wkv_state("wkv_forward_state", torch.float32, w, u, k, v, s_in, y, s_out, stream)
+
+
+def wkv_forward_bf16_state(w, u, k, v, s_in=None, y=None, s_out=None, stream=None):
+    """wkv_forward_state with bf16 k/v/y; the state stays fp32."""
+    import torch
+    return _wkv_state("wkv_forward_bf16_state", torch.bfloat16, w, u, k, v, s_in, y, s_out,
+                      stream)
 
 
 def wkv_forward_noalloc(w, u, k, v, y=None, stream=None):
@@ -258,6 +308,7 @@ def wkv_set_fault_injection(skip_tile: int = -1, spin_limit: int = 0):
 
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan",
+           "wkv_forward_state", "wkv_forward_bf16_state",
            "wkv_forward_host", "wkv_forward_bf16_host", "diag_scan_host", "wkv_device_status",
            "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
            "wkv_get_tile_steps", "WkvError", "lib", "LIB_PATH"]

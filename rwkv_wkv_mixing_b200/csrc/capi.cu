@@ -17,6 +17,7 @@
 
 #include "chunked_scan.cuh"
 #include "persistent_scan.cuh"
+#include "serial_wkv.cuh"
 #include "wkv_b200.h"
 #include "wkv_ops.cuh"
 
@@ -368,9 +369,40 @@ wkv_status launch_persistent(const typename Op::Args &args, int64_t B, int64_t T
     return WKV_OK;
 }
 
+// Sequences of at most this many steps (single-token decoding included) run
+// on the serial kernel: one thread per (row, channel), no tiles, no workspace.
+constexpr int64_t kSerialMaxSteps = 16;
+
+template <class Op>
+wkv_status launch_serial(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
+                         cudaStream_t stream) {
+    // four channels per thread when every access can be a 4-element vector
+    const size_t vb = 4 * sizeof(typename Op::io_t);
+    const auto al = [](const void *p, size_t a) {
+        return p == nullptr || reinterpret_cast<uintptr_t>(p) % a == 0;
+    };
+    const bool vec4 = C % 4 == 0 && al(args.x0, vb) && al(args.x1, vb) && al(args.y, vb) &&
+                      al(args.s_in, 16) && al(args.s_out, 16);
+    const int vw = vec4 ? 4 : 1;
+    const int64_t blocks = (B * (C / vw) + kSerialThreads - 1) / kSerialThreads;
+    if (vec4)
+        wkv_serial_kernel<Op, 4><<<static_cast<unsigned>(blocks), kSerialThreads, 0, stream>>>(
+            args, static_cast<int>(B), static_cast<int>(T), static_cast<int>(C));
+    else
+        wkv_serial_kernel<Op, 1><<<static_cast<unsigned>(blocks), kSerialThreads, 0, stream>>>(
+            args, static_cast<int>(B), static_cast<int>(T), static_cast<int>(C));
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
 template <class Op>
 wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t C,
                     CUtensorMapDataType dt, cudaStream_t stream, int dev) {
+    if constexpr (Op::kSerialForm) {
+        if (T <= kSerialMaxSteps && (B * C + kSerialThreads - 1) / kSerialThreads <= INT32_MAX)
+            return launch_serial<Op>(args, B, T, C, stream);
+    }
     const void *ptrs[3] = {args.x0, args.x1, args.y};
     const bool tma = tma_eligible(ptrs, 3, sizeof(typename Op::io_t), T, C);
     switch (g_tile_steps.load()) {
@@ -396,8 +428,8 @@ wkv_status current_device(int *dev) {
 
 template <typename IO>
 wkv_status wkv_common(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
-                      const IO *k, const IO *v, IO *y, cudaStream_t stream,
-                      CUtensorMapDataType dt) {
+                      const IO *k, const IO *v, IO *y, const float *s_in, float *s_out,
+                      cudaStream_t stream, CUtensorMapDataType dt) {
     t_err.clear();
     bool empty = false;
     wkv_status st = check_sizes(B, T, C, &empty);
@@ -414,7 +446,19 @@ wkv_status wkv_common(int64_t B, int64_t T, int64_t C, const float *w, const flo
     if (overlaps(y, n, k, n) || overlaps(y, n, v, n) || overlaps(y, n, w, nc) ||
         overlaps(y, n, u, nc))
         return fail(WKV_ERR_INVALID_ARG, "y overlaps an input");
-    typename WkvOp<IO, sizeof(IO) == 2 ? 2 : 1>::Args args{k, v, y, w, u};
+    const size_t ns = static_cast<size_t>(B) * 3 * C * sizeof(float);
+    if (s_in != nullptr && (st = check_buffer(s_in, ns, 4, "s_in", dev)) != WKV_OK) return st;
+    if (s_out != nullptr) {
+        if ((st = check_buffer(s_out, ns, 4, "s_out", dev)) != WKV_OK) return st;
+        if (overlaps(s_out, ns, k, n) || overlaps(s_out, ns, v, n) || overlaps(s_out, ns, y, n) ||
+            overlaps(s_out, ns, w, nc) || overlaps(s_out, ns, u, nc))
+            return fail(WKV_ERR_INVALID_ARG, "s_out overlaps k, v, y, w or u");
+        if (s_in != nullptr && s_in != s_out && overlaps(s_out, ns, s_in, ns))
+            return fail(WKV_ERR_INVALID_ARG, "s_out overlaps s_in without being the same buffer");
+    }
+    if (overlaps(y, n, s_in, s_in ? ns : 0))
+        return fail(WKV_ERR_INVALID_ARG, "y overlaps s_in");
+    typename WkvOp<IO, sizeof(IO) == 2 ? 2 : 1>::Args args{k, v, y, w, u, s_in, s_out};
     return dispatch<WkvOp<IO, sizeof(IO) == 2 ? 2 : 1>>(args, B, T, C, dt, stream, dev);
 }
 
@@ -680,7 +724,8 @@ extern "C" {
 
 wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
                        const float *k, const float *v, float *y, cudaStream_t stream) {
-    return wkv_common<float>(B, T, C, w, u, k, v, y, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+    return wkv_common<float>(B, T, C, w, u, k, v, y, nullptr, nullptr, stream,
+                             CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
 }
 
 wkv_status wkv_forward_bf16(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
@@ -688,7 +733,24 @@ wkv_status wkv_forward_bf16(int64_t B, int64_t T, int64_t C, const float *w, con
                             cudaStream_t stream) {
     return wkv_common<__nv_bfloat16>(B, T, C, w, u, reinterpret_cast<const __nv_bfloat16 *>(k),
                                      reinterpret_cast<const __nv_bfloat16 *>(v),
-                                     reinterpret_cast<__nv_bfloat16 *>(y), stream,
+                                     reinterpret_cast<__nv_bfloat16 *>(y), nullptr, nullptr,
+                                     stream, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+wkv_status wkv_forward_state(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                             const float *k, const float *v, float *y, const float *s_in,
+                             float *s_out, cudaStream_t stream) {
+    return wkv_common<float>(B, T, C, w, u, k, v, y, s_in, s_out, stream,
+                             CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+}
+
+wkv_status wkv_forward_bf16_state(int64_t B, int64_t T, int64_t C, const float *w,
+                                  const float *u, const wkv_bf16_t *k, const wkv_bf16_t *v,
+                                  wkv_bf16_t *y, const float *s_in, float *s_out,
+                                  cudaStream_t stream) {
+    return wkv_common<__nv_bfloat16>(B, T, C, w, u, reinterpret_cast<const __nv_bfloat16 *>(k),
+                                     reinterpret_cast<const __nv_bfloat16 *>(v),
+                                     reinterpret_cast<__nv_bfloat16 *>(y), s_in, s_out, stream,
                                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 

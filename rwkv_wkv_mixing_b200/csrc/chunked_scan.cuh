@@ -175,7 +175,8 @@ __global__ void __launch_bounds__(NW * 32, 3)
                 const int len = max(0, min(LS, g.T - (t0 + s * LS)));
                 agg[j] = Op::combine(agg[j], Op::make(vals), static_cast<float>(len), prm[j]);
             }
-            X[j] = Op::carry0(args, b, c0 + lane * CPT + j, g.C);
+            // the state before step 0 seeds the first segment only
+            X[j] = seg == 0 ? Op::carry0(args, b, c0 + lane * CPT + j, g.C) : Op::identity();
         }
         if (chained) {
             const bool last = seg == g.n_seg - 1;
@@ -205,6 +206,13 @@ __global__ void __launch_bounds__(NW * 32, 3)
                     publish<Op, CG>(ws, g, tile, inc, kFlagIncl, epoch, lane);
                 }
             }
+        }
+        if (seg == g.n_seg - 1) {  // the state after the last step
+            const float len = static_cast<float>(min(LT, g.T - t0));
+#pragma unroll
+            for (int j = 0; j < CPT; ++j)
+                Op::store_final(args, b, c0 + lane * CPT + j, g.C,
+                                Op::combine(X[j], agg[j], len, prm[j]));
         }
 #pragma unroll
         for (int j = 0; j < CPT; ++j)

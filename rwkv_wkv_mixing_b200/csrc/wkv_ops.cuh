@@ -44,6 +44,52 @@ struct Vec<float, 2> {
 };
 
 template <>
+struct Vec<float, 4> {
+    __device__ __forceinline__ static void load(const float *p, float (&x)[4]) {
+        const float4 t = *reinterpret_cast<const float4 *>(p);
+        x[0] = t.x;
+        x[1] = t.y;
+        x[2] = t.z;
+        x[3] = t.w;
+    }
+    __device__ __forceinline__ static void store(float *p, const float (&x)[4]) {
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+};
+
+template <>
+struct Vec<__nv_bfloat16, 1> {
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&x)[1]) {
+        x[0] = __bfloat162float(*p);
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, const float (&x)[1]) {
+        *p = __float2bfloat16_rn(x[0]);  // round to nearest even
+    }
+};
+
+template <>
+struct Vec<__nv_bfloat16, 4> {
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&x)[4]) {
+        const uint2 t = *reinterpret_cast<const uint2 *>(p);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t.y));
+        x[0] = lo.x;
+        x[1] = lo.y;
+        x[2] = hi.x;
+        x[3] = hi.y;
+    }
+    // round to nearest even
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, const float (&x)[4]) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(x[2], x[3]);
+        uint2 t;
+        t.x = *reinterpret_cast<const uint32_t *>(&lo);
+        t.y = *reinterpret_cast<const uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(p) = t;
+    }
+};
+
+template <>
 struct Vec<__nv_bfloat16, 2> {
     __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&x)[2]) {
         float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
@@ -93,6 +139,7 @@ struct WkvOp {
     static constexpr int CPT = CPT_;
     static constexpr int CG = 32 * CPT;
     static constexpr int NV = 3;
+    static constexpr bool kSerialForm = true;  // has the per-step form of serial_wkv.cuh
     struct Param {
         float u, w;  // bonus and decay (natural units)
         float U, D;  // e^u, e^{-w}
@@ -105,6 +152,8 @@ struct WkvOp {
         const IO *x1;  // v [B, T, C]
         IO *y;         // y [B, T, C]
         const float *w, *u;  // [C]
+        const float *s_in;   // [B, 3, C] state before step 0, or nullptr (empty)
+        float *s_out;        // [B, 3, C] state after the last step, or nullptr
     };
     // per-thread facts pass 1 leaves for pass 2 of the same sub-chunk
     struct Scratch {
@@ -122,8 +171,26 @@ struct WkvOp {
         return q;
     }
     __device__ __forceinline__ static State identity() { return {0.f, 0.f, kNoScale}; }
-    __device__ __forceinline__ static State carry0(const Args &, int, int, int) {
-        return identity();  // empty past before the first step
+    // The state before step 0: planes a, b, p of s_in for batch row b
+    // (sums (num, den) = (a, b) e^p), or the empty past.  a = b = 0 or
+    // p = -inf is the empty past whatever the other fields hold.
+    __device__ __forceinline__ static State carry0(const Args &args, int b, int c, int C) {
+        if (args.s_in == nullptr || c >= C) return identity();
+        const float *s = args.s_in + static_cast<size_t>(b) * 3 * C + c;
+        return state_in(s[0], s[C], s[2 * C]);
+    }
+    __device__ __forceinline__ static State state_in(float a, float b, float p) {
+        if ((a == 0.f && b == 0.f) || p == -__int_as_float(0x7f800000)) return identity();
+        return {a, b, p};
+    }
+    // the state after the last step, to s_out (when given) in the same planes
+    __device__ __forceinline__ static void store_final(const Args &args, int b, int c, int C,
+                                                       const State &st) {
+        if (args.s_out == nullptr || c >= C) return;
+        float *s = args.s_out + static_cast<size_t>(b) * 3 * C + c;
+        s[0] = st.a;
+        s[C] = st.b;
+        s[2 * C] = st.p;
     }
     __device__ __forceinline__ static State nan_state() {
         const float n = __int_as_float(0x7fffffff);
@@ -342,6 +409,7 @@ struct ScanOp {
     static constexpr int CPT = 1;
     static constexpr int CG = 32;
     static constexpr int NV = 2;
+    static constexpr bool kSerialForm = false;
     struct Param {};
     struct State {
         float A, H;
@@ -361,6 +429,7 @@ struct ScanOp {
         if (args.h0 != nullptr && c < C) s.H = args.h0[static_cast<size_t>(b) * C + c];
         return s;
     }
+    __device__ __forceinline__ static void store_final(const Args &, int, int, int, const State &) {}
     __device__ __forceinline__ static State nan_state() {
         const float n = __int_as_float(0x7fffffff);
         return {n, n};

@@ -42,6 +42,10 @@ def test_host_side_argument_errors():
     assert lib.wkv_forward(0, 4, 4, None, None, None, None, None, None) == wkv.WKV_OK
     assert lib.wkv_forward_bf16(3, 0, 4, None, None, None, None, None, None) == wkv.WKV_OK
     assert lib.diag_scan(1, 1, 0, None, None, None, None, None) == wkv.WKV_OK
+    assert lib.wkv_forward_state(-2, 1, 4, None, None, None, None, None, None, None, None) == \
+        wkv.WKV_ERR_INVALID_ARG
+    assert lib.wkv_forward_bf16_state(2, 0, 4, None, None, None, None, None, None, None,
+                                      None) == wkv.WKV_OK
     # sizes beyond the int32 range of one dimension
     assert lib.wkv_forward(1, 1 << 31, 1, None, None, None, None, None, None) == \
         wkv.WKV_ERR_INVALID_ARG

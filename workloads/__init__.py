@@ -25,6 +25,14 @@ Named workloads (shapes from RWKV-4 models and the minGRU scan form):
   w = exp(U(-6,0)); u ~ N(0,1)
 * ``scan_mingru`` diagonal scan fp32, B=64 T=4096 D=256 in minGRU form:
   z = sigmoid(N(0,1)), h~ ~ N(0,1), a = 1 - z, b = z * h~, h0 = 0
+* ``wkv_decode`` WKV fp32 RNN-mode decoding, one token per sequence: B=1024
+  sequences, T=1, C=2560 (RWKV-4-3B width), k, v, w, u as ``wkv_169m``, plus
+  a state per (sequence, channel) from ``make_wkv_state``
+
+States (``make_wkv_state``): [B, 3, C] float32 planes (a, b, p) standing for
+the past sums (a, b) e^p.  Drawn with their own generator, seed + 1, in the
+order: the past mean m ~ N(0, 1), ln b ~ U(-1, 1), p ~ N(0, p_sigma); then
+a = m * b (so a / b = m stays within the range of v).
 """
 from __future__ import annotations
 
@@ -36,7 +44,7 @@ import numpy as np
 __all__ = [
     "WkvSpec", "ScanSpec", "WORKLOADS", "WkvInputs", "ScanInputs",
     "make_wkv", "make_scan", "bf16_round", "bf16_bits", "bf16_bits_to_f32",
-    "get_workload",
+    "get_workload", "make_wkv_state",
 ]
 
 
@@ -53,6 +61,7 @@ class WkvSpec:
     w_log: tuple = ("normal", -0.5, 0.5)   # log w ~ N(m, s) or U(lo, hi)
     u_sigma: float = 0.5          # u ~ N(0, u_sigma)
     seed: int = 0
+    state: bool = False           # the workload starts from a drawn state
 
     @property
     def elements(self) -> int:
@@ -80,6 +89,8 @@ WORKLOADS = {
     "wkv_3b_bf16": WkvSpec("wkv_3b_bf16", 8, 4096, 2560, "bf16", 1.0, 1.0, ("uniform", -3.0, 1.0), 0.5),
     "wkv_long": WkvSpec("wkv_long", 1, 131072, 1024, "f32", 3.0, 1.0, ("uniform", -6.0, 0.0), 1.0),
     "scan_mingru": ScanSpec("scan_mingru", 64, 4096, 256),
+    "wkv_decode": WkvSpec("wkv_decode", 1024, 1, 2560, "f32", 1.0, 1.0, ("uniform", -3.0, 1.0),
+                          0.5, state=True),
 }
 
 
@@ -124,6 +135,7 @@ class WkvInputs:
     v: np.ndarray   # [B, T, C] float32
     k_bits: Optional[np.ndarray] = None
     v_bits: Optional[np.ndarray] = None
+    s_in: Optional[np.ndarray] = None   # [B, 3, C] float32 when spec.state
 
 
 @dataclasses.dataclass
@@ -160,10 +172,20 @@ def make_wkv(spec, *, B=None, T=None, C=None, seed=None) -> WkvInputs:
     v = rng.normal(0.0, spec.v_sigma, size=shape).astype(np.float32)
     w = np.exp(_draw_log_w(rng, spec.w_log, spec.C)).astype(np.float32)
     u = rng.normal(0.0, spec.u_sigma, size=spec.C).astype(np.float32)
+    s_in = make_wkv_state(spec.B, spec.C, spec.seed) if spec.state else None
     if spec.dtype == "bf16":
         kb, vb = bf16_bits(k), bf16_bits(v)
-        return WkvInputs(spec, w, u, bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), kb, vb)
-    return WkvInputs(spec, w, u, k, v)
+        return WkvInputs(spec, w, u, bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), kb, vb, s_in)
+    return WkvInputs(spec, w, u, k, v, s_in=s_in)
+
+
+def make_wkv_state(B: int, C: int, seed: int = 0, p_sigma: float = 2.0) -> np.ndarray:
+    """A random non-empty WKV state [B, 3, C] float32 (planes a, b, p)."""
+    rng = np.random.default_rng(seed + 1)
+    mean = rng.normal(0.0, 1.0, size=(B, C))
+    b = np.exp(rng.uniform(-1.0, 1.0, size=(B, C)))
+    p = rng.normal(0.0, p_sigma, size=(B, C))
+    return np.stack([mean * b, b, p], axis=1).astype(np.float32)
 
 
 def make_scan(spec, *, B=None, T=None, D=None, seed=None, with_h0=None) -> ScanInputs:
