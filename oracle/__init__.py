@@ -21,6 +21,12 @@ Pieces (all float64; each cites the page it follows):
   from a given state (the past sums before step 0, RNN mode) and returning
   the state after the last step; ``wkv_direct_points(..., s_in=)`` likewise.
   A state is [B, 3, C]: planes a, b, p with (num, den) = (a, b) e^p.
+* ``token_shift``         -- the token-shift interpolation that feeds the
+  time-mixing projections, mu x_t + (1 - mu) x_{t-1} (eqs. (11)-(13) of
+  "RWKV：基于RNN的LLM", section 二.1; x_{-1} is the layer's saved last token,
+  "last_x", of the HarmonyOS RWKV article's time-mixing code section, or 0).
+* ``sigmoid`` / ``wkv_gated`` -- the receptance gate sigma(r_t) (.) wkv_t of
+  eq. (15) of the same page and of the LRU review's RWKV variant.
 * ``wkv_slru_ratio_np``   -- the "RWKV = ratio of two SLRUs" form from the
   review of "Resurrecting Recurrent Neural Networks for Long Sequences"
   (section on the RWKV variant), unstabilised; |k| small only.
@@ -52,6 +58,7 @@ __all__ = [
     "build", "max_threads", "wkv_direct", "wkv_direct_points", "wkv_direct_np",
     "wkv_rnn", "wkv_slru_ratio_np", "scan_rnn", "scan_direct_points",
     "wkv_direct_state", "wkv_rnn_state", "state_mean_logden",
+    "token_shift", "sigmoid", "wkv_gated",
 ]
 
 
@@ -274,3 +281,45 @@ def scan_direct_points(a, b, h0, points, nthreads: int = 0) -> np.ndarray:
                                      None if h0 is None else _ptr(h0),
                                      pts.size, _ptr(pts), _ptr(out), nthreads)
     return out
+
+
+# ---------------------------------------------------------------------------
+# The elementwise steps around WKV in the time-mixing block
+# ---------------------------------------------------------------------------
+def token_shift(x, mu, x_prev=None):
+    """Token shift ("RWKV：基于RNN的LLM", section 二.1, eqs. (11)-(13)): for
+    each mixing vector mu_m (rows of ``mu``, [n_mix, C]),
+
+        out[m, b, t] = mu_m * x[b, t] + (1 - mu_m) * x[b, t-1],
+
+    with x[b, -1] = x_prev[b] (the token before this call, [B, C]) or 0.
+    Returns (out [n_mix, B, T, C], x_last [B, C] = x[:, T-1]), float64.
+    The pages print eqs. (16)-(17) with a minus before (1 - mu); the plus of
+    eqs. (11)-(13) is the reading taken everywhere."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = np.asarray(mu, dtype=np.float64)
+    if mu.ndim == 1:
+        mu = mu[None]
+    B, T, C = x.shape
+    if mu.shape[1] != C:
+        raise ValueError("mu must be [n_mix, C]")
+    prev = np.zeros((B, 1, C)) if x_prev is None else \
+        np.asarray(x_prev, dtype=np.float64).reshape(B, 1, C)
+    shifted = np.concatenate([prev, x[:, :-1]], axis=1)        # x_{t-1}
+    out = np.stack([m * x + (1.0 - m) * shifted for m in mu])  # [n_mix, B, T, C]
+    return out, x[:, -1].copy()
+
+
+def sigmoid(r):
+    """The logistic function 1 / (1 + e^{-r}), float64."""
+    r = np.asarray(r, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-r))
+
+
+def wkv_gated(w, u, k, v, r, s_in=None):
+    """sigma(r_t) (.) wkv_t (eq. (15) of "RWKV：基于RNN的LLM" before the output
+    projection; the LRU review's RWKV variant), wkv from the RNN-mode oracle,
+    optionally from a state.  Returns (out, s_out)."""
+    y, s_out = wkv_rnn_state(w, u, k, v, s_in)
+    return sigmoid(r) * y, s_out

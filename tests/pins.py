@@ -354,6 +354,117 @@ def run_wkv_state_pins(fn):
 
 
 # ---------------------------------------------------------------------------
+# Token shift: fn(x, mu, x_prev) -> (out [n_mix, B, T, C], x_last [B, C])
+# ---------------------------------------------------------------------------
+def token_shift_worked_example(fn, tol=1e-15):
+    g = read_golden("token_shift_worked_example.txt")
+    x = np.array([float(a) for a in g["x"]]).reshape(1, 3, 2)
+    x_prev = np.array([float(a) for a in g["x_prev"]]).reshape(1, 2)
+    mu = np.array([float(a) for a in g["mu"]]).reshape(2, 2)
+    out, last = fn(x, mu, x_prev)
+    fails = []
+    msg = _close(out, np.array([float(a) for a in g["out"]]).reshape(2, 1, 3, 2), tol)
+    if msg: fails.append(f"token shift worked example: {msg}")
+    msg = _close(last, np.array([float(a) for a in g["x_last"]]).reshape(1, 2), 0.0)
+    if msg: fails.append(f"token shift last token: {msg}")
+    return fails
+
+
+def token_shift_special_cases(fn, tol=0.0):
+    """mu = 1 keeps x_t, mu = 0 takes x_{t-1} (x_prev at t = 0), mu = 1/2
+    averages the two; no x_prev is a zero x_prev."""
+    rng = np.random.default_rng(31)
+    B, T, C = 2, 9, 5
+    x = rng.normal(0, 1, (B, T, C)); xp = rng.normal(0, 1, (B, C))
+    mu = np.stack([np.ones(C), np.zeros(C), np.full(C, 0.5)])
+    out, last = fn(x, mu, xp)
+    shifted = np.concatenate([xp[:, None], x[:, :-1]], axis=1)
+    fails = []
+    for m, want, name in ((0, x, "mu = 1"), (1, shifted, "mu = 0"),
+                          (2, 0.5 * (x + shifted), "mu = 1/2")):
+        msg = _close(np.asarray(out)[m], want, tol if m < 2 else 1e-15)
+        if msg: fails.append(f"token shift {name}: {msg}")
+    msg = _close(last, x[:, -1], 0.0)
+    if msg: fails.append(f"token shift last token: {msg}")
+    o0, _ = fn(x, mu, None)
+    o1, _ = fn(x, mu, np.zeros((B, C)))
+    msg = _close(o0, o1, 0.0)
+    if msg: fails.append(f"token shift without x_prev: {msg}")
+    return fails
+
+
+def token_shift_chaining(fn, tol=1e-15):
+    """Two calls handing on the last token equal one call."""
+    rng = np.random.default_rng(32)
+    B, T, C = 3, 20, 6
+    x = rng.normal(0, 1, (B, T, C)); xp = rng.normal(0, 1, (B, C))
+    mu = rng.uniform(0, 1, (3, C))
+    out, last = fn(x, mu, xp)
+    o1, l1 = fn(x[:, :7], mu, xp)
+    o2, l2 = fn(x[:, 7:], mu, l1)
+    msg = _close(np.concatenate([o1, o2], axis=2), out, tol) or _close(l2, last, 0.0)
+    return [f"token shift chaining: {msg}"] if msg else []
+
+
+TOKEN_SHIFT_PINS = [token_shift_worked_example, token_shift_special_cases, token_shift_chaining]
+
+
+def run_token_shift_pins(fn):
+    fails = []
+    for pin in TOKEN_SHIFT_PINS:
+        try:
+            fails += pin(fn)
+        except Exception as e:
+            fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
+    return fails
+
+
+# ---------------------------------------------------------------------------
+# Gated WKV: fn(w, u, k, v, r) -> sigma(r) (.) wkv
+# ---------------------------------------------------------------------------
+def gate_worked_example(fn, tol=1e-12):
+    g = read_golden("wkv_gate_worked_example.txt")
+    w = np.array([-np.log(float(g["w_exp_neg"][0]))])
+    u = np.array([np.log(float(g["u_exp"][0]))])
+    k = np.log(np.array([float(x) for x in g["k_exp"]]))[None, :, None]
+    v = np.array([float(x) for x in g["v"]])[None, :, None]
+    r = np.log(np.array([float(x) for x in g["r_exp"]]))[None, :, None]
+    msg = _close(fn(w, u, k, v, r), np.array([float(x) for x in g["out"]])[None, :, None], tol)
+    return [f"gate worked example: {msg}"] if msg else []
+
+
+def gate_limits(fn, tol=1e-12):
+    """r = +60 passes wkv through (sigma = 1 in float64); r = 0 halves it;
+    sigma(r) + sigma(-r) = 1; r = -60 closes the gate."""
+    w, u, k, v = _rand_wkv(33, B=2, T=30, C=4)
+    rng = np.random.default_rng(33)
+    r = rng.normal(0, 2, k.shape)
+    open_ = np.asarray(fn(w, u, k, v, np.full(k.shape, 60.0)))
+    fails = [f"gate open, stateless pins: {f}" for f in run_wkv_pins(
+        lambda w_, u_, k_, v_: fn(w_, u_, k_, v_, np.full(np.shape(k_), 60.0)))]
+    msg = _close(fn(w, u, k, v, np.zeros(k.shape)), 0.5 * open_, tol)
+    if msg: fails.append(f"gate at r = 0: {msg}")
+    msg = _close(np.asarray(fn(w, u, k, v, r)) + np.asarray(fn(w, u, k, v, -r)), open_, tol)
+    if msg: fails.append(f"gate symmetry: {msg}")
+    msg = _close(fn(w, u, k, v, np.full(k.shape, -60.0)), np.zeros(k.shape), 1e-25)
+    if msg: fails.append(f"gate closed: {msg}")
+    return fails
+
+
+GATE_PINS = [gate_worked_example, gate_limits]
+
+
+def run_gate_pins(fn):
+    fails = []
+    for pin in GATE_PINS:
+        try:
+            fails += pin(fn)
+        except Exception as e:
+            fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
+    return fails
+
+
+# ---------------------------------------------------------------------------
 # diagonal scan pins
 # ---------------------------------------------------------------------------
 def scan_worked_example(fn, tol=1e-12):

@@ -279,6 +279,65 @@ def test_planted_mistake_in_state_oracle_is_caught(name, tmp_path):
     assert pins.run_wkv_state_pins(mut) != []
 
 
+# --- token shift and receptance gate ---------------------------------------
+def test_token_shift_oracle_passes_pins():
+    assert pins.run_token_shift_pins(oracle.token_shift) == []
+
+
+def _token_shift_variant(kind):
+    def fn(x, mu, x_prev):
+        x = np.asarray(x, float); mu = np.asarray(mu, float)
+        B, T, C = x.shape
+        prev = np.zeros((B, 1, C)) if (x_prev is None or kind == "prev_ignored") else \
+            np.asarray(x_prev, float).reshape(B, 1, C)
+        sh = np.concatenate([prev, x[:, :-1]], axis=1)
+        if kind == "shift_two":
+            sh = np.concatenate([prev, prev, x[:, :-2]], axis=1)[:, :T]
+        outs = []
+        for m in mu:
+            if kind == "mu_swapped":
+                outs.append(m * sh + (1 - m) * x)
+            elif kind == "minus_reading":   # eqs. (16)-(17) as printed
+                outs.append(m * x - (1 - m) * sh)
+            else:
+                outs.append(m * x + (1 - m) * sh)
+        last = x[:, -2] if kind == "last_off_by_one" else x[:, -1]
+        return np.stack(outs), last
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["mu_swapped", "minus_reading", "prev_ignored", "shift_two",
+                                  "last_off_by_one"])
+def test_planted_mistake_in_token_shift_is_caught(kind):
+    assert pins.run_token_shift_pins(_token_shift_variant("none")) == []
+    assert pins.run_token_shift_pins(_token_shift_variant(kind)) != []
+
+
+def _gate(w, u, k, v, r):
+    return oracle.wkv_gated(w, u, k, v, r)[0]
+
+
+def test_gate_oracle_passes_pins():
+    assert pins.run_gate_pins(_gate) == []
+    assert abs(float(oracle.sigmoid(np.log(3.0))) - 0.75) < 1e-16
+    assert float(oracle.sigmoid(-800.0)) == 0.0 and float(oracle.sigmoid(800.0)) == 1.0
+
+
+@pytest.mark.parametrize("kind", ["tanh", "neg", "ungated", "gate_on_v"])
+def test_planted_mistake_in_gate_is_caught(kind):
+    def fn(w, u, k, v, r):
+        y = oracle.wkv_rnn(w, u, k, v)
+        r = np.asarray(r, float)
+        if kind == "tanh":
+            return np.tanh(r) * y
+        if kind == "neg":
+            return oracle.sigmoid(-r) * y
+        if kind == "ungated":
+            return y
+        return oracle.wkv_rnn(w, u, k, oracle.sigmoid(r) * np.asarray(v))
+    assert pins.run_gate_pins(fn) != []
+
+
 # --- diagonal scan ---------------------------------------------------------
 def scan_rnn(a, b, h0):
     return oracle.scan_rnn(a, b, h0)
