@@ -188,87 +188,126 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 class DeviceWorkload:
     """Inputs resident in HBM, rotated over `n_sets` copies, and the C-ABI
-    call of one step with raw device pointers."""
+    call of one step with raw device pointers.
+
+    kinds: "wkv" (plain, with a state read and written in place, or with the
+    receptance gate), "scan" (diagonal scan), "shift" (token shift, the
+    saved last token read and written in place)."""
 
     def __init__(self, name, torch, lib, l2_bytes):
         self.name = name
-        self.spec = workloads.WORKLOADS[name]
+        self.spec = spec = workloads.WORKLOADS[name]
         self.torch = torch
         self.lib = lib
         dev = torch.device("cuda", torch.cuda.current_device())
-        self.is_scan = isinstance(self.spec, workloads.ScanSpec)
-        if self.is_scan:
+        self.dev = dev
+        self.consts = {}
+        self.has_state = self.gated = False
+        if isinstance(spec, workloads.ScanSpec):
+            self.kind = "scan"
             x = workloads.make_scan(name)
             B, T, C = x.a.shape
-            self.host = {"x0": x.a, "x1": x.b}
-            self.dtype, self.es, self.tdtype = "f32", 4, torch.float32
-            self.params = []
-            self.param_bytes = 0
+            self.dtype, self.es = "f32", 4
+            self.host = {"a": x.a, "b": x.b}
+            self.outputs = {"h": (B, T, C)}
+            alg = 12 * B * T * C
+        elif isinstance(spec, workloads.ShiftSpec):
+            self.kind = "shift"
+            x = workloads.make_token_shift(name)
+            B, T, C = x.x.shape
+            bf = spec.dtype == "bf16"
+            self.dtype, self.es = spec.dtype, 2 if bf else 4
+            self.host = {"x": x.x_bits.view(np.int16) if bf else x.x,
+                         "xp": x.x_prev_bits.view(np.int16) if bf else x.x_prev}
+            self.consts["mu"] = torch.from_numpy(x.mu).to(dev)
+            self.n_mix = x.mu.shape[0]
+            self.outputs = {"out": (self.n_mix, B, T, C)}
+            alg = self.es * B * T * C * (1 + self.n_mix) + 2 * self.es * B * C + 4 * self.n_mix * C
         else:
+            self.kind = "wkv"
             x = workloads.make_wkv(name)
             B, T, C = x.k.shape
-            if x.spec.dtype == "bf16":
-                self.host = {"x0": x.k_bits.view(np.int16), "x1": x.v_bits.view(np.int16)}
-                self.dtype, self.es, self.tdtype = "bf16", 2, torch.bfloat16
-            else:
-                self.host = {"x0": x.k, "x1": x.v}
-                self.dtype, self.es, self.tdtype = "f32", 4, torch.float32
-            self.params = [torch.from_numpy(x.w).to(dev), torch.from_numpy(x.u).to(dev)]
-            self.param_bytes = 2 * 4 * C
+            bf = spec.dtype == "bf16"
+            self.dtype, self.es = spec.dtype, 2 if bf else 4
+            self.host = {"k": x.k_bits.view(np.int16) if bf else x.k,
+                         "v": x.v_bits.view(np.int16) if bf else x.v}
+            self.gated = x.r is not None
+            if self.gated:
+                self.host["r"] = x.r_bits.view(np.int16) if bf else x.r
+            self.has_state = x.s_in is not None
+            if self.has_state:
+                self.host["s"] = x.s_in
+            self.consts["w"] = torch.from_numpy(x.w).to(dev)
+            self.consts["u"] = torch.from_numpy(x.u).to(dev)
+            self.outputs = {"y": (B, T, C)}
+            alg = self.es * B * T * C * (4 if self.gated else 3) + 8 * C + \
+                (24 * B * C if self.has_state else 0)
         self.inputs = x
         self.B, self.T, self.C = B, T, C
         self.elements = B * T * C
-        # a workload with a state reads it and writes it back (in place)
-        self.has_state = getattr(x, "s_in", None) is not None
-        self.state_bytes = 2 * 3 * 4 * B * C if self.has_state else 0
-        self.alg_bytes = 3 * self.es * self.elements + self.param_bytes + self.state_bytes
-        set_bytes = 3 * self.es * self.elements + self.state_bytes
-        self.set_bytes = set_bytes
-        self.n_sets = 1 if set_bytes >= 3 * l2_bytes else int(np.ceil(3 * l2_bytes / set_bytes)) + 1
-        x0 = self._to_dev(self.host["x0"], dev)
-        x1 = self._to_dev(self.host["x1"], dev)
-        s0 = torch.from_numpy(x.s_in).to(dev) if self.has_state else None
+        self.alg_bytes = alg
+        # bytes one step touches, for sizing the rotation against L2
+        self.set_bytes = alg
+        self.n_sets = 1 if alg >= 3 * l2_bytes else int(np.ceil(3 * l2_bytes / alg)) + 1
+        first = {k: self._to_dev(v) for k, v in self.host.items()}
         self.sets = []
         for i in range(self.n_sets):
-            a = x0 if i == 0 else x0.clone()
-            b = x1 if i == 0 else x1.clone()
-            st = None if s0 is None else (s0 if i == 0 else s0.clone())
-            self.sets.append((a, b, torch.empty_like(a), st))
+            st = {k: (t if i == 0 else t.clone()) for k, t in first.items()}
+            for k, shape in self.outputs.items():
+                st[k] = torch.empty(shape, dtype=first[next(iter(first))].dtype, device=dev)
+            self.sets.append(st)
         self.stream = torch.cuda.current_stream()
 
-    def _to_dev(self, arr, dev):
+    def _to_dev(self, arr):
         t = self.torch.from_numpy(np.ascontiguousarray(arr))
-        if self.dtype == "bf16":
+        if arr.dtype == np.int16:
             t = t.view(self.torch.bfloat16)
-        return t.to(dev)
+        return t.to(self.dev)
 
-    def call(self, x0, x1, y, st=None):
-        """One C-ABI call on torch's current stream (the capture stream while a
-        graph is being captured)."""
+    def api(self):
+        if self.kind == "scan":
+            return "diag_scan"
+        bf = "_bf16" if self.dtype == "bf16" else ""
+        if self.kind == "shift":
+            return "wkv_token_shift" + bf
+        if self.gated:
+            return f"wkv_forward{bf}_gated"
+        return f"wkv_forward{bf}_state" if self.has_state else f"wkv_forward{bf}"
+
+    def call(self, d, stream=None):
+        """One C-ABI call on `stream` (default: torch's current stream, the
+        capture stream while a graph is being captured) over the buffers `d`."""
         lib = self.lib
-        sh = self.torch.cuda.current_stream().cuda_stream
-        if self.is_scan:
-            return lib.diag_scan(self.B, self.T, self.C, x0.data_ptr(), x1.data_ptr(), None,
-                                 y.data_ptr(), sh)
-        if st is not None:   # state in and out, updated in place
-            fn = lib.wkv_forward_bf16_state if self.dtype == "bf16" else lib.wkv_forward_state
-            return fn(self.B, self.T, self.C, self.params[0].data_ptr(),
-                      self.params[1].data_ptr(), x0.data_ptr(), x1.data_ptr(), y.data_ptr(),
-                      st.data_ptr(), st.data_ptr(), sh)
-        fn = lib.wkv_forward_bf16 if self.dtype == "bf16" else lib.wkv_forward
-        return fn(self.B, self.T, self.C, self.params[0].data_ptr(), self.params[1].data_ptr(),
-                  x0.data_ptr(), x1.data_ptr(), y.data_ptr(), sh)
+        sh = (stream or self.torch.cuda.current_stream()).cuda_stream
+        B, T, C = self.B, self.T, self.C
+        fn = getattr(lib, self.api())
+        if self.kind == "scan":
+            return fn(B, T, C, d["a"].data_ptr(), d["b"].data_ptr(), None, d["h"].data_ptr(), sh)
+        if self.kind == "shift":   # last token handed on in place
+            return fn(B, T, C, self.n_mix, d["x"].data_ptr(), d["xp"].data_ptr(),
+                      self.consts["mu"].data_ptr(), d["out"].data_ptr(), d["xp"].data_ptr(), sh)
+        w, u = self.consts["w"].data_ptr(), self.consts["u"].data_ptr()
+        s = d["s"].data_ptr() if self.has_state else None   # state updated in place
+        if self.gated:
+            return fn(B, T, C, w, u, d["k"].data_ptr(), d["v"].data_ptr(), d["r"].data_ptr(),
+                      d["y"].data_ptr(), s, s, sh)
+        if self.has_state:
+            return fn(B, T, C, w, u, d["k"].data_ptr(), d["v"].data_ptr(), d["y"].data_ptr(),
+                      s, s, sh)
+        return fn(B, T, C, w, u, d["k"].data_ptr(), d["v"].data_ptr(), d["y"].data_ptr(), sh)
 
     def kernel(self):
         """The kernel a step launches (the library's dispatch rule)."""
-        if not self.is_scan and self.T <= 16:
+        if self.kind == "shift":
+            return "token_shift_kernel"
+        if self.kind == "wkv" and self.T <= 16:
             return "wkv_serial_kernel"
         if self.lib.wkv_get_tile_steps() in (8, 32):
             return "chunked_scan_kernel"
         return "persistent_scan_kernel"
 
     def step(self, i):
-        st = self.call(*self.sets[i % self.n_sets])
+        st = self.call(self.sets[i % self.n_sets])
         if st != 0:
             raise RuntimeError(f"library call failed: {st}: {self.lib.wkv_last_error().decode()}")
 
@@ -359,51 +398,57 @@ def host_overhead_us(torch, wl, n=200):
 
 
 def e2e_leg(torch, wl, steps):
-    """Through the C ABI with host buffers: every step is one call of the
-    library's host-buffer entry point on pinned host memory, which uploads the
-    step's inputs, computes and downloads the result (overlapped in chunks)
-    and returns when the result is on the host.  Timed with CUDA events on the
-    current stream around the synchronous calls."""
+    """End to end through the library with host buffers, timed with CUDA
+    events on the current stream around synchronous steps.  WKV and the scan
+    go through the library's host-buffer entry points (upload, compute and
+    download overlapped in chunks inside the call).  The entry points with no
+    host-buffer form (state, gate, token shift) run as a user would: pinned
+    host -> device copies of the step's inputs, the device call, device ->
+    host copies of its outputs, on one stream, synchronised."""
     lib = wl.lib
-    hx0 = torch.from_numpy(np.ascontiguousarray(wl.host["x0"])).pin_memory()
-    hx1 = torch.from_numpy(np.ascontiguousarray(wl.host["x1"])).pin_memory()
-    hy = torch.empty_like(hx0).pin_memory()
-    hp = [p.cpu().pin_memory() for p in wl.params]
-    hs = None
-    if wl.has_state:
-        # no host-buffer entry point takes a state: the user-side sequence is
-        # pinned copies in, the device call, copies out, on one stream
-        hs = torch.from_numpy(wl.inputs.s_in).pin_memory()
-        dx0, dx1, dy, ds = (torch.empty(t.shape, dtype=t.dtype, device="cuda")
-                            for t in (hx0, hx1, hy, hs))
-        if wl.dtype == "bf16":
-            dx0, dx1, dy = (t.view(torch.bfloat16) for t in (dx0, dx1, dy))
-        dp = wl.params
-        api = ("wkv_forward_bf16_state" if wl.dtype == "bf16" else "wkv_forward_state") + \
-            " with pinned copies on one stream"
-        fn = getattr(lib, "wkv_forward_bf16_state" if wl.dtype == "bf16" else "wkv_forward_state")
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in wl.host.items()}
+    outs = {k: torch.empty(shape, dtype=torch.int16 if wl.dtype == "bf16" else torch.float32
+                           ).pin_memory() for k, shape in wl.outputs.items()}
+    hp = {k: t.cpu().pin_memory() for k, t in wl.consts.items()}
+    host_api = wl.kind == "scan" or (wl.kind == "wkv" and not wl.gated and not wl.has_state)
+    if host_api:
+        if wl.kind == "scan":
+            api = "diag_scan_host"
+            call = lambda: lib.diag_scan_host(wl.B, wl.T, wl.C, pinned["a"].data_ptr(),  # noqa: E731
+                                              pinned["b"].data_ptr(), None, outs["h"].data_ptr())
+        else:
+            api = "wkv_forward_bf16_host" if wl.dtype == "bf16" else "wkv_forward_host"
+            fn = getattr(lib, api)
+            call = lambda: fn(wl.B, wl.T, wl.C, hp["w"].data_ptr(), hp["u"].data_ptr(),  # noqa: E731
+                              pinned["k"].data_ptr(), pinned["v"].data_ptr(),
+                              outs["y"].data_ptr())
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values()) + \
+            sum(t.numel() * t.element_size() for t in hp.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    else:
+        api = wl.api() + " with pinned copies on one stream"
+        d = {k: torch.empty(t.shape, dtype=t.dtype, device=wl.dev) for k, t in pinned.items()}
+        d.update({k: torch.empty(t.shape, dtype=t.dtype, device=wl.dev) for k, t in outs.items()})
+        if wl.dtype == "bf16":   # bf16 storage travels as int16 bits
+            d = {k: (t.view(torch.bfloat16) if t.dtype == torch.int16 else t)
+                 for k, t in d.items()}
+        back = dict(outs)
+        # in-place state / last token comes back too
+        for k in ("s", "xp"):
+            if k in pinned:
+                back[k] = pinned[k]
 
         def call():
             stream = torch.cuda.current_stream()
-            dx0.copy_(hx0.view(dx0.dtype) if wl.dtype == "bf16" else hx0, non_blocking=True)
-            dx1.copy_(hx1.view(dx1.dtype) if wl.dtype == "bf16" else hx1, non_blocking=True)
-            ds.copy_(hs, non_blocking=True)
-            st = fn(wl.B, wl.T, wl.C, dp[0].data_ptr(), dp[1].data_ptr(), dx0.data_ptr(),
-                    dx1.data_ptr(), dy.data_ptr(), ds.data_ptr(), ds.data_ptr(),
-                    stream.cuda_stream)
-            hy.copy_(dy.view(hy.dtype) if wl.dtype == "bf16" else dy, non_blocking=True)
-            hs.copy_(ds, non_blocking=True)
+            for k, t in pinned.items():
+                d[k].view(t.dtype).copy_(t, non_blocking=True)
+            st = wl.call(d, stream)
+            for k, t in back.items():
+                t.copy_(d[k].view(t.dtype), non_blocking=True)
             stream.synchronize()
             return st
-    elif wl.is_scan:
-        api = "diag_scan_host"
-        call = lambda: lib.diag_scan_host(wl.B, wl.T, wl.C, hx0.data_ptr(), hx1.data_ptr(),  # noqa: E731
-                                          None, hy.data_ptr())
-    else:
-        api = "wkv_forward_bf16_host" if wl.dtype == "bf16" else "wkv_forward_host"
-        fn = getattr(lib, api)
-        call = lambda: fn(wl.B, wl.T, wl.C, hp[0].data_ptr(), hp[1].data_ptr(),  # noqa: E731
-                          hx0.data_ptr(), hx1.data_ptr(), hy.data_ptr())
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+        d2h = sum(t.numel() * t.element_size() for t in back.values())
 
     def one():
         st = call()
@@ -423,11 +468,6 @@ def e2e_leg(torch, wl, steps):
     b.synchronize()
     wall_ms = (time.perf_counter() - t0) / steps * 1e3
     ms = a.elapsed_time(b) / steps
-    h2d = hx0.numel() * hx0.element_size() * 2 + (wl.param_bytes if hs is None else 0)
-    d2h = hy.numel() * hy.element_size()
-    if hs is not None:   # the state travels both ways
-        h2d += hs.numel() * 4
-        d2h += hs.numel() * 4
     return {"value": wl.elements / (ms / 1e3), "unit": "elem/s", "ms_per_step": ms,
             "wall_ms_per_step": wall_ms, "steps": steps, "api": api,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -450,6 +490,15 @@ def oracle_runner(name, max_elements=None):
         a, b = np.ascontiguousarray(a[:rows]), np.ascontiguousarray(b[:rows])
         fn = lambda: oracle.scan_rnn(a, b, None)   # noqa: E731
         return fn, rows * T * C, f"{rows} of {B} batch rows (all T={T}, D={C})"
+    if isinstance(spec, workloads.ShiftSpec):
+        x = workloads.make_token_shift(name)
+        B, T, C = x.x.shape
+        rows = B if max_elements is None else max(1, min(B, max_elements // (T * C)))
+        xs = np.ascontiguousarray(x.x[:rows], dtype=np.float64)
+        xp = np.ascontiguousarray(x.x_prev[:rows], dtype=np.float64)
+        mu = x.mu.astype(np.float64)
+        fn = lambda: oracle.token_shift(xs, mu, xp)   # noqa: E731
+        return fn, rows * T * C, f"{rows} of {B} batch rows (all T={T}, C={C})"
     x = workloads.make_wkv(name)
     k, v = x.k.astype(np.float64), x.v.astype(np.float64)
     w, u = x.w.astype(np.float64), x.u.astype(np.float64)
@@ -461,8 +510,12 @@ def oracle_runner(name, max_elements=None):
             chans = max(1, min(C, max_elements // T))
     k = np.ascontiguousarray(k[:rows, :, :chans]); v = np.ascontiguousarray(v[:rows, :, :chans])
     w, u = w[:chans], u[:chans]
-    if x.s_in is not None:
-        s_in = np.ascontiguousarray(x.s_in[:rows, :, :chans], dtype=np.float64)
+    s_in = None if x.s_in is None else \
+        np.ascontiguousarray(x.s_in[:rows, :, :chans], dtype=np.float64)
+    if x.r is not None:
+        r = np.ascontiguousarray(x.r[:rows, :, :chans], dtype=np.float64)
+        fn = lambda: oracle.wkv_gated(w, u, k, v, r, s_in)   # noqa: E731
+    elif s_in is not None:
         fn = lambda: oracle.wkv_rnn_state(w, u, k, v, s_in)   # noqa: E731
     else:
         fn = lambda: oracle.wkv_rnn(w, u, k, v)   # noqa: E731
@@ -506,13 +559,13 @@ def run_reference(args):
     value = n * args.steps / dt
     spec = workloads.WORKLOADS[args.workload]
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "elem/s",
+        "impl": "reference", "metric": metric_for(spec), "value": value, "unit": "elem/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(spec, args.workload),
         "cpu_baseline": {"value": value, "unit": "elem/s", "cores": oracle.max_threads(),
-                         "kind": "oracle", "sample": f"{desc} per step, float64 RNN-mode oracle"},
+                         "kind": "oracle", "sample": f"{desc} per step, float64 oracle"},
         "e2e": {"value": value, "unit": "elem/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -538,9 +591,24 @@ def workload_config(spec, name):
     if isinstance(spec, workloads.ScanSpec):
         return {"workload": name, "op": "diag_scan", "B": spec.B, "T": spec.T, "D": spec.D,
                 "io": "f32"}
-    op = "wkv_forward" + ("_bf16" if spec.dtype == "bf16" else "") + \
-        ("_state (state [B,3,C] fp32 read and written in place)" if spec.state else "")
+    bf = "_bf16" if spec.dtype == "bf16" else ""
+    if isinstance(spec, workloads.ShiftSpec):
+        return {"workload": name, "op": f"wkv_token_shift{bf} ({spec.n_mix} mixing vectors, "
+                "last token read and written in place)", "B": spec.B, "T": spec.T, "C": spec.C,
+                "io": spec.dtype}
+    if spec.gated:
+        op = f"wkv_forward{bf}_gated (sigma(r) * wkv in one pass)"
+    elif spec.state:
+        op = f"wkv_forward{bf}_state (state [B,3,C] fp32 read and written in place)"
+    else:
+        op = f"wkv_forward{bf}"
     return {"workload": name, "op": op, "B": spec.B, "T": spec.T, "C": spec.C, "io": spec.dtype}
+
+
+def metric_for(spec):
+    if isinstance(spec, workloads.ShiftSpec):
+        return "token shift B·T·C elems/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+    return METRIC
 
 
 # ---------------------------------------------------------------------------
@@ -653,7 +721,7 @@ def main(argv=None):
                                          if args.launch == "graph" else ""),
                 "gpu": props.name, "sms": props.multi_processor_count})
     line = {
-        "metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world,
+        "metric": metric_for(wl.spec), "value": value, "unit": "elem/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic (seeded, distributions of the named workload)",

@@ -141,6 +141,56 @@ WKV_API wkv_status wkv_forward_bf16_state(int64_t B, int64_t T, int64_t C,
                                           wkv_bf16_t *y, const float *s_in, float *s_out,
                                           cudaStream_t stream);
 
+/* WKV forward with the receptance gate fused into its output: eq. (15) of
+ * "RWKV：基于RNN的LLM" (section 二.1) applies sigma(r_t) (.) wkv_t before the
+ * output projection (the same gate closes the RWKV form in the review of
+ * "Resurrecting Recurrent Neural Networks for Long Sequences"), so
+ *
+ *     y[b,t,c] = wkv[b,t,c] / (1 + e^{-r[b,t,c]})
+ *
+ * with wkv as in wkv_forward_state.  r: [B, T, C] of the I/O type, read in the
+ * same pass as k and v, so the gate costs one extra input stream and no extra
+ * output round trip.  s_in / s_out: as wkv_forward_state (either may be NULL).
+ * r must not overlap y or s_out; other arguments, checks and layout as
+ * wkv_forward_state. */
+WKV_API wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C,
+                                     const float *w, const float *u,
+                                     const float *k, const float *v, const float *r, float *y,
+                                     const float *s_in, float *s_out, cudaStream_t stream);
+
+/* wkv_forward_gated with bfloat16 k/v/r/y (fp32 w, u and fp32 state). */
+WKV_API wkv_status wkv_forward_bf16_gated(int64_t B, int64_t T, int64_t C,
+                                          const float *w, const float *u,
+                                          const wkv_bf16_t *k, const wkv_bf16_t *v,
+                                          const wkv_bf16_t *r, wkv_bf16_t *y,
+                                          const float *s_in, float *s_out, cudaStream_t stream);
+
+/* Token shift, the prologue of the time-mixing block: eqs. (11)-(13) of
+ * "RWKV：基于RNN的LLM" (section 二.1) feed each projection the interpolation
+ *
+ *     out[m, b, t, c] = mu[m, c] * x[b, t, c] + (1 - mu[m, c]) * x[b, t-1, c]
+ *
+ * of every token with the one before it, one mixing vector per projection
+ * (the pages also print eqs. (16)-(17) with a minus sign; the plus of eqs.
+ * (11)-(13) is the reading taken).  All n_mix (1..4) interpolations come from
+ * one read of x.  x[b, -1] is x_prev[b] (the last token of the previous call,
+ * the layer's saved "last_x" in the HarmonyOS RWKV article's time-mixing
+ * code), or 0 when x_prev is NULL; x_last (if not NULL) receives x[b, T-1].
+ * Layout: x [B, T, C]; mu [n_mix, C] float; out [n_mix, B, T, C] (one dense
+ * [B, T, C] tensor per mixing vector); x_prev, x_last [B, C].  x_last may be
+ * the same buffer as x_prev (update in place); out must not overlap any
+ * input, nor x_last.  mu = 1 reproduces x and mu = 0 the shifted x exactly. */
+WKV_API wkv_status wkv_token_shift(int64_t B, int64_t T, int64_t C, int64_t n_mix,
+                                   const float *x, const float *x_prev, const float *mu,
+                                   float *out, float *x_last, cudaStream_t stream);
+
+/* wkv_token_shift on bfloat16 x / x_prev / out / x_last (fp32 mu; computed in
+ * fp32, rounded to nearest even). */
+WKV_API wkv_status wkv_token_shift_bf16(int64_t B, int64_t T, int64_t C, int64_t n_mix,
+                                        const wkv_bf16_t *x, const wkv_bf16_t *x_prev,
+                                        const float *mu, wkv_bf16_t *out, wkv_bf16_t *x_last,
+                                        cudaStream_t stream);
+
 /* Diagonal linear scan, fp32.  a, b, h: [B, T, D] float; h0: [B, D] float or
  * NULL (zero initial state).  Pointers must be 4-byte aligned. */
 WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,

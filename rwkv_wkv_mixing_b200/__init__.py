@@ -10,6 +10,8 @@ raises if the library has not been built.
     y = wkv_forward(w, u, k, v)            # fp32 [B,T,C] k, v; [C] w, u
     y = wkv_forward_bf16(w, u, k, v)       # bf16 k, v -> bf16 y, fp32 state
     y, s = wkv_forward_state(w, u, k, v, s_in)   # + state [B,3,C] in and out
+    y = wkv_forward_gated(w, u, k, v, r)   # sigma(r) * wkv, one pass
+    out = token_shift(x, mu, x_prev)       # [n_mix,B,T,C] mu x_t + (1-mu) x_{t-1}
     h = diag_scan(a, b, h0=None)           # fp32 [B,T,D]; h0 [B,D] or None
     y = wkv_forward_host(w, u, k, v)       # the same on CPU tensors, copies overlapped
 """
@@ -42,6 +44,10 @@ _SIGS = {
     "wkv_forward_noalloc": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_state": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_bf16_state": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_gated": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_forward_bf16_gated": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_token_shift": ([_i64, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_token_shift_bf16": ([_i64, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "diag_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_bf16_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
@@ -171,6 +177,78 @@ def wkv_forward_bf16_state(w, u, k, v, s_in=None, y=None, s_out=None, stream=Non
     import torch
     return _wkv_state("wkv_forward_bf16_state", torch.bfloat16, w, u, k, v, s_in, y, s_out,
                       stream)
+
+
+def wkv_forward_gated(w, u, k, v, r, y=None, s_in=None, s_out=None, stream=None):
+    """sigma(r) (.) wkv in one pass (eq. (15) before the output projection);
+    k, v, r, y fp32 or all bf16 (then the bf16 entry point runs).  Optional
+    state [B, 3, C] fp32 in (``s_in``) and out (``s_out``, may be s_in)."""
+    import torch
+    io = k.dtype
+    if io not in (torch.float32, torch.bfloat16):
+        raise TypeError("k must be float32 or bfloat16")
+    _need(k, "k", io, 3)
+    _need(v, "v", io, 3)
+    _need(r, "r", io, 3)
+    _need(w, "w", torch.float32, 1)
+    _need(u, "u", torch.float32, 1)
+    if k.shape != v.shape or k.shape != r.shape:
+        raise ValueError("k, v and r must have one shape")
+    B, T, C = k.shape
+    if w.shape[0] != C or u.shape[0] != C:
+        raise ValueError("w and u must be [C]")
+    for t, name in ((s_in, "s_in"), (s_out, "s_out")):
+        if t is not None:
+            _need(t, name, torch.float32, 3)
+            if tuple(t.shape) != (B, 3, C):
+                raise ValueError(f"{name} must be [B, 3, C] = {(B, 3, C)}")
+    if y is None:
+        y = torch.empty_like(k)
+    else:
+        _need(y, "y", io, 3)
+        if y.shape != k.shape:
+            raise ValueError("y must have the shape of k")
+    fn = "wkv_forward_gated" if io == torch.float32 else "wkv_forward_bf16_gated"
+    _check(getattr(lib, fn)(B, T, C, w.data_ptr(), u.data_ptr(), k.data_ptr(), v.data_ptr(),
+                            r.data_ptr(), y.data_ptr(),
+                            None if s_in is None else s_in.data_ptr(),
+                            None if s_out is None else s_out.data_ptr(),
+                            _stream_handle(stream)), fn)
+    return y
+
+
+def token_shift(x, mu, x_prev=None, out=None, x_last=None, stream=None):
+    """mu[m] x_t + (1 - mu[m]) x_{t-1} for every row m of ``mu`` ([n_mix, C]
+    fp32) from one read of x ([B, T, C] fp32 or bf16); x_{-1} = x_prev [B, C]
+    (zeros if None).  Returns out [n_mix, B, T, C]; ``x_last`` [B, C], if
+    given, receives x[:, T-1] (it may be x_prev)."""
+    import torch
+    io = x.dtype
+    if io not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", io, 3)
+    B, T, C = x.shape
+    _need(mu, "mu", torch.float32, 2)
+    if mu.shape[1] != C or not 1 <= mu.shape[0] <= 4:
+        raise ValueError("mu must be [n_mix, C] with 1 <= n_mix <= 4")
+    n_mix = mu.shape[0]
+    for t, name in ((x_prev, "x_prev"), (x_last, "x_last")):
+        if t is not None:
+            _need(t, name, io, 2)
+            if tuple(t.shape) != (B, C):
+                raise ValueError(f"{name} must be [B, C] = {(B, C)}")
+    if out is None:
+        out = torch.empty((n_mix, B, T, C), dtype=io, device=x.device)
+    else:
+        _need(out, "out", io, 4)
+        if tuple(out.shape) != (n_mix, B, T, C):
+            raise ValueError("out must be [n_mix, B, T, C]")
+    fn = "wkv_token_shift" if io == torch.float32 else "wkv_token_shift_bf16"
+    _check(getattr(lib, fn)(B, T, C, n_mix, x.data_ptr(),
+                            None if x_prev is None else x_prev.data_ptr(), mu.data_ptr(),
+                            out.data_ptr(), None if x_last is None else x_last.data_ptr(),
+                            _stream_handle(stream)), fn)
+    return out
 
 
 def wkv_forward_noalloc(w, u, k, v, y=None, stream=None):
@@ -308,7 +386,7 @@ def wkv_set_fault_injection(skip_tile: int = -1, spin_limit: int = 0):
 
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan",
-           "wkv_forward_state", "wkv_forward_bf16_state",
+           "wkv_forward_state", "wkv_forward_bf16_state", "wkv_forward_gated", "token_shift",
            "wkv_forward_host", "wkv_forward_bf16_host", "diag_scan_host", "wkv_device_status",
            "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
            "wkv_get_tile_steps", "WkvError", "lib", "LIB_PATH"]

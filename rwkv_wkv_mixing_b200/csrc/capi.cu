@@ -18,6 +18,7 @@
 #include "chunked_scan.cuh"
 #include "persistent_scan.cuh"
 #include "serial_wkv.cuh"
+#include "token_shift.cuh"
 #include "wkv_b200.h"
 #include "wkv_ops.cuh"
 
@@ -254,7 +255,7 @@ int sm_count(int dev) {
 // look-back workspace of one call; `cg` channels and `lt` steps per tile.
 struct Plan {
     Geometry g;
-    CUtensorMap maps[3];
+    CUtensorMap maps[4];  // x0, x1, y, and x2 for three-input ops
     Workspace ws;
 };
 
@@ -280,9 +281,11 @@ wkv_status make_plan(const typename Op::Args &args, int64_t B, int64_t T, int64_
     std::memset(p->maps, 0, sizeof p->maps);
     g.use_tma = 0;
     if (want_tma) {
-        const void *ptrs[3] = {args.x0, args.x1, args.y};
-        g.use_tma = tma_eligible(ptrs, 3, sizeof(io_t), T, C) ? 1 : 0;
-        for (int i = 0; i < 3 && g.use_tma; ++i)
+        const void *ptrs[4] = {args.x0, args.x1, args.y, nullptr};
+        int n = 3;
+        if constexpr (Op::NIN == 3) ptrs[n++] = args.x2;
+        g.use_tma = tma_eligible(ptrs, n, sizeof(io_t), T, C) ? 1 : 0;
+        for (int i = 0; i < n && g.use_tma; ++i)
             if (!make_map(&p->maps[i], ptrs[i], dt, sizeof(io_t), B, T, C, CG, lt)) g.use_tma = 0;
     }
     std::memset(&p->ws, 0, sizeof p->ws);
@@ -326,8 +329,8 @@ wkv_status launch_chunked(const typename Op::Args &args, int64_t B, int64_t T, i
     static std::atomic<uint64_t> configured{0};
     if ((st = configure_once(kern, smem, dev, configured)) != WKV_OK) return st;
     cudaGetLastError();  // clear a stale error so the check below is about this launch
-    kern<<<static_cast<unsigned>(p.g.tiles), NW * 32, smem, stream>>>(p.maps[0], p.maps[1],
-                                                                       p.maps[2], args, p.g, p.ws);
+    kern<<<static_cast<unsigned>(p.g.tiles), NW * 32, smem, stream>>>(
+        p.maps[0], p.maps[1], p.maps[2], p.maps[3], args, p.g, p.ws);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     return WKV_OK;
@@ -363,7 +366,7 @@ wkv_status launch_persistent(const typename Op::Args &args, int64_t B, int64_t T
     cfg.numAttrs = 1;
     cudaGetLastError();
     cudaError_t err =
-        cudaLaunchKernelEx(&cfg, kern, p.maps[0], p.maps[1], p.maps[2], args, p.g, p.ws);
+        cudaLaunchKernelEx(&cfg, kern, p.maps[0], p.maps[1], p.maps[2], p.maps[3], args, p.g, p.ws);
     if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     return WKV_OK;
@@ -382,7 +385,7 @@ wkv_status launch_serial(const typename Op::Args &args, int64_t B, int64_t T, in
         return p == nullptr || reinterpret_cast<uintptr_t>(p) % a == 0;
     };
     const bool vec4 = C % 4 == 0 && al(args.x0, vb) && al(args.x1, vb) && al(args.y, vb) &&
-                      al(args.s_in, 16) && al(args.s_out, 16);
+                      al(args.x2, vb) && al(args.s_in, 16) && al(args.s_out, 16);
     const int vw = vec4 ? 4 : 1;
     const int64_t blocks = (B * (C / vw) + kSerialThreads - 1) / kSerialThreads;
     if (vec4)
@@ -403,20 +406,39 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
         if (T <= kSerialMaxSteps && (B * C + kSerialThreads - 1) / kSerialThreads <= INT32_MAX)
             return launch_serial<Op>(args, B, T, C, stream);
     }
-    const void *ptrs[3] = {args.x0, args.x1, args.y};
-    const bool tma = tma_eligible(ptrs, 3, sizeof(typename Op::io_t), T, C);
-    switch (g_tile_steps.load()) {
-        case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
-        case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
-        case 64:
-            return tma ? launch_persistent<Op, 64, 4, 6, 12>(args, B, T, C, dt, stream, dev)
-                       : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
-        case 256:
-            return tma ? launch_persistent<Op, 256, 8, 2, 3>(args, B, T, C, dt, stream, dev)
-                       : launch_chunked<Op, 256, 8>(args, B, T, C, dt, stream, dev);
-        default:
-            return tma ? launch_persistent<Op, 128, 4, 4, 6>(args, B, T, C, dt, stream, dev)
-                       : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
+    const void *ptrs[4] = {args.x0, args.x1, args.y, nullptr};
+    int nptr = 3;
+    if constexpr (Op::NIN == 3) ptrs[nptr++] = args.x2;
+    const bool tma = tma_eligible(ptrs, nptr, sizeof(typename Op::io_t), T, C);
+    if constexpr (Op::NIN == 3) {
+        // a third input tile per stage: fewer stages and groups fit in shared memory
+        switch (g_tile_steps.load()) {
+            case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
+            case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
+            case 64:
+                return tma ? launch_persistent<Op, 64, 4, 4, 6>(args, B, T, C, dt, stream, dev)
+                           : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
+            case 256:
+                return tma ? launch_persistent<Op, 256, 8, 1, 2>(args, B, T, C, dt, stream, dev)
+                           : launch_chunked<Op, 256, 8>(args, B, T, C, dt, stream, dev);
+            default:
+                return tma ? launch_persistent<Op, 128, 4, 3, 4>(args, B, T, C, dt, stream, dev)
+                           : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
+        }
+    } else {
+        switch (g_tile_steps.load()) {
+            case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
+            case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
+            case 64:
+                return tma ? launch_persistent<Op, 64, 4, 6, 12>(args, B, T, C, dt, stream, dev)
+                           : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
+            case 256:
+                return tma ? launch_persistent<Op, 256, 8, 2, 3>(args, B, T, C, dt, stream, dev)
+                           : launch_chunked<Op, 256, 8>(args, B, T, C, dt, stream, dev);
+            default:
+                return tma ? launch_persistent<Op, 128, 4, 4, 6>(args, B, T, C, dt, stream, dev)
+                           : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
+        }
     }
 }
 
@@ -426,10 +448,10 @@ wkv_status current_device(int *dev) {
     return WKV_OK;
 }
 
-template <typename IO>
+template <typename IO, bool GATED = false>
 wkv_status wkv_common(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
                       const IO *k, const IO *v, IO *y, const float *s_in, float *s_out,
-                      cudaStream_t stream, CUtensorMapDataType dt) {
+                      cudaStream_t stream, CUtensorMapDataType dt, const IO *r = nullptr) {
     t_err.clear();
     bool empty = false;
     wkv_status st = check_sizes(B, T, C, &empty);
@@ -446,20 +468,90 @@ wkv_status wkv_common(int64_t B, int64_t T, int64_t C, const float *w, const flo
     if (overlaps(y, n, k, n) || overlaps(y, n, v, n) || overlaps(y, n, w, nc) ||
         overlaps(y, n, u, nc))
         return fail(WKV_ERR_INVALID_ARG, "y overlaps an input");
+    if (GATED) {
+        if ((st = check_buffer(r, n, sizeof(IO), "r", dev)) != WKV_OK) return st;
+        if (overlaps(y, n, r, n)) return fail(WKV_ERR_INVALID_ARG, "y overlaps r");
+    }
     const size_t ns = static_cast<size_t>(B) * 3 * C * sizeof(float);
     if (s_in != nullptr && (st = check_buffer(s_in, ns, 4, "s_in", dev)) != WKV_OK) return st;
     if (s_out != nullptr) {
         if ((st = check_buffer(s_out, ns, 4, "s_out", dev)) != WKV_OK) return st;
         if (overlaps(s_out, ns, k, n) || overlaps(s_out, ns, v, n) || overlaps(s_out, ns, y, n) ||
-            overlaps(s_out, ns, w, nc) || overlaps(s_out, ns, u, nc))
-            return fail(WKV_ERR_INVALID_ARG, "s_out overlaps k, v, y, w or u");
+            overlaps(s_out, ns, w, nc) || overlaps(s_out, ns, u, nc) ||
+            overlaps(s_out, ns, r, GATED ? n : 0))
+            return fail(WKV_ERR_INVALID_ARG, "s_out overlaps k, v, r, y, w or u");
         if (s_in != nullptr && s_in != s_out && overlaps(s_out, ns, s_in, ns))
             return fail(WKV_ERR_INVALID_ARG, "s_out overlaps s_in without being the same buffer");
     }
     if (overlaps(y, n, s_in, s_in ? ns : 0))
         return fail(WKV_ERR_INVALID_ARG, "y overlaps s_in");
-    typename WkvOp<IO, sizeof(IO) == 2 ? 2 : 1>::Args args{k, v, y, w, u, s_in, s_out};
-    return dispatch<WkvOp<IO, sizeof(IO) == 2 ? 2 : 1>>(args, B, T, C, dt, stream, dev);
+    using Op = WkvOp<IO, sizeof(IO) == 2 ? 2 : 1, GATED>;
+    typename Op::Args args{k, v, y, w, u, s_in, s_out, GATED ? r : nullptr};
+    return dispatch<Op>(args, B, T, C, dt, stream, dev);
+}
+
+// ---- token shift ----------------------------------------------------------------
+template <typename IO, int VW>
+wkv_status launch_shift(int n_mix, const IO *x, const IO *x_prev, const float *mu, IO *out,
+                        IO *x_last, int64_t B, int64_t T, int64_t C, cudaStream_t stream) {
+    const int64_t chunks = (T + kShiftChunk - 1) / kShiftChunk;
+    const int64_t threads = B * chunks * (C / VW);
+    const int64_t blocks = (threads + kShiftThreads - 1) / kShiftThreads;
+    if (blocks > INT32_MAX) return fail(WKV_ERR_INVALID_ARG, "problem too large for one launch");
+    const dim3 grid(static_cast<unsigned>(blocks));
+    const int b = static_cast<int>(B), t = static_cast<int>(T), c = static_cast<int>(C);
+    switch (n_mix) {
+        case 1: token_shift_kernel<IO, VW, 1><<<grid, kShiftThreads, 0, stream>>>(x, x_prev, mu, out, x_last, b, t, c); break;
+        case 2: token_shift_kernel<IO, VW, 2><<<grid, kShiftThreads, 0, stream>>>(x, x_prev, mu, out, x_last, b, t, c); break;
+        case 3: token_shift_kernel<IO, VW, 3><<<grid, kShiftThreads, 0, stream>>>(x, x_prev, mu, out, x_last, b, t, c); break;
+        default: token_shift_kernel<IO, VW, 4><<<grid, kShiftThreads, 0, stream>>>(x, x_prev, mu, out, x_last, b, t, c); break;
+    }
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
+template <typename IO>
+wkv_status shift_common(int64_t B, int64_t T, int64_t C, int64_t n_mix, const IO *x,
+                        const IO *x_prev, const float *mu, IO *out, IO *x_last,
+                        cudaStream_t stream) {
+    t_err.clear();
+    if (n_mix < 1 || n_mix > 4) return fail(WKV_ERR_INVALID_ARG, "n_mix must be 1..4");
+    bool empty = false;
+    wkv_status st = check_sizes(B, T, C, &empty);
+    if (st != WKV_OK || empty) return st;
+    int dev = 0;
+    if ((st = current_device(&dev)) != WKV_OK) return st;
+    const size_t n = static_cast<size_t>(B) * T * C * sizeof(IO);
+    const size_t nrow = static_cast<size_t>(B) * C * sizeof(IO);
+    const size_t nmu = static_cast<size_t>(n_mix) * C * sizeof(float);
+    const size_t nout = static_cast<size_t>(n_mix) * n;
+    if ((st = check_buffer(x, n, sizeof(IO), "x", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(mu, nmu, 4, "mu", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(out, nout, sizeof(IO), "out", dev)) != WKV_OK) return st;
+    if (x_prev != nullptr && (st = check_buffer(x_prev, nrow, sizeof(IO), "x_prev", dev)) != WKV_OK)
+        return st;
+    if (x_last != nullptr && (st = check_buffer(x_last, nrow, sizeof(IO), "x_last", dev)) != WKV_OK)
+        return st;
+    if (overlaps(out, nout, x, n) || overlaps(out, nout, mu, nmu) ||
+        overlaps(out, nout, x_prev, x_prev ? nrow : 0) ||
+        overlaps(out, nout, x_last, x_last ? nrow : 0))
+        return fail(WKV_ERR_INVALID_ARG, "out overlaps x, mu, x_prev or x_last");
+    if (x_last != nullptr) {
+        if (overlaps(x_last, nrow, x, n) || overlaps(x_last, nrow, mu, nmu))
+            return fail(WKV_ERR_INVALID_ARG, "x_last overlaps x or mu");
+        if (x_prev != nullptr && x_prev != x_last && overlaps(x_last, nrow, x_prev, nrow))
+            return fail(WKV_ERR_INVALID_ARG, "x_last overlaps x_prev without being the same buffer");
+    }
+    const auto al = [](const void *p, size_t a) {
+        return p == nullptr || reinterpret_cast<uintptr_t>(p) % a == 0;
+    };
+    const size_t vb = 4 * sizeof(IO);
+    const bool vec4 = C % 4 == 0 && al(x, vb) && al(x_prev, vb) && al(out, vb) &&
+                      al(x_last, vb) && al(mu, 16);
+    const int nm = static_cast<int>(n_mix);
+    return vec4 ? launch_shift<IO, 4>(nm, x, x_prev, mu, out, x_last, B, T, C, stream)
+                : launch_shift<IO, 1>(nm, x, x_prev, mu, out, x_last, B, T, C, stream);
 }
 
 // ---- host-buffer entry points: a chunked copy / compute pipeline ------------
@@ -752,6 +844,38 @@ wkv_status wkv_forward_bf16_state(int64_t B, int64_t T, int64_t C, const float *
                                      reinterpret_cast<const __nv_bfloat16 *>(v),
                                      reinterpret_cast<__nv_bfloat16 *>(y), s_in, s_out, stream,
                                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                             const float *k, const float *v, const float *r, float *y,
+                             const float *s_in, float *s_out, cudaStream_t stream) {
+    return wkv_common<float, true>(B, T, C, w, u, k, v, y, s_in, s_out, stream,
+                                   CU_TENSOR_MAP_DATA_TYPE_FLOAT32, r);
+}
+
+wkv_status wkv_forward_bf16_gated(int64_t B, int64_t T, int64_t C, const float *w,
+                                  const float *u, const wkv_bf16_t *k, const wkv_bf16_t *v,
+                                  const wkv_bf16_t *r, wkv_bf16_t *y, const float *s_in,
+                                  float *s_out, cudaStream_t stream) {
+    return wkv_common<__nv_bfloat16, true>(
+        B, T, C, w, u, reinterpret_cast<const __nv_bfloat16 *>(k),
+        reinterpret_cast<const __nv_bfloat16 *>(v), reinterpret_cast<__nv_bfloat16 *>(y), s_in,
+        s_out, stream, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, reinterpret_cast<const __nv_bfloat16 *>(r));
+}
+
+wkv_status wkv_token_shift(int64_t B, int64_t T, int64_t C, int64_t n_mix, const float *x,
+                           const float *x_prev, const float *mu, float *out, float *x_last,
+                           cudaStream_t stream) {
+    return shift_common<float>(B, T, C, n_mix, x, x_prev, mu, out, x_last, stream);
+}
+
+wkv_status wkv_token_shift_bf16(int64_t B, int64_t T, int64_t C, int64_t n_mix,
+                                const wkv_bf16_t *x, const wkv_bf16_t *x_prev, const float *mu,
+                                wkv_bf16_t *out, wkv_bf16_t *x_last, cudaStream_t stream) {
+    using bf = __nv_bfloat16;
+    return shift_common<bf>(B, T, C, n_mix, reinterpret_cast<const bf *>(x),
+                            reinterpret_cast<const bf *>(x_prev), mu, reinterpret_cast<bf *>(out),
+                            reinterpret_cast<bf *>(x_last), stream);
 }
 
 wkv_status diag_scan(int64_t B, int64_t T, int64_t D, const float *a, const float *b,

@@ -39,7 +39,7 @@ namespace wkvb {
 
 template <class Op, int LT, int NW>
 constexpr size_t chunked_scan_smem_bytes() {
-    return 2ull * LT * 32 * Op::CPT * sizeof(typename Op::io_t) +
+    return static_cast<size_t>(Op::NIN) * LT * 32 * Op::CPT * sizeof(typename Op::io_t) +
            static_cast<size_t>(NW + 1) * Op::NV * 32 * Op::CPT * sizeof(float);
 }
 
@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(NW * 32, 3)
     chunked_scan_kernel(const __grid_constant__ CUtensorMap map_x0,
                         const __grid_constant__ CUtensorMap map_x1,
                         const __grid_constant__ CUtensorMap map_y,
+                        const __grid_constant__ CUtensorMap map_x2,  // NIN == 3 only
                         const typename Op::Args args, const Geometry g, const Workspace ws) {
     using io_t = typename Op::io_t;
     using State = typename Op::State;
@@ -59,7 +60,8 @@ __global__ void __launch_bounds__(NW * 32, 3)
     extern __shared__ __align__(128) unsigned char smem[];
     io_t *s_x0 = reinterpret_cast<io_t *>(smem);            // [LT][CG], outputs overwrite it
     io_t *s_x1 = s_x0 + LT * CG;                            // [LT][CG]
-    float *s_sum = reinterpret_cast<float *>(s_x1 + LT * CG);  // [NW][NV][CG]
+    io_t *s_x2 = s_x1 + (Op::NIN == 3 ? LT * CG : 0);       // [LT][CG] r, when NIN == 3
+    float *s_sum = reinterpret_cast<float *>(s_x0 + Op::NIN * LT * CG);  // [NW][NV][CG]
     float *s_carry = s_sum + NW * NV * CG;                   // [NV][CG]
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_tile;
@@ -105,22 +107,26 @@ __global__ void __launch_bounds__(NW * 32, 3)
     // ---- stage the tile ---------------------------------------------------
     if (g.use_tma) {
         if (tid == 0) {
-            mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(2 * LT * CG * sizeof(io_t)));
+            mbar_arrive_expect_tx(&s_bar,
+                                  static_cast<uint32_t>(Op::NIN * LT * CG * sizeof(io_t)));
             tma_load_3d(s_x0, &map_x0, &s_bar, c0, t0, b);
             tma_load_3d(s_x1, &map_x1, &s_bar, c0, t0, b);
+            if constexpr (Op::NIN == 3) tma_load_3d(s_x2, &map_x2, &s_bar, c0, t0, b);
         }
     } else {
         for (int i = tid; i < LT * CG; i += NW * 32) {
             const int tl = i / CG, cl = i - (i / CG) * CG;
             const int t = t0 + tl, c = c0 + cl;
-            io_t a = io_zero<io_t>(), bb = io_zero<io_t>();
+            io_t a = io_zero<io_t>(), bb = io_zero<io_t>(), rr = io_zero<io_t>();
             if (t < g.T && c < g.C) {
                 const size_t o = (static_cast<size_t>(b) * g.T + t) * g.C + c;
                 a = args.x0[o];
                 bb = args.x1[o];
+                if constexpr (Op::NIN == 3) rr = args.x2[o];
             }
             s_x0[i] = a;
             s_x1[i] = bb;
+            if constexpr (Op::NIN == 3) s_x2[i] = rr;
         }
     }
     Param prm[CPT];
@@ -236,7 +242,8 @@ __global__ void __launch_bounds__(NW * 32, 3)
                 cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(warp * LS), prm[j]);
             }
         }
-        Op::template sweep<LS>(cur, p0, p1, nval, prm, sc, p0, CG, true);
+        Op::template sweep<LS>(cur, p0, p1, s_x2 + s0 * CG + lane * CPT, nval, prm, sc, p0, CG,
+                               true);
     }
 
     // ---- write the output tile ----------------------------------------------

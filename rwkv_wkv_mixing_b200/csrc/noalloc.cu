@@ -219,7 +219,7 @@ extern "C" wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const
         ws.records = reinterpret_cast<uint4 *>(base + kHeader);
     }
 
-    CUtensorMap maps[3];
+    CUtensorMap maps[4];  // k, v, y; the fourth (a gate input) is unused here
     std::memset(maps, 0, sizeof maps);
     const bool tma = reinterpret_cast<uintptr_t>(k) % 16 == 0 &&
                      reinterpret_cast<uintptr_t>(v) % 16 == 0 &&
@@ -237,13 +237,13 @@ extern "C" wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const
     if (tma) {
         const int grid = g.tiles < sms ? g.tiles : sms;
         persistent_scan_kernel<Op, kTileSteps, 4, 4, 6>
-            <<<grid, Persistent::kThreads, Persistent::kSmemBytes, stream>>>(maps[0], maps[1],
-                                                                              maps[2], args, g, ws);
+            <<<grid, Persistent::kThreads, Persistent::kSmemBytes, stream>>>(
+                maps[0], maps[1], maps[2], maps[3], args, g, ws);
     } else {
         chunked_scan_kernel<Op, kTileSteps, kChunkedWarps>
             <<<static_cast<unsigned>(g.tiles), kChunkedWarps * 32,
                chunked_scan_smem_bytes<Op, kTileSteps, kChunkedWarps>(), stream>>>(
-                maps[0], maps[1], maps[2], args, g, ws);
+                maps[0], maps[1], maps[2], maps[3], args, g, ws);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");

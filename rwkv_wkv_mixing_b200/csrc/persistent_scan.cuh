@@ -2,7 +2,7 @@
 // map can describe).
 //
 // One thread block per SM stays resident for the whole launch.  Warp 0 is the
-// producer: one lane takes tile tickets and streams each tile's two input
+// producer: one lane takes tile tickets and streams each tile's NIN input
 // tensors (LT steps x CG channels) into a ring of NSTAGE shared-memory stages
 // with TMA tile loads, each stage guarded by a "full" and an "empty" mbarrier.
 // The remaining warps form NC consumer groups of NWG warps; group g handles
@@ -38,7 +38,7 @@ struct PersistentCfg {
     static constexpr int CPT = Op::CPT, NV = Op::NV, CG = 32 * CPT, LS = LT / NWG;
     static constexpr int kThreads = (1 + NC * NWG) * 32;
     static constexpr size_t kTileElems = static_cast<size_t>(LT) * CG;
-    static constexpr size_t kStageBytes = 2 * kTileElems * sizeof(typename Op::io_t);
+    static constexpr size_t kStageBytes = Op::NIN * kTileElems * sizeof(typename Op::io_t);
     static constexpr size_t kSmemBytes =
         NSTAGE * kStageBytes + static_cast<size_t>(NC) * (NWG + 1) * NV * CG * sizeof(float);
     static_assert(LT % NWG == 0, "tile length must split evenly over a group's warps");
@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
     persistent_scan_kernel(const __grid_constant__ CUtensorMap map_x0,
                            const __grid_constant__ CUtensorMap map_x1,
                            const __grid_constant__ CUtensorMap map_y,
+                           const __grid_constant__ CUtensorMap map_x2,  // NIN == 3 only
                            const typename Op::Args args, const Geometry g, const Workspace ws) {
     using Cfg = PersistentCfg<Op, LT, NWG, NC, NSTAGE>;
     using io_t = typename Op::io_t;
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
     constexpr int CPT = Cfg::CPT, NV = Cfg::NV, CG = Cfg::CG, LS = Cfg::LS;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    io_t *s_stage = reinterpret_cast<io_t *>(smem);  // [NSTAGE][2][LT][CG]
+    io_t *s_stage = reinterpret_cast<io_t *>(smem);  // [NSTAGE][NIN][LT][CG]
     float *s_sum = reinterpret_cast<float *>(smem + NSTAGE * Cfg::kStageBytes);  // [NC][NWG][NV][CG]
     float *s_carry = s_sum + NC * NWG * NV * CG;                                   // [NC][NV][CG]
     __shared__ __align__(8) uint64_t full_bar[NSTAGE];
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             prefetch_tensormap(&map_x0);
             prefetch_tensormap(&map_x1);
             prefetch_tensormap(&map_y);
+            if constexpr (Op::NIN == 3) prefetch_tensormap(&map_x2);
             int sentinels = 0;
             int next_static = static_cast<int>(blockIdx.x);
             for (int it = 0; sentinels < NC; ++it) {
@@ -173,11 +175,14 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                     const int rem = tile - seg * g.tiles_per_seg;
                     const int b = rem / g.n_cg;
                     const int c0 = (rem - b * g.n_cg) * CG;
-                    io_t *dst = s_stage + static_cast<size_t>(s) * 2 * Cfg::kTileElems;
+                    io_t *dst = s_stage + static_cast<size_t>(s) * Op::NIN * Cfg::kTileElems;
                     s_last_it[s] = it;
                     mbar_arrive_expect_tx(&full_bar[s], static_cast<uint32_t>(Cfg::kStageBytes));
                     tma_load_3d(dst, &map_x0, &full_bar[s], c0, seg * LT, b);
                     tma_load_3d(dst + Cfg::kTileElems, &map_x1, &full_bar[s], c0, seg * LT, b);
+                    if constexpr (Op::NIN == 3)
+                        tma_load_3d(dst + 2 * Cfg::kTileElems, &map_x2, &full_bar[s], c0,
+                                    seg * LT, b);
                 }
             }
         }
@@ -212,8 +217,10 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             const int b = rem / g.n_cg;
             const int t0 = seg * LT;
             const int c0 = (rem - b * g.n_cg) * CG;
-            io_t *s_x0 = s_stage + static_cast<size_t>(s) * 2 * Cfg::kTileElems;
+            io_t *s_x0 = s_stage + static_cast<size_t>(s) * Op::NIN * Cfg::kTileElems;
             const io_t *s_x1 = s_x0 + Cfg::kTileElems;
+            // the third input (r) when there is one; never read otherwise
+            const io_t *s_x2 = Op::NIN == 3 ? s_x1 + Cfg::kTileElems : s_x1;
 
             Param prm[CPT];
 #pragma unroll
@@ -316,7 +323,8 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                         cur[j] = Op::combine(cur[j], Op::make(vals), static_cast<float>(wg * LS), prm[j]);
                     }
                 }
-                Op::template sweep<LS>(cur, p0, p1, nval, prm, sc, p0, CG, true);
+                Op::template sweep<LS>(cur, p0, p1, s_x2 + s0 * CG + lane * CPT, nval, prm, sc,
+                                       p0, CG, true);
             }
             fence_proxy_async_smem();
             named_bar_sync(bar_id, NWG * 32);

@@ -7,9 +7,10 @@
 //
 // With a handful of steps there is nothing to parallelise over time: the
 // chunked kernels' tiles, look-back and workspace would only add latency.
-// The work is a pure stream -- per channel and step 2 loads and 1 store,
-// plus 3 state words in and out -- so the kernel is built for bytes in
-// flight: VW = 4 channels per thread turns every access into one 16-byte
+// The work is a pure stream -- per channel and step 2 loads (3 with the
+// receptance gate) and 1 store, plus 3 state words in and out -- so the
+// kernel is built for bytes in flight: VW = 4 channels per thread turns every
+// access into one 16-byte
 // (fp32) or 8-byte (bf16) vector access, and consecutive threads own
 // consecutive channel groups, so each warp access is one contiguous run.
 // The per-step update is the max-stabilised one the chunked kernels use for
@@ -62,6 +63,12 @@ __global__ void __launch_bounds__(kSerialThreads)
         Vec<IO, VW>::load(args.x1 + o, v);
 #pragma unroll
         for (int j = 0; j < VW; ++j) y[j] = Op::step_exact(s[j], k[j], v[j], q[j]);
+        if constexpr (Op::kGated) {  // sigma(r) (.) wkv
+            float r[VW];
+            Vec<IO, VW>::load(args.x2 + o, r);
+#pragma unroll
+            for (int j = 0; j < VW; ++j) y[j] *= gate_sigmoid(r[j]);
+        }
         Vec<IO, VW>::store(args.y + o, y);
     }
 

@@ -111,6 +111,13 @@ __device__ __forceinline__ float wkv_output(float a, float b, float e, float v) 
     return v + fmaf(-b, v, a) * rcp_approx(b + e);
 }
 
+// The receptance gate sigma(r) = 1 / (1 + e^{-r}) of eq. (15) of
+// "RWKV：基于RNN的LLM".  Saturates cleanly: e^{-r} = inf gives 0, e^{-r} = 0
+// gives 1.
+__device__ __forceinline__ float gate_sigmoid(float r) {
+    return rcp_approx(1.f + ex2_approx(-r * kLog2e));
+}
+
 // ---------------------------------------------------------------------------
 // WKV, eq. (14) of "RWKV：基于RNN的LLM" (section 二.1, Time-mixing block):
 //   y_t = (num_t + e^{u + k_t} v_t) / (den_t + e^{u + k_t}),
@@ -133,12 +140,16 @@ __device__ __forceinline__ float wkv_output(float a, float b, float e, float v) 
 // 2^64.  Otherwise the sub-chunk takes the per-step max-stabilised update,
 // whose every exponent is <= 0 for any finite input.
 // ---------------------------------------------------------------------------
-template <typename IO, int CPT_>
+// GATED: the outputs are sigma(r_t) (.) wkv_t (eq. (15) before the output
+// projection), r read as a third input tensor alongside k and v.
+template <typename IO, int CPT_, bool GATED = false>
 struct WkvOp {
     using io_t = IO;
     static constexpr int CPT = CPT_;
     static constexpr int CG = 32 * CPT;
     static constexpr int NV = 3;
+    static constexpr int NIN = GATED ? 3 : 2;  // input tensors per tile: k, v (, r)
+    static constexpr bool kGated = GATED;
     static constexpr bool kSerialForm = true;  // has the per-step form of serial_wkv.cuh
     struct Param {
         float u, w;  // bonus and decay (natural units)
@@ -154,6 +165,7 @@ struct WkvOp {
         const float *w, *u;  // [C]
         const float *s_in;   // [B, 3, C] state before step 0, or nullptr (empty)
         float *s_out;        // [B, 3, C] state after the last step, or nullptr
+        const IO *x2;        // r [B, T, C] (GATED only)
     };
     // per-thread facts pass 1 leaves for pass 2 of the same sub-chunk
     struct Scratch {
@@ -334,11 +346,12 @@ struct WkvOp {
 
     // outputs go to out[i * ostride] (shared or global memory); when `valid`
     // is false this thread's channels are past C and nothing is stored
+    // (p2: the r rows when GATED, else unused)
     template <int LS>
     __device__ __forceinline__ static void sweep(const State (&carry)[CPT], const IO *p0,
-                                                 const IO *p1, int n, const Param (&q)[CPT],
-                                                 const Scratch (&sc)[CPT], IO *out, size_t ostride,
-                                                 bool valid) {
+                                                 const IO *p1, const IO *p2, int n,
+                                                 const Param (&q)[CPT], const Scratch (&sc)[CPT],
+                                                 IO *out, size_t ostride, bool valid) {
         // reference per channel, and whether the fixed-reference form is safe
         float M[CPT], M2[CPT], A[CPT], Bs[CPT];
         bool fast = true;
@@ -359,10 +372,12 @@ struct WkvOp {
             if (n == LS) {
 #pragma unroll 8
                 for (int i = 0; i < LS; ++i)
-                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, M2, A, Bs, q);
+                    fast_step(p0 + i * CG, p1 + i * CG, p2 + i * CG, out + i * ostride, valid, M,
+                              M2, A, Bs, q);
             } else {
                 for (int i = 0; i < n; ++i)
-                    fast_step(p0 + i * CG, p1 + i * CG, out + i * ostride, valid, M, M2, A, Bs, q);
+                    fast_step(p0 + i * CG, p1 + i * CG, p2 + i * CG, out + i * ostride, valid, M,
+                              M2, A, Bs, q);
             }
         } else {
             State s[CPT];
@@ -374,15 +389,24 @@ struct WkvOp {
                 Vec<IO, CPT>::load(p1 + i * CG, v);
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) y[j] = step_exact(s[j], k[j], v[j], q[j]);
+                if constexpr (GATED) apply_gate(p2 + i * CG, y);
                 if (valid) Vec<IO, CPT>::store(out + i * ostride, y);
             }
         }
     }
 
-    __device__ __forceinline__ static void fast_step(const IO *pk, const IO *pv, IO *py, bool valid,
-                                                     const float (&M)[CPT], const float (&M2)[CPT],
-                                                     float (&A)[CPT], float (&Bs)[CPT],
-                                                     const Param (&q)[CPT]) {
+    // y <- sigma(r) (.) y for this thread's channels, r read at pr
+    __device__ __forceinline__ static void apply_gate(const IO *pr, float (&y)[CPT]) {
+        float r[CPT];
+        Vec<IO, CPT>::load(pr, r);
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) y[j] *= gate_sigmoid(r[j]);
+    }
+
+    __device__ __forceinline__ static void fast_step(const IO *pk, const IO *pv, const IO *pr,
+                                                     IO *py, bool valid, const float (&M)[CPT],
+                                                     const float (&M2)[CPT], float (&A)[CPT],
+                                                     float (&Bs)[CPT], const Param (&q)[CPT]) {
         float k[CPT], v[CPT], y[CPT];
         Vec<IO, CPT>::load(pk, k);
         Vec<IO, CPT>::load(pv, v);
@@ -394,6 +418,7 @@ struct WkvOp {
             A[j] = fmaf(A[j], q[j].D, e * v[j]);
             Bs[j] = fmaf(Bs[j], q[j].D, e);
         }
+        if constexpr (GATED) apply_gate(pr, y);
         if (valid) Vec<IO, CPT>::store(py, y);
     }
 };
@@ -409,6 +434,8 @@ struct ScanOp {
     static constexpr int CPT = 1;
     static constexpr int CG = 32;
     static constexpr int NV = 2;
+    static constexpr int NIN = 2;
+    static constexpr bool kGated = false;
     static constexpr bool kSerialForm = false;
     struct Param {};
     struct State {
@@ -472,9 +499,9 @@ struct ScanOp {
 
     template <int LS>
     __device__ __forceinline__ static void sweep(const State (&carry)[1], const float *p0,
-                                                 const float *p1, int n, const Param (&)[1],
-                                                 const Scratch (&)[1], float *out, size_t ostride,
-                                                 bool valid) {
+                                                 const float *p1, const float *, int n,
+                                                 const Param (&)[1], const Scratch (&)[1],
+                                                 float *out, size_t ostride, bool valid) {
         float H = carry[0].H;
         if (n == LS) {
 #pragma unroll 8

@@ -25,6 +25,10 @@ Named workloads (shapes from RWKV-4 models and the minGRU scan form):
   w = exp(U(-6,0)); u ~ N(0,1)
 * ``scan_mingru`` diagonal scan fp32, B=64 T=4096 D=256 in minGRU form:
   z = sigmoid(N(0,1)), h~ ~ N(0,1), a = 1 - z, b = z * h~, h0 = 0
+* ``wkv_3b_gated_bf16`` the receptance-gated WKV sigma(r) (.) wkv with bf16
+  k/v/r/y, B=8 T=4096 C=2560; k, v, w, u as ``wkv_3b_bf16``, then r ~ N(0, 2)
+* ``shift_3b_bf16`` token shift (3 mixing vectors: k, v, r) on bf16 x,
+  B=8 T=4096 C=2560; x ~ N(0, 1), mu ~ U(0, 1) (see ``make_token_shift``)
 * ``wkv_decode`` WKV fp32 RNN-mode decoding, one token per sequence: B=1024
   sequences, T=1, C=2560 (RWKV-4-3B width), k, v, w, u as ``wkv_169m``, plus
   a state per (sequence, channel) from ``make_wkv_state``
@@ -44,7 +48,7 @@ import numpy as np
 __all__ = [
     "WkvSpec", "ScanSpec", "WORKLOADS", "WkvInputs", "ScanInputs",
     "make_wkv", "make_scan", "bf16_round", "bf16_bits", "bf16_bits_to_f32",
-    "get_workload", "make_wkv_state",
+    "get_workload", "make_wkv_state", "ShiftSpec", "ShiftInputs", "make_token_shift",
 ]
 
 
@@ -62,6 +66,8 @@ class WkvSpec:
     u_sigma: float = 0.5          # u ~ N(0, u_sigma)
     seed: int = 0
     state: bool = False           # the workload starts from a drawn state
+    gated: bool = False           # also draws the receptance r ~ N(0, r_sigma)
+    r_sigma: float = 2.0
 
     @property
     def elements(self) -> int:
@@ -91,7 +97,28 @@ WORKLOADS = {
     "scan_mingru": ScanSpec("scan_mingru", 64, 4096, 256),
     "wkv_decode": WkvSpec("wkv_decode", 1024, 1, 2560, "f32", 1.0, 1.0, ("uniform", -3.0, 1.0),
                           0.5, state=True),
+    "wkv_3b_gated_bf16": WkvSpec("wkv_3b_gated_bf16", 8, 4096, 2560, "bf16", 1.0, 1.0,
+                                 ("uniform", -3.0, 1.0), 0.5, gated=True),
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class ShiftSpec:
+    """Shape of one token-shift workload."""
+    name: str
+    B: int
+    T: int
+    C: int
+    n_mix: int = 3
+    dtype: str = "f32"
+    seed: int = 0
+
+    @property
+    def elements(self) -> int:
+        return self.B * self.T * self.C
+
+
+WORKLOADS["shift_3b_bf16"] = ShiftSpec("shift_3b_bf16", 8, 4096, 2560, 3, "bf16")
 
 
 def get_workload(name: str):
@@ -136,6 +163,8 @@ class WkvInputs:
     k_bits: Optional[np.ndarray] = None
     v_bits: Optional[np.ndarray] = None
     s_in: Optional[np.ndarray] = None   # [B, 3, C] float32 when spec.state
+    r: Optional[np.ndarray] = None      # [B, T, C] float32 when spec.gated
+    r_bits: Optional[np.ndarray] = None
 
 
 @dataclasses.dataclass
@@ -172,11 +201,43 @@ def make_wkv(spec, *, B=None, T=None, C=None, seed=None) -> WkvInputs:
     v = rng.normal(0.0, spec.v_sigma, size=shape).astype(np.float32)
     w = np.exp(_draw_log_w(rng, spec.w_log, spec.C)).astype(np.float32)
     u = rng.normal(0.0, spec.u_sigma, size=spec.C).astype(np.float32)
+    r = rng.normal(0.0, spec.r_sigma, size=shape).astype(np.float32) if spec.gated else None
     s_in = make_wkv_state(spec.B, spec.C, spec.seed) if spec.state else None
     if spec.dtype == "bf16":
         kb, vb = bf16_bits(k), bf16_bits(v)
-        return WkvInputs(spec, w, u, bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), kb, vb, s_in)
-    return WkvInputs(spec, w, u, k, v, s_in=s_in)
+        rb = bf16_bits(r) if r is not None else None
+        return WkvInputs(spec, w, u, bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), kb, vb, s_in,
+                         None if rb is None else bf16_bits_to_f32(rb), rb)
+    return WkvInputs(spec, w, u, k, v, s_in=s_in, r=r)
+
+
+@dataclasses.dataclass
+class ShiftInputs:
+    spec: ShiftSpec
+    x: np.ndarray        # [B, T, C] float32 (bf16-rounded values for bf16)
+    mu: np.ndarray       # [n_mix, C] float32
+    x_prev: np.ndarray   # [B, C] float32 (bf16-rounded for bf16)
+    x_bits: Optional[np.ndarray] = None
+    x_prev_bits: Optional[np.ndarray] = None
+
+
+def make_token_shift(spec, *, B=None, T=None, C=None, n_mix=None, seed=None) -> ShiftInputs:
+    """Draw one token-shift workload: x ~ N(0, 1) [B, T, C], mu ~ U(0, 1)
+    [n_mix, C], x_prev ~ N(0, 1) [B, C], in that order."""
+    if isinstance(spec, str):
+        spec = WORKLOADS[spec]
+    spec = dataclasses.replace(
+        spec, B=spec.B if B is None else B, T=spec.T if T is None else T,
+        C=spec.C if C is None else C, n_mix=spec.n_mix if n_mix is None else n_mix,
+        seed=spec.seed if seed is None else seed)
+    rng = np.random.default_rng(spec.seed)
+    x = rng.normal(0.0, 1.0, size=(spec.B, spec.T, spec.C)).astype(np.float32)
+    mu = rng.uniform(0.0, 1.0, size=(spec.n_mix, spec.C)).astype(np.float32)
+    xp = rng.normal(0.0, 1.0, size=(spec.B, spec.C)).astype(np.float32)
+    if spec.dtype == "bf16":
+        xb, pb = bf16_bits(x), bf16_bits(xp)
+        return ShiftInputs(spec, bf16_bits_to_f32(xb), mu, bf16_bits_to_f32(pb), xb, pb)
+    return ShiftInputs(spec, x, mu, xp)
 
 
 def make_wkv_state(B: int, C: int, seed: int = 0, p_sigma: float = 2.0) -> np.ndarray:
