@@ -70,6 +70,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--tile-steps", type=int, default=0,
+                    help="steps per tile (8, 32, 64, 128, 256); 0 keeps the library default")
     ap.add_argument("--launch", default="graph", choices=["graph", "direct"],
                     help="replay the K steps from CUDA graphs (default) or call directly")
     return ap.parse_args(argv)
@@ -639,6 +641,8 @@ def main(argv=None):
     import rwkv_wkv_mixing_b200 as wkv
     props = torch.cuda.get_device_properties(local)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    if args.tile_steps:
+        wkv.wkv_set_tile_steps(args.tile_steps)
     wl = DeviceWorkload(args.workload, torch, wkv.lib, l2)
 
     def barrier():

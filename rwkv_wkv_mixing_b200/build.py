@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libwkv_b200.so")
 SOURCES = ["capi.cu", "noalloc.cu"]
-HEADERS = ["chunked_scan.cuh", "persistent_scan.cuh", "scan_common.cuh", "wkv_ops.cuh", "ptx.cuh"]
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -164,6 +164,11 @@ __global__ void __launch_bounds__(NW * 32, 3)
 
     // ---- carry into the tile (warp 0) ---------------------------------------
     if (warp == 0) {
+        // the look-back's first records are loaded now and land while the
+        // warp folds and publishes this tile's aggregate
+        LookbackPrefetch<Op> pf;
+        const bool lb = chained && seg > 0;
+        if (lb) lookback_prefetch<Op>(ws, g, tile, lane, pf);
         State agg[CPT], X[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(NW * 32, 3)
                     publish<Op, CG>(ws, g, tile, agg, kFlagAgg, epoch, lane);
                 // decoupled look-back over the tiles before this one in time
                 State run[CPT];
-                if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run)) {
+                if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run, lb ? &pf : nullptr)) {
                     atomicExch(ws.status, kStatusTimeout);  // this lane gave up
 #pragma unroll
                     for (int j = 0; j < CPT; ++j) run[j] = Op::nan_state();

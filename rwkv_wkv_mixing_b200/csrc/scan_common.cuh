@@ -112,6 +112,31 @@ __device__ __forceinline__ void finish_launch(const Workspace &ws, bool chained,
     }
 }
 
+// The first records a tile's look-back will read, loaded ahead of time: the
+// look-back does not depend on the tile's own data, so the carry warp issues
+// these loads before it folds and publishes its own aggregate, and they land
+// while it does.
+template <class Op>
+struct LookbackPrefetch {
+    static constexpr int kHops = 4 / Op::CPT;
+    uint4 rec[Op::CPT][kHops];
+};
+
+template <class Op>
+__device__ __forceinline__ void lookback_prefetch(const Workspace &ws, const Geometry &g, int tile,
+                                                  int lane, LookbackPrefetch<Op> &pf) {
+    constexpr int CPT = Op::CPT, CG = 32 * CPT;
+    const long long S = g.tiles_per_seg;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+#pragma unroll
+        for (int i = 0; i < LookbackPrefetch<Op>::kHops; ++i) {
+            const long long q = static_cast<long long>(tile) - (i + 1) * S;
+            pf.rec[j][i] = make_uint4(0u, 0u, 0u, 0u);
+            if (q >= 0) pf.rec[j][i] = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
+        }
+}
+
 // Decoupled look-back for one tile, each lane for its own CPT channels.  The
 // tiles before this one in time are tile - S, tile - 2S, ... (S = tiles per
 // time segment).  A lane folds its channel's records newest first -- a tile
@@ -124,8 +149,10 @@ template <class Op, int LT>
 __device__ __forceinline__ bool lookback(const Workspace &ws, const Geometry &g, int tile,
                                          unsigned long long epoch,
                                          const typename Op::Param (&prm)[Op::CPT], int lane,
-                                         typename Op::State (&run)[Op::CPT]) {
+                                         typename Op::State (&run)[Op::CPT],
+                                         const LookbackPrefetch<Op> *pre = nullptr) {
     constexpr int CPT = Op::CPT, CG = 32 * CPT, HB = 4;  // hops per batch of loads
+    constexpr int PH = LookbackPrefetch<Op>::kHops;
     const long long S = g.tiles_per_seg;
     bool ok = true;
 #pragma unroll
@@ -134,15 +161,19 @@ __device__ __forceinline__ bool lookback(const Workspace &ws, const Geometry &g,
         float run_len = 0.f;
         long long base = tile;
         bool done = false;
+        bool first = true;
         while (!done && ok) {
             uint4 rec[HB];
 #pragma unroll
             for (int i = 0; i < HB; ++i) {
                 const long long q = base - (i + 1) * S;
                 rec[i] = make_uint4(0u, 0u, 0u, 0u);
-                if (q >= 0)
+                if (first && pre != nullptr && i < PH)
+                    rec[i] = pre->rec[j][i];   // possibly stale: re-polled below if not ready
+                else if (q >= 0)
                     rec[i] = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
             }
+            first = false;
 #pragma unroll
             for (int i = 0; i < HB; ++i) {
                 if (done || !ok) break;

@@ -111,6 +111,13 @@ __device__ __forceinline__ float wkv_output(float a, float b, float e, float v) 
     return v + fmaf(-b, v, a) * rcp_approx(b + e);
 }
 
+// e^x through the MUFU ex2 unit, for factors that weigh one term against a
+// term of weight exactly 1 (arguments <= 0 after max-normalisation): the
+// relative error, about 2^-22 plus |x| 2^-24 from rounding x log2(e), only
+// matters where e^x is large, i.e. for small |x|.  Not for factors that get
+// raised to powers (the per-step decay e^{-w} uses expf).
+__device__ __forceinline__ float fast_exp(float x) { return ex2_approx(x * kLog2e); }
+
 // The receptance gate sigma(r) = 1 / (1 + e^{-r}) of eq. (15) of
 // "RWKV：基于RNN的LLM".  Saturates cleanly: e^{-r} = inf gives 0, e^{-r} = 0
 // gives 1.
@@ -127,8 +134,13 @@ __device__ __forceinline__ float gate_sigmoid(float r) {
 // Stepping the state: (num, den)_{t+1} = e^{-w} (num, den)_t + e^{k_t} (v_t, 1).
 //
 // Pass 1 (summary of a sub-chunk ending at step `end`, from the empty state):
-// p = m = max_i (k_i - (end-i) w), then a = sum_i e^{k_i - (end-i) w - m} v_i,
-// b = the same without v_i: every exponent is <= 0 and the largest term is 1.
+// one round finds max k and min k (packed pairs for bf16), a second sums
+// a = sum_i e^{k_i - (end-i) w - p} v_i and b = the same without v_i against
+// the reference p = max k, so every exponent is <= 0.  Any reference is the
+// same state; max k only risks that every term of a chunk whose largest key
+// is decayed away falls far below 1 -- when b < 2^-60 the chunk is summed
+// again against the exact largest exponent p = max_i (k_i - (end-i) w),
+// whose term is exactly 1.
 //
 // Pass 2 (outputs of a sub-chunk from the state before it): one reference
 // M = max(p_in, max_i k_i) for the whole sub-chunk, state scaled to e^M, so
@@ -220,7 +232,7 @@ struct WkvOp {
     __device__ __forceinline__ static void pack(const State &s, float &x, float &y,
                                                 uint32_t &bits16) {
         const float pi = fminf(fmaxf(ceilf(s.p), -32768.f), 32767.f);
-        const float f = expf(s.p - pi);
+        const float f = fast_exp(s.p - pi);
         x = s.a * f;
         y = s.b * f;
         bits16 = static_cast<uint32_t>(static_cast<int>(pi) + 32768);
@@ -233,7 +245,7 @@ struct WkvOp {
                                                     const Param &q) {
         const float pd = fmaf(-r_len, q.w, l.p);
         const float m = fmaxf(pd, r.p);
-        const float fl = expf(pd - m), fr = expf(r.p - m);
+        const float fl = fast_exp(pd - m), fr = fast_exp(r.p - m);
         return {fmaf(l.a, fl, r.a * fr), fmaf(l.b, fl, r.b * fr), m};
     }
 
@@ -249,33 +261,79 @@ struct WkvOp {
             return (x - r) * kLog2e;
     }
 
+    // round 1: largest and smallest key of each channel over n rows
     template <int LS>
-    __device__ __forceinline__ static void summarize(const IO *p0, const IO *p1, int n,
-                                                     const Param (&q)[CPT], State (&out)[CPT],
-                                                     Scratch (&sc)[CPT]) {
-        float m[CPT], m2[CPT], kx[CPT], kn[CPT], a[CPT], b[CPT];
+    __device__ __forceinline__ static void key_range(const IO *p0, int n, float (&kx)[CPT],
+                                                     float (&kn)[CPT]) {
+        if constexpr (sizeof(IO) == 2 && CPT == 2) {
+            // bf16 pairs: max and min are exact in bf16, two channels per op
+            const __nv_bfloat16 ninf = __ushort_as_bfloat16(0xff80u), pinf = __ushort_as_bfloat16(0x7f80u);
+            __nv_bfloat162 hx = __halves2bfloat162(ninf, ninf), hn = __halves2bfloat162(pinf, pinf);
+            if (n == LS) {
+#pragma unroll 8
+                for (int i = 0; i < LS; ++i) {
+                    const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(p0 + i * CG);
+                    hx = __hmax2(hx, k2);
+                    hn = __hmin2(hn, k2);
+                }
+            } else {
+                for (int i = 0; i < n; ++i) {
+                    const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(p0 + i * CG);
+                    hx = __hmax2(hx, k2);
+                    hn = __hmin2(hn, k2);
+                }
+            }
+            const float2 fx = __bfloat1622float2(hx), fn = __bfloat1622float2(hn);
+            kx[0] = fx.x;
+            kx[1] = fx.y;
+            kn[0] = fn.x;
+            kn[1] = fn.y;
+        } else {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                kx[j] = kNoScale;
+                kn[j] = -kNoScale;
+            }
+            if (n == LS) {
+#pragma unroll 8
+                for (int i = 0; i < LS; ++i) {
+                    float k[CPT];
+                    Vec<IO, CPT>::load(p0 + i * CG, k);
+#pragma unroll
+                    for (int j = 0; j < CPT; ++j) {
+                        kx[j] = fmaxf(kx[j], k[j]);
+                        kn[j] = fminf(kn[j], k[j]);
+                    }
+                }
+            } else {
+                for (int i = 0; i < n; ++i) {
+                    float k[CPT];
+                    Vec<IO, CPT>::load(p0 + i * CG, k);
+#pragma unroll
+                    for (int j = 0; j < CPT; ++j) {
+                        kx[j] = fmaxf(kx[j], k[j]);
+                        kn[j] = fminf(kn[j], k[j]);
+                    }
+                }
+            }
+        }
+    }
+
+    // round 2: a = sum_i e^{k_i - (end-i) w - ref} v_i, b = the same without
+    // v_i, over n rows ending at row n-1
+    template <int LS>
+    __device__ __forceinline__ static void chunk_sums(const IO *p0, const IO *p1, int n,
+                                                      const Param (&q)[CPT],
+                                                      const float (&ref)[CPT], float (&a)[CPT],
+                                                      float (&b)[CPT]) {
+        float ref2[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
-            m[j] = kNoScale;
-            kx[j] = kNoScale;
-            kn[j] = -kNoScale;
+            ref2[j] = ref[j] * kLog2e;
             a[j] = 0.f;
             b[j] = 0.f;
         }
         if (n == LS) {
-#pragma unroll 8
-            for (int i = 0; i < LS; ++i) {
-                float k[CPT];
-                Vec<IO, CPT>::load(p0 + i * CG, k);
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) {
-                    m[j] = fmaxf(m[j], fmaf(static_cast<float>(i - (LS - 1)), q[j].w, k[j]));
-                    kx[j] = fmaxf(kx[j], k[j]);
-                    kn[j] = fminf(kn[j], k[j]);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < CPT; ++j) m2[j] = m[j] * kLog2e;
 #pragma unroll 8
             for (int i = 0; i < LS; ++i) {
                 float k[CPT], v[CPT];
@@ -284,24 +342,12 @@ struct WkvOp {
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) {
                     const float x = fmaf(static_cast<float>(i - (LS - 1)), q[j].w, k[j]);
-                    const float e = ex2_approx(exp_arg(x, m[j], m2[j]));
+                    const float e = ex2_approx(exp_arg(x, ref[j], ref2[j]));
                     a[j] = fmaf(e, v[j], a[j]);
                     b[j] += e;
                 }
             }
         } else {
-            for (int i = 0; i < n; ++i) {
-                float k[CPT];
-                Vec<IO, CPT>::load(p0 + i * CG, k);
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) {
-                    m[j] = fmaxf(m[j], fmaf(static_cast<float>(i - (n - 1)), q[j].w, k[j]));
-                    kx[j] = fmaxf(kx[j], k[j]);
-                    kn[j] = fminf(kn[j], k[j]);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < CPT; ++j) m2[j] = m[j] * kLog2e;
             for (int i = 0; i < n; ++i) {
                 float k[CPT], v[CPT];
                 Vec<IO, CPT>::load(p0 + i * CG, k);
@@ -309,15 +355,64 @@ struct WkvOp {
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) {
                     const float x = fmaf(static_cast<float>(i - (n - 1)), q[j].w, k[j]);
-                    const float e = ex2_approx(exp_arg(x, m[j], m2[j]));
+                    const float e = ex2_approx(exp_arg(x, ref[j], ref2[j]));
                     a[j] = fmaf(e, v[j], a[j]);
                     b[j] += e;
                 }
             }
         }
+    }
+
+    // the exact largest exponent max_i (k_i - (end-i) w) of one channel
+    __device__ __forceinline__ static float largest_exponent(const IO *p0, int n, int j,
+                                                             const Param &q) {
+        float m = kNoScale;
+        for (int i = 0; i < n; ++i) {
+            float k[CPT];
+            Vec<IO, CPT>::load(p0 + i * CG, k);
+            m = fmaxf(m, fmaf(static_cast<float>(i - (n - 1)), q.w, k[j]));
+        }
+        return m;
+    }
+
+    template <int LS>
+    __device__ __forceinline__ static void summarize(const IO *p0, const IO *p1, int n,
+                                                     const Param (&q)[CPT], State (&out)[CPT],
+                                                     Scratch (&sc)[CPT]) {
+        if (n <= 0) {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                out[j] = identity();
+                sc[j] = {kNoScale, -kNoScale};
+            }
+            return;
+        }
+        float kx[CPT], kn[CPT], a[CPT], b[CPT];
+        key_range<LS>(p0, n, kx, kn);
+        chunk_sums<LS>(p0, p1, n, q, kx, a, b);
+        float ref[CPT];
+        bool redo = false;
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
-            out[j] = {a[j], b[j], m[j]};
+            ref[j] = kx[j];
+            if (!(b[j] >= 0x1p-60f)) {  // the chunk's weight sits far below max k
+                ref[j] = largest_exponent(p0, n, j, q[j]);
+                redo = true;
+            }
+        }
+        if (redo) {
+            float a2[CPT], b2[CPT];
+            chunk_sums<LS>(p0, p1, n, q, ref, a2, b2);
+#pragma unroll
+            for (int j = 0; j < CPT; ++j)
+                if (ref[j] != kx[j]) {
+                    a[j] = a2[j];
+                    b[j] = b2[j];
+                }
+        }
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            out[j] = {a[j], b[j], ref[j]};
             sc[j] = {kx[j], kn[j]};
         }
     }
@@ -359,7 +454,7 @@ struct WkvOp {
         for (int j = 0; j < CPT; ++j) {
             M[j] = fmaxf(carry[j].p, sc[j].kmax);
             M2[j] = M[j] * kLog2e;
-            const float s = expf(carry[j].p - M[j]);
+            const float s = fast_exp(carry[j].p - M[j]);
             A[j] = carry[j].a * s;
             Bs[j] = carry[j].b * s;
             // den_t >= e^{u + k_t - M}, and den_t >= b_in e^{p_in - M - t w}
@@ -413,8 +508,9 @@ struct WkvOp {
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
             const float e = ex2_approx(exp_arg(k[j], M[j], M2[j]));
-            const float eu = e * q[j].U;
-            y[j] = wkv_output(A[j], Bs[j], eu, v[j]);
+            // (A + e U v) / (Bs + e U) in the residual form of wkv_output, the
+            // denominator in one FMA
+            y[j] = v[j] + fmaf(-Bs[j], v[j], A[j]) * rcp_approx(fmaf(e, q[j].U, Bs[j]));
             A[j] = fmaf(A[j], q[j].D, e * v[j]);
             Bs[j] = fmaf(Bs[j], q[j].D, e);
         }

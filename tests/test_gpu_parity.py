@@ -169,6 +169,35 @@ def test_wkv_f32_extreme_values(m):
     assert_close(got, want, wkv_tol(T, np.abs(v).max()), "extreme")
 
 
+@pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
+def test_wkv_chunk_whose_largest_key_decays_away(m, bf16):
+    """Sub-chunks whose largest key comes first and is decayed far below the
+    rest (w = 10, one key of +30 among keys of -30): summed against max k
+    every term would sit below 2^-60, so pass 1 re-sums them against the
+    exact largest exponent; results still match the oracle."""
+    rng = np.random.default_rng(37)
+    B, T, C = 2, 600, 64
+    k = np.full((B, T, C), -30.0) + rng.normal(0, 0.5, (B, T, C))
+    k[:, ::32, :] = 30.0          # the first step of every 32-step sub-chunk
+    k[:, 5::97, :16] = 45.0       # and a few late spikes elsewhere
+    v = rng.normal(0, 1, (B, T, C))
+    w = np.concatenate([np.full(32, 10.0), np.exp(rng.uniform(-3, 3, 32))])
+    u = rng.normal(0, 1, C)
+    if bf16:
+        kb, vb = workloads.bf16_bits(k.astype(np.float32)), workloads.bf16_bits(v.astype(np.float32))
+        k, v = workloads.bf16_bits_to_f32(kb), workloads.bf16_bits_to_f32(vb)
+        y = m.wkv_forward_bf16(dev(w), dev(u), bf16_dev(kb), bf16_dev(vb))
+        torch.cuda.synchronize()
+        got = y.float().double().cpu().numpy()
+        tol = 2e-2 * np.abs(v).max()
+    else:
+        k, v = k.astype(np.float32), v.astype(np.float32)
+        got = run_f32(m, w.astype(np.float32), u.astype(np.float32), k, v)
+        tol = wkv_tol(T, np.abs(v).max())
+    want = oracle.wkv_rnn(w.astype(np.float32), u.astype(np.float32), k, v)
+    assert_close(got, want, tol, "decayed-away largest key")
+
+
 def test_wkv_on_side_streams_concurrently(m):
     """Two streams at once: each has its own look-back workspace."""
     xs = [workloads.make_wkv("wkv_169m", B=2, T=2000, C=128, seed=s) for s in (41, 42)]
