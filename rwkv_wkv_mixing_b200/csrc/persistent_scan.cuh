@@ -78,7 +78,14 @@ __device__ __forceinline__ bool wait_fill(uint64_t *bar, const int *fill_it, int
     const volatile int *stamp = fill_it;
     const unsigned long long t0 = global_timer_ns();
     for (unsigned n = 0;; ++n) {
-        if (*stamp == it && mbar_try_wait(bar, parity)) return true;
+        // try_wait suspends the warp in hardware until the phase completes
+        // (or a time limit passes), so waiting costs no issue slots; a
+        // completed phase whose stamp is not ours is an older fill of the
+        // stage: back off until the producer re-arms it for this iteration
+        if (mbar_try_wait(bar, parity)) {
+            if (*stamp == it) return true;
+            __nanosleep(64);
+        }
         if ((n & 63u) == 63u) {
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > kBarrierWaitNs) {
