@@ -304,7 +304,7 @@ class DeviceWorkload:
             return "token_shift_kernel"
         if self.kind == "wkv" and self.T <= 16:
             return "wkv_serial_kernel"
-        if self.lib.wkv_get_tile_steps() in (8, 32):
+        if self.lib.wkv_tile_steps_for(self.B, self.T, self.C, self.es) in (8, 32):
             return "chunked_scan_kernel"
         return "persistent_scan_kernel"
 
@@ -720,7 +720,7 @@ def main(argv=None):
                 "l2": (f"inputs rotate over {wl.n_sets} buffer sets "
                        f"({wl.n_sets * wl.set_bytes / 1e6:.0f} MB > L2 "
                        f"{l2 / 1e6:.0f} MB)"),
-                "tile_steps": wkv.wkv_get_tile_steps(),
+                "tile_steps": wkv.wkv_tile_steps_for(wl.B, wl.T, wl.C, wl.es),
                 "launch": args.launch + (" (K steps replayed from captured graphs)"
                                          if args.launch == "graph" else ""),
                 "gpu": props.name, "sms": props.multi_processor_count})

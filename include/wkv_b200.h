@@ -261,11 +261,16 @@ WKV_API const char *wkv_last_error(void);
 WKV_API wkv_status wkv_release_workspaces(void);
 
 /* Tuning knob, process-wide: the number of steps one thread block stages per
- * tile (8, 32, 64, 128 or 256; default 128).  Results do not depend on it
- * beyond rounding: it only moves the boundaries where chunk summaries are
+ * tile (8, 32, 64, 128 or 256), or 0 (the default) to let each call choose:
+ * 128, or 256 for sequences longer than 4096 steps whose rows and channels
+ * make fewer than 64 tiles per tile-length of time.  Results do not depend on
+ * it beyond rounding: it only moves the boundaries where chunk summaries are
  * combined.  WKV_ERR_INVALID_ARG for any other value. */
 WKV_API wkv_status wkv_set_tile_steps(int steps);
 WKV_API int wkv_get_tile_steps(void);
+/* The tile length a WKV or scan call of this shape uses now (elem_bytes: 4
+ * for fp32 I/O, 2 for bf16); 0 for an invalid shape. */
+WKV_API int wkv_tile_steps_for(int64_t B, int64_t T, int64_t C, int elem_bytes);
 
 /* Test hook for failure detection, process-wide, for later launches of the
  * allocating entry points.  skip_tile >= 0: that tile (in the launch's

@@ -57,6 +57,7 @@ _SIGS = {
     "wkv_release_workspaces": ([], _i32),
     "wkv_set_tile_steps": ([_i32], _i32),
     "wkv_get_tile_steps": ([], _i32),
+    "wkv_tile_steps_for": ([_i64, _i64, _i64, _i32], _i32),
     "wkv_set_fault_injection": ([_i32, _i64], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -375,7 +376,13 @@ def wkv_set_tile_steps(steps: int):
 
 
 def wkv_get_tile_steps() -> int:
+    """The knob's value; 0 means each call chooses (see wkv_tile_steps_for)."""
     return int(lib.wkv_get_tile_steps())
+
+
+def wkv_tile_steps_for(B: int, T: int, C: int, elem_bytes: int = 4) -> int:
+    """The tile length a call of this shape uses under the current knob."""
+    return int(lib.wkv_tile_steps_for(B, T, C, elem_bytes))
 
 
 def wkv_set_fault_injection(skip_tile: int = -1, spin_limit: int = 0):
@@ -389,4 +396,4 @@ __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan"
            "wkv_forward_state", "wkv_forward_bf16_state", "wkv_forward_gated", "token_shift",
            "wkv_forward_host", "wkv_forward_bf16_host", "diag_scan_host", "wkv_device_status",
            "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
-           "wkv_get_tile_steps", "WkvError", "lib", "LIB_PATH"]
+           "wkv_get_tile_steps", "wkv_tile_steps_for", "WkvError", "lib", "LIB_PATH"]

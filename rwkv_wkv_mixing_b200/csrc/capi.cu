@@ -76,7 +76,7 @@ const Driver &driver() {
 }
 
 // ---- tuning knob: tile length in steps ---------------------------------------
-std::atomic<int> g_tile_steps{128};
+std::atomic<int> g_tile_steps{0};  // 0: chosen per call (tile_steps_for)
 
 // ---- fault-injection test hook (see wkv_set_fault_injection) -----------------
 std::atomic<int> g_fault_skip_tile{-1};
@@ -372,6 +372,17 @@ wkv_status launch_persistent(const typename Op::Args &args, int64_t B, int64_t T
     return WKV_OK;
 }
 
+// Steps per tile: the knob's value, or when it is 0, 128 unless a time
+// segment holds too few tiles to keep the SMs' consumer groups fed -- long
+// sequences over few rows and channels -- where 256-step tiles halve the
+// length of the carry chain between tiles.
+int tile_steps_for(int64_t B, int64_t T, int64_t C, int cg) {
+    const int knob = g_tile_steps.load();
+    if (knob != 0) return knob;
+    const int64_t tiles_per_seg = B * ((C + cg - 1) / cg);
+    return (T > 4096 && tiles_per_seg < 64) ? 256 : 128;
+}
+
 // Sequences of at most this many steps (single-token decoding included) run
 // on the serial kernel: one thread per (row, channel), no tiles, no workspace.
 constexpr int64_t kSerialMaxSteps = 16;
@@ -410,9 +421,10 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
     int nptr = 3;
     if constexpr (Op::NIN == 3) ptrs[nptr++] = args.x2;
     const bool tma = tma_eligible(ptrs, nptr, sizeof(typename Op::io_t), T, C);
+    const int lt = tile_steps_for(B, T, C, 32 * Op::CPT);
     if constexpr (Op::NIN == 3) {
         // a third input tile per stage: fewer stages and groups fit in shared memory
-        switch (g_tile_steps.load()) {
+        switch (lt) {
             case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
             case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
             case 64:
@@ -426,7 +438,7 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
                            : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
         }
     } else {
-        switch (g_tile_steps.load()) {
+        switch (lt) {
             case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
             case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
             case 64:
@@ -952,13 +964,18 @@ wkv_status wkv_release_workspaces(void) {
 
 wkv_status wkv_set_tile_steps(int steps) {
     t_err.clear();
-    if (steps != 8 && steps != 32 && steps != 64 && steps != 128 && steps != 256)
-        return fail(WKV_ERR_INVALID_ARG, "tile steps must be 8, 32, 64, 128 or 256");
+    if (steps != 0 && steps != 8 && steps != 32 && steps != 64 && steps != 128 && steps != 256)
+        return fail(WKV_ERR_INVALID_ARG, "tile steps must be 0 (automatic), 8, 32, 64, 128 or 256");
     g_tile_steps.store(steps);
     return WKV_OK;
 }
 
 int wkv_get_tile_steps(void) { return g_tile_steps.load(); }
+
+int wkv_tile_steps_for(int64_t B, int64_t T, int64_t C, int elem_bytes) {
+    if (B < 1 || T < 1 || C < 1 || (elem_bytes != 2 && elem_bytes != 4)) return 0;
+    return tile_steps_for(B, T, C, elem_bytes == 2 ? 64 : 32);
+}
 
 wkv_status wkv_set_fault_injection(int skip_tile, long long spin_limit) {
     t_err.clear();

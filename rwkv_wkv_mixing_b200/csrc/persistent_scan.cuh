@@ -45,7 +45,7 @@ struct PersistentCfg {
     static_assert(LT <= 256, "TMA box rows are limited to 256");
     static_assert(NSTAGE > NC, "one stage per group plus at least one being loaded");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
-    static_assert(1 + NC <= 16, "named barrier ids");
+    static_assert(2 + NC <= 16, "named barrier ids: 0, one per group, one for all consumers");
 };
 
 // Wait for phase `parity` of `bar`; false if the block is aborting or the
@@ -140,9 +140,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
     // dependency on the previous grid in the stream, nothing global is read
     // before that grid has finished
     grid_dependency_wait();
-    if (threadIdx.x == 0) s_epoch = chained ? epoch_of(ws) : 0ull;
     __syncthreads();
-    const unsigned long long epoch = s_epoch;
     volatile int *abort_flag = &s_abort;
 
     if (warp == 0) {
@@ -162,6 +160,8 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                     if (chained) {
                         // tickets go out in the order blocks ask for them, so a
                         // tile only ever waits for tiles already being worked on
+                        // (one ticket per stage: handing a block consecutive
+                        // tickets up front delays the tiles later ones depend on)
                         const unsigned t = atomicAdd(ws.ticket, 1u);
                         tile = t < static_cast<unsigned>(g.tiles) ? static_cast<int>(t) : -1;
                     } else {
@@ -196,6 +196,11 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
         __syncwarp();
     } else {
         // ---------------- consumer group ----------------
+        // the launch's epoch, read by one consumer thread while the producer
+        // already takes tickets and starts loads
+        if (threadIdx.x == 32) s_epoch = chained ? epoch_of(ws) : 0ull;
+        named_bar_sync(NC + 1, NC * NWG * 32);
+        const unsigned long long epoch = s_epoch;
         const int cw = warp - 1;
         const int grp = cw / NWG, wg = cw - grp * NWG;
         const int gtid = wg * 32 + lane;

@@ -53,6 +53,13 @@ def test_host_side_argument_errors():
     assert lib.wkv_set_tile_steps(100) == wkv.WKV_ERR_INVALID_ARG
     assert lib.wkv_set_tile_steps(64) == wkv.WKV_OK and lib.wkv_get_tile_steps() == 64
     assert lib.wkv_set_tile_steps(256) == wkv.WKV_OK and lib.wkv_get_tile_steps() == 256
+    assert lib.wkv_tile_steps_for(8, 1024, 768, 4) == 256
+    assert lib.wkv_set_tile_steps(0) == wkv.WKV_OK and lib.wkv_get_tile_steps() == 0
+    # automatic: 128 steps, 256 for long sequences over few tiles per segment
+    assert lib.wkv_tile_steps_for(8, 1024, 768, 4) == 128
+    assert lib.wkv_tile_steps_for(1, 131072, 1024, 4) == 256
+    assert lib.wkv_tile_steps_for(8, 4096, 2560, 2) == 128
+    assert lib.wkv_tile_steps_for(0, 1, 1, 4) == 0
 
 
 def test_product_path_has_no_cpu_fallback():
