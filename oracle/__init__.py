@@ -25,6 +25,11 @@ Pieces (all float64; each cites the page it follows):
   time-mixing projections, mu x_t + (1 - mu) x_{t-1} (eqs. (11)-(13) of
   "RWKV：基于RNN的LLM", section 二.1; x_{-1} is the layer's saved last token,
   "last_x", of the HarmonyOS RWKV article's time-mixing code section, or 0).
+* ``lru_scan``            -- the LRU's complex diagonal recurrence
+  x_t = lambda x_{t-1} + gamma u_t with lambda = e^{-e^{nu_log} + i e^{theta_log}}
+  (review of "Resurrecting Recurrent Neural Networks for Long Sequences",
+  linear-RNN section), complex128; ``lru_direct_points`` is its unrolled sum
+  x_t = gamma sum_k lambda^{t-k} u_k (+ lambda^{t+1} x_{-1}).
 * ``sigmoid`` / ``wkv_gated`` -- the receptance gate sigma(r_t) (.) wkv_t of
   eq. (15) of the same page and of the LRU review's RWKV variant.
 * ``wkv_slru_ratio_np``   -- the "RWKV = ratio of two SLRUs" form from the
@@ -58,7 +63,7 @@ __all__ = [
     "build", "max_threads", "wkv_direct", "wkv_direct_points", "wkv_direct_np",
     "wkv_rnn", "wkv_slru_ratio_np", "scan_rnn", "scan_direct_points",
     "wkv_direct_state", "wkv_rnn_state", "state_mean_logden",
-    "token_shift", "sigmoid", "wkv_gated",
+    "token_shift", "sigmoid", "wkv_gated", "lru_lambda", "lru_scan", "lru_direct_points",
 ]
 
 
@@ -323,3 +328,51 @@ def wkv_gated(w, u, k, v, r, s_in=None):
     optionally from a state.  Returns (out, s_out)."""
     y, s_out = wkv_rnn_state(w, u, k, v, s_in)
     return sigmoid(r) * y, s_out
+
+
+# ---------------------------------------------------------------------------
+# LRU: complex diagonal linear recurrence
+# ---------------------------------------------------------------------------
+def lru_lambda(nu_log, theta_log):
+    """lambda = r e^{i theta} with r = e^{-nu}, nu = e^{nu_log}, theta = e^{theta_log}
+    (the LRU review's parameterisation, linear-RNN section)."""
+    nu = np.exp(np.asarray(nu_log, dtype=np.float64))
+    theta = np.exp(np.asarray(theta_log, dtype=np.float64))
+    return np.exp(-nu) * np.exp(1j * theta)
+
+
+def lru_scan(nu_log, theta_log, gamma, u, x0=None):
+    """x_t = lambda x_{t-1} + gamma u_t per channel, x_{-1} = x0 (0 if None).
+    u: complex [B, T, D] (or real); gamma: [D] real or None (1).  Returns
+    complex128 [B, T, D]."""
+    lam = lru_lambda(nu_log, theta_log)
+    u = np.asarray(u)
+    B, T, D = u.shape
+    g = np.ones(D) if gamma is None else np.asarray(gamma, dtype=np.float64)
+    x = np.zeros((B, D), dtype=np.complex128) if x0 is None else \
+        np.asarray(x0, dtype=np.complex128).reshape(B, D).copy()
+    out = np.empty((B, T, D), dtype=np.complex128)
+    for t in range(T):
+        x = lam * x + g * u[:, t].astype(np.complex128)
+        out[:, t] = x
+    return out
+
+
+def lru_direct_points(nu_log, theta_log, gamma, u, x0, points):
+    """The unrolled sum x_t = gamma sum_{k<=t} lambda^{t-k} u_k + lambda^{t+1} x_{-1}
+    at flat indices b*T*D + t*D + d (powers from exp of the scaled exponent)."""
+    nu = np.exp(np.asarray(nu_log, dtype=np.float64))
+    theta = np.exp(np.asarray(theta_log, dtype=np.float64))
+    u = np.asarray(u).astype(np.complex128)
+    B, T, D = u.shape
+    g = np.ones(D) if gamma is None else np.asarray(gamma, dtype=np.float64)
+    out = np.empty(len(points), dtype=np.complex128)
+    for j, f in enumerate(np.asarray(points, dtype=np.int64)):
+        b, t, d = f // (T * D), (f // D) % T, f % D
+        n = t - np.arange(t + 1)                     # t - k for k = 0..t
+        pw = np.exp(n * (-nu[d] + 1j * theta[d]))    # lambda^{t-k}
+        acc = g[d] * np.sum(pw * u[b, :t + 1, d])
+        if x0 is not None:
+            acc += np.exp((t + 1) * (-nu[d] + 1j * theta[d])) * complex(np.asarray(x0)[b, d])
+        out[j] = acc
+    return out

@@ -37,8 +37,10 @@ def read_golden(name):
 
 
 def _close(got, want, tol):
-    got = np.asarray(got, dtype=np.float64)
-    want = np.asarray(want, dtype=np.float64)
+    got, want = np.asarray(got), np.asarray(want)
+    cplx = np.iscomplexobj(got) or np.iscomplexobj(want)
+    got = got.astype(np.complex128 if cplx else np.float64)
+    want = want.astype(np.complex128 if cplx else np.float64)
     if got.shape != want.shape:
         return f"shape {got.shape} != {want.shape}"
     err = np.max(np.abs(got - want)) if got.size else 0.0
@@ -459,6 +461,110 @@ def run_gate_pins(fn):
     for pin in GATE_PINS:
         try:
             fails += pin(fn)
+        except Exception as e:
+            fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
+    return fails
+
+
+# ---------------------------------------------------------------------------
+# LRU scan: fn(nu_log, theta_log, gamma, u, x0) -> complex x [B, T, D]
+# ---------------------------------------------------------------------------
+def lru_worked_example(fn, tol=1e-14):
+    g = read_golden("lru_worked_example.txt")
+    nu_log = np.array([np.log(-np.log(float(g["r"][0])))])
+    theta_log = np.array([np.log(np.pi * float(g["theta_over_pi"][0]))])
+    u = (np.array([float(x) for x in g["u_re"]]) + 1j * np.array([float(x) for x in g["u_im"]]))
+    u = u.reshape(1, 3, 1)
+    out = []
+    for case, x0 in (("case1", None), ("case2", np.array([[float(g["case2_x0_re"][0]) +
+                                                           1j * float(g["case2_x0_im"][0])]]))):
+        want = np.array([float(x) for x in g[f"{case}_x_re"]]) + \
+            1j * np.array([float(x) for x in g[f"{case}_x_im"]])
+        got = np.asarray(fn(nu_log, theta_log, np.array([float(g[f"{case}_gamma"][0])]), u, x0))
+        msg = _close(got.reshape(-1), want, tol)
+        if msg: out.append(f"lru worked example {case}: {msg}")
+    return out
+
+
+def lru_impulse(fn, tol=1e-12):
+    """u = delta at t = 0: x_t = gamma lambda^t = gamma r^t (cos t theta + i sin t theta)."""
+    D, T = 4, 50
+    nu_log = np.log(np.array([0.01, 0.1, 0.5, 2.0]))
+    theta_log = np.log(np.array([0.3, 1.0, 2.5, 6.0]))
+    gamma = np.array([1.0, 0.5, 2.0, 0.1])
+    u = np.zeros((1, T, D), dtype=complex); u[0, 0] = 1.0
+    t = np.arange(T)[:, None]
+    r, th = np.exp(-np.exp(nu_log)), np.exp(theta_log)
+    want = gamma * r ** t * (np.cos(t * th) + 1j * np.sin(t * th))
+    msg = _close(np.asarray(fn(nu_log, theta_log, gamma, u, None))[0], want, tol)
+    return [f"lru impulse response: {msg}"] if msg else []
+
+
+def lru_real_case(fn, tol=1e-12, scan=None):
+    """theta -> 0 makes lambda real (= e^{-nu}): real and imaginary parts each
+    follow the real diagonal scan with a = e^{-nu}, b = gamma u."""
+    rng = np.random.default_rng(41)
+    B, T, D = 2, 40, 3
+    nu_log = rng.normal(-1, 1, D); theta_log = np.full(D, -200.0)
+    gamma = rng.uniform(0.5, 1.5, D)
+    u = rng.normal(0, 1, (B, T, D)) + 1j * rng.normal(0, 1, (B, T, D))
+    x0 = rng.normal(0, 1, (B, D)) + 1j * rng.normal(0, 1, (B, D))
+    got = np.asarray(fn(nu_log, theta_log, gamma, u, x0))
+    a = np.broadcast_to(np.exp(-np.exp(nu_log)), (B, T, D))
+    out = []
+    for part, name in ((np.real, "re"), (np.imag, "im")):
+        want = scan(a, gamma * part(u), part(x0))
+        msg = _close(part(got), want, tol)
+        if msg: out.append(f"lru real case ({name}): {msg}")
+    return out
+
+
+def lru_linearity_and_chaining(fn, tol=1e-12):
+    rng = np.random.default_rng(42)
+    B, T, D = 2, 30, 4
+    nu_log, theta_log = rng.normal(-2, 1, D), rng.normal(0, 1, D)
+    gamma = rng.uniform(0.5, 1.5, D)
+    u = rng.normal(0, 1, (B, T, D)) + 1j * rng.normal(0, 1, (B, T, D))
+    x0 = rng.normal(0, 1, (B, D)) + 1j * rng.normal(0, 1, (B, D))
+    x = np.asarray(fn(nu_log, theta_log, gamma, u, x0))
+    out = []
+    rot = np.exp(0.7j)
+    msg = _close(np.asarray(fn(nu_log, theta_log, gamma, rot * u, rot * x0)), rot * x, tol)
+    if msg: out.append(f"lru rotation equivariance: {msg}")
+    x1 = np.asarray(fn(nu_log, theta_log, gamma, u[:, :11], x0))
+    x2 = np.asarray(fn(nu_log, theta_log, gamma, u[:, 11:], x1[:, -1]))
+    msg = _close(np.concatenate([x1, x2], axis=1), x, tol)
+    if msg: out.append(f"lru chaining: {msg}")
+    return out
+
+
+def lru_variance(fn):
+    """For iid zero-mean u, E|x_t|^2 = gamma^2 (1 - r^{2(t+1)}) / (1 - r^2) E|u|^2
+    (the LRU review's initialisation section); checked statistically."""
+    rng = np.random.default_rng(43)
+    B, T, D = 4000, 24, 2
+    nu_log = np.log(-np.log(np.array([0.9, 0.5])))
+    theta_log = np.log(np.array([1.0, 2.0]))
+    gamma = np.array([1.0, 0.7])
+    u = (rng.normal(0, 1, (B, T, D)) + 1j * rng.normal(0, 1, (B, T, D))) / np.sqrt(2)
+    x = np.asarray(fn(nu_log, theta_log, gamma, u, None))
+    r = np.array([0.9, 0.5])
+    t = np.arange(T)[:, None]
+    want = gamma ** 2 * (1 - r ** (2 * (t + 1))) / (1 - r ** 2)
+    got = np.mean(np.abs(x) ** 2, axis=0)
+    rel = np.max(np.abs(got - want) / want)
+    return [] if rel < 0.1 else [f"lru variance formula: rel err {rel:.3f}"]
+
+
+LRU_PINS = [lru_worked_example, lru_impulse, lru_real_case, lru_linearity_and_chaining,
+            lru_variance]
+
+
+def run_lru_pins(fn, scan):
+    fails = []
+    for pin in LRU_PINS:
+        try:
+            fails += pin(fn, scan=scan) if pin is lru_real_case else pin(fn)
         except Exception as e:
             fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
     return fails

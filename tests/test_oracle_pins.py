@@ -338,6 +338,43 @@ def test_planted_mistake_in_gate_is_caught(kind):
     assert pins.run_gate_pins(fn) != []
 
 
+# --- LRU complex scan ----------------------------------------------------
+def _lru_points(nu_log, theta_log, gamma, u, x0):
+    u = np.asarray(u)
+    pts = np.arange(u.size)
+    return oracle.lru_direct_points(nu_log, theta_log, gamma, u, x0, pts).reshape(u.shape)
+
+
+@pytest.mark.parametrize("fn", [oracle.lru_scan, _lru_points], ids=["recurrence", "unrolled"])
+def test_lru_oracle_passes_pins(fn):
+    assert pins.run_lru_pins(fn, oracle.scan_rnn) == []
+
+
+@pytest.mark.parametrize("kind", ["conj", "gamma_on_state", "x0_undecayed", "r_squared"])
+def test_planted_mistake_in_lru_is_caught(kind):
+    def fn(nu_log, theta_log, gamma, u, x0):
+        lam = oracle.lru_lambda(nu_log, theta_log)
+        if kind == "conj":
+            lam = np.conj(lam)
+        if kind == "r_squared":
+            lam = lam * np.abs(lam)
+        u = np.asarray(u).astype(complex)
+        B, T, D = u.shape
+        g = np.ones(D) if gamma is None else np.asarray(gamma, float)
+        x = np.zeros((B, D), complex) if x0 is None else np.asarray(x0, complex).copy()
+        out = np.empty((B, T, D), complex)
+        for t in range(T):
+            if kind == "gamma_on_state":
+                x = g * (lam * x + u[:, t])
+            elif kind == "x0_undecayed" and t == 0:
+                x = x + g * u[:, t]
+            else:
+                x = lam * x + g * u[:, t]
+            out[:, t] = x
+        return out
+    assert pins.run_lru_pins(fn, oracle.scan_rnn) != []
+
+
 # --- diagonal scan ---------------------------------------------------------
 def scan_rnn(a, b, h0):
     return oracle.scan_rnn(a, b, h0)
@@ -393,3 +430,17 @@ def test_worked_examples_read():
     assert len(g["y"]) == len(g["v"]) == 4
     g = pins.read_golden("scan_worked_example.txt")
     assert len(g["h"]) == len(g["a"]) == 4
+
+
+def test_minlstm_workload_is_a_convex_scan():
+    """minLSTM's normalised gates sum to one (f' + i' = 1), so each state is a
+    convex combination of the previous one and the candidate: the scan stays
+    within the running range of the candidates (h0 = 0 included)."""
+    x = workloads.make_scan("scan_minlstm", B=3, T=200, D=8)
+    f_prime = x.a.astype(np.float64)
+    i_prime = x.b.astype(np.float64) / x.h_tilde.astype(np.float64)
+    assert np.allclose(f_prime + i_prime, 1.0, atol=1e-6)
+    h = oracle.scan_rnn(x.a, x.b, None)
+    lo = np.minimum(np.minimum.accumulate(x.h_tilde, axis=1), 0.0)
+    hi = np.maximum(np.maximum.accumulate(x.h_tilde, axis=1), 0.0)
+    assert np.all(h >= lo - 1e-6) and np.all(h <= hi + 1e-6)

@@ -25,6 +25,14 @@ Named workloads (shapes from RWKV-4 models and the minGRU scan form):
   w = exp(U(-6,0)); u ~ N(0,1)
 * ``scan_mingru`` diagonal scan fp32, B=64 T=4096 D=256 in minGRU form:
   z = sigmoid(N(0,1)), h~ ~ N(0,1), a = 1 - z, b = z * h~, h0 = 0
+* ``scan_mingru_bf16`` the same minGRU-form scan with bf16 a, b, h storage
+  (values rounded to bf16 after the float32 recipe)
+* ``scan_minlstm`` diagonal scan fp32, B=64 T=4096 D=256 in minLSTM form:
+  f = sigmoid(N(0,1)), i = sigmoid(N(0,1)), h~ ~ N(0,1) (drawn in that order),
+  a = f / (f + i), b = i / (f + i) * h~, h0 = 0 (the normalised gates of the
+  "Were RNNs All We Needed?" article's minLSTM section)
+* ``lru_256`` the LRU's complex diagonal recurrence, B=64 T=4096 D=256 complex
+  channels (see ``make_lru``)
 * ``wkv_3b_gated_bf16`` the receptance-gated WKV sigma(r) (.) wkv with bf16
   k/v/r/y, B=8 T=4096 C=2560; k, v, w, u as ``wkv_3b_bf16``, then r ~ N(0, 2)
 * ``shift_3b_bf16`` token shift (3 mixing vectors: k, v, r) on bf16 x,
@@ -49,6 +57,7 @@ __all__ = [
     "WkvSpec", "ScanSpec", "WORKLOADS", "WkvInputs", "ScanInputs",
     "make_wkv", "make_scan", "bf16_round", "bf16_bits", "bf16_bits_to_f32",
     "get_workload", "make_wkv_state", "ShiftSpec", "ShiftInputs", "make_token_shift",
+    "LruSpec", "LruInputs", "make_lru",
 ]
 
 
@@ -76,13 +85,15 @@ class WkvSpec:
 
 @dataclasses.dataclass(frozen=True)
 class ScanSpec:
-    """Shape of one minGRU-form diagonal scan workload."""
+    """Shape of one diagonal scan workload (minGRU or minLSTM form)."""
     name: str
     B: int
     T: int
     D: int
     seed: int = 0
     with_h0: bool = False         # minGRU recipe uses h0 = 0 (passed as "none")
+    form: str = "mingru"          # "mingru" or "minlstm"
+    dtype: str = "f32"            # "f32" or "bf16" storage of a, b, h
 
     @property
     def elements(self) -> int:
@@ -95,6 +106,8 @@ WORKLOADS = {
     "wkv_3b_bf16": WkvSpec("wkv_3b_bf16", 8, 4096, 2560, "bf16", 1.0, 1.0, ("uniform", -3.0, 1.0), 0.5),
     "wkv_long": WkvSpec("wkv_long", 1, 131072, 1024, "f32", 3.0, 1.0, ("uniform", -6.0, 0.0), 1.0),
     "scan_mingru": ScanSpec("scan_mingru", 64, 4096, 256),
+    "scan_mingru_bf16": ScanSpec("scan_mingru_bf16", 64, 4096, 256, dtype="bf16"),
+    "scan_minlstm": ScanSpec("scan_minlstm", 64, 4096, 256, form="minlstm"),
     "wkv_decode": WkvSpec("wkv_decode", 1024, 1, 2560, "f32", 1.0, 1.0, ("uniform", -3.0, 1.0),
                           0.5, state=True),
     "wkv_3b_gated_bf16": WkvSpec("wkv_3b_gated_bf16", 8, 4096, 2560, "bf16", 1.0, 1.0,
@@ -170,10 +183,12 @@ class WkvInputs:
 @dataclasses.dataclass
 class ScanInputs:
     spec: ScanSpec
-    a: np.ndarray   # [B, T, D] float32
-    b: np.ndarray   # [B, T, D] float32
+    a: np.ndarray   # [B, T, D] float32 (bf16-rounded values for bf16)
+    b: np.ndarray   # [B, T, D] float32 (bf16-rounded values for bf16)
     h0: Optional[np.ndarray]   # [B, D] float32 or None (zeros)
     h_tilde: Optional[np.ndarray] = None   # [B, T, D] float32, the candidate states
+    a_bits: Optional[np.ndarray] = None    # bf16 storage for bf16 workloads
+    b_bits: Optional[np.ndarray] = None
 
 
 def _draw_log_w(rng, spec_w, C):
@@ -250,7 +265,8 @@ def make_wkv_state(B: int, C: int, seed: int = 0, p_sigma: float = 2.0) -> np.nd
 
 
 def make_scan(spec, *, B=None, T=None, D=None, seed=None, with_h0=None) -> ScanInputs:
-    """Draw one minGRU-form diagonal-scan workload (a = 1 - z, b = z * h~)."""
+    """Draw one diagonal-scan workload: minGRU form (a = 1 - z, b = z * h~)
+    or minLSTM form (a = f / (f + i), b = i / (f + i) * h~)."""
     if isinstance(spec, str):
         spec = WORKLOADS[spec]
     spec = dataclasses.replace(
@@ -259,9 +275,81 @@ def make_scan(spec, *, B=None, T=None, D=None, seed=None, with_h0=None) -> ScanI
         with_h0=spec.with_h0 if with_h0 is None else with_h0)
     rng = np.random.default_rng(spec.seed)
     shape = (spec.B, spec.T, spec.D)
-    z = 1.0 / (1.0 + np.exp(-rng.normal(0.0, 1.0, size=shape)))
-    h_tilde = rng.normal(0.0, 1.0, size=shape)
-    a = (1.0 - z).astype(np.float32)
-    b = (z * h_tilde).astype(np.float32)
+    if spec.form == "minlstm":
+        f = 1.0 / (1.0 + np.exp(-rng.normal(0.0, 1.0, size=shape)))
+        i = 1.0 / (1.0 + np.exp(-rng.normal(0.0, 1.0, size=shape)))
+        h_tilde = rng.normal(0.0, 1.0, size=shape)
+        a = (f / (f + i)).astype(np.float32)
+        b = (i / (f + i) * h_tilde).astype(np.float32)
+    else:
+        z = 1.0 / (1.0 + np.exp(-rng.normal(0.0, 1.0, size=shape)))
+        h_tilde = rng.normal(0.0, 1.0, size=shape)
+        a = (1.0 - z).astype(np.float32)
+        b = (z * h_tilde).astype(np.float32)
     h0 = rng.normal(0.0, 1.0, size=(spec.B, spec.D)).astype(np.float32) if spec.with_h0 else None
+    if spec.dtype == "bf16":
+        ab, bb = bf16_bits(a), bf16_bits(b)
+        return ScanInputs(spec, bf16_bits_to_f32(ab), bf16_bits_to_f32(bb), h0,
+                          h_tilde.astype(np.float32), ab, bb)
     return ScanInputs(spec, a, b, h0, h_tilde.astype(np.float32))
+
+
+@dataclasses.dataclass(frozen=True)
+class LruSpec:
+    """Shape of one LRU (complex diagonal recurrence) workload."""
+    name: str
+    B: int
+    T: int
+    D: int
+    r_min: float = 0.9
+    r_max: float = 0.999
+    seed: int = 0
+    with_x0: bool = False
+
+    @property
+    def elements(self) -> int:
+        return self.B * self.T * self.D
+
+
+WORKLOADS["lru_256"] = LruSpec("lru_256", 64, 4096, 256)
+
+
+@dataclasses.dataclass
+class LruInputs:
+    spec: LruSpec
+    nu_log: np.ndarray     # [D] float32
+    theta_log: np.ndarray  # [D] float32
+    gamma: np.ndarray      # [D] float32
+    u: np.ndarray          # [B, T, D, 2] float32: real and imaginary parts
+    x0: Optional[np.ndarray] = None   # [B, D, 2] float32 or None
+
+    def u_complex(self):
+        return self.u[..., 0].astype(np.float64) + 1j * self.u[..., 1].astype(np.float64)
+
+    def x0_complex(self):
+        if self.x0 is None:
+            return None
+        return self.x0[..., 0].astype(np.float64) + 1j * self.x0[..., 1].astype(np.float64)
+
+
+def make_lru(spec, *, B=None, T=None, D=None, seed=None, with_x0=None) -> LruInputs:
+    """Draw one LRU workload with the LRU review's initialisation: r^2 ~
+    U[r_min^2, r_max^2], theta ~ U[0, 2 pi], stored as nu_log = ln(-ln r)
+    and theta_log = ln theta; gamma = sqrt(1 - r^2); u complex with real and
+    imaginary parts ~ N(0, 1/2); drawn in that order (x0 last, same law as u)."""
+    if isinstance(spec, str):
+        spec = WORKLOADS[spec]
+    spec = dataclasses.replace(
+        spec, B=spec.B if B is None else B, T=spec.T if T is None else T,
+        D=spec.D if D is None else D, seed=spec.seed if seed is None else seed,
+        with_x0=spec.with_x0 if with_x0 is None else with_x0)
+    rng = np.random.default_rng(spec.seed)
+    r = np.sqrt(rng.uniform(spec.r_min ** 2, spec.r_max ** 2, size=spec.D))
+    theta = rng.uniform(0.0, 2.0 * np.pi, size=spec.D)
+    nu_log = np.log(-np.log(r)).astype(np.float32)
+    theta_log = np.log(theta).astype(np.float32)
+    gamma = np.sqrt(1.0 - r ** 2).astype(np.float32)
+    u = rng.normal(0.0, np.sqrt(0.5), size=(spec.B, spec.T, spec.D, 2)).astype(np.float32)
+    x0 = rng.normal(0.0, np.sqrt(0.5), size=(spec.B, spec.D, 2)).astype(np.float32) \
+        if spec.with_x0 else None
+    return LruInputs(spec, nu_log, theta_log, gamma, u, x0)
