@@ -32,6 +32,10 @@ Pieces (all float64; each cites the page it follows):
   x_t = gamma sum_k lambda^{t-k} u_k (+ lambda^{t+1} x_{-1}).
 * ``sigmoid`` / ``wkv_gated`` -- the receptance gate sigma(r_t) (.) wkv_t of
   eq. (15) of the same page and of the LRU review's RWKV variant.
+* ``wkv_backward_direct`` / ``wkv_backward_rnn`` -- gradients of eq. (14)
+  with respect to k, v, w and u (the pages give none): the derivative of a
+  softmax-weighted mean written out per output (O(T^2)), and the same by a
+  forward and a reverse recurrence (O(T)).
 * ``wkv_slru_ratio_np``   -- the "RWKV = ratio of two SLRUs" form from the
   review of "Resurrecting Recurrent Neural Networks for Long Sequences"
   (section on the RWKV variant), unstabilised; |k| small only.
@@ -64,6 +68,7 @@ __all__ = [
     "wkv_rnn", "wkv_slru_ratio_np", "scan_rnn", "scan_direct_points",
     "wkv_direct_state", "wkv_rnn_state", "state_mean_logden",
     "token_shift", "sigmoid", "wkv_gated", "lru_lambda", "lru_scan", "lru_direct_points",
+    "wkv_backward_direct", "wkv_backward_rnn",
 ]
 
 
@@ -94,6 +99,10 @@ def _get():
                 "oracle_wkv_direct_points_s": [i64, i64, i64, p, p, p, p, p, i64, p, p,
                                                ctypes.c_int],
                 "oracle_wkv_rnn_s": [i64, i64, i64, p, p, p, p, p, p, p, ctypes.c_int],
+                "oracle_wkv_backward_direct": [i64, i64, i64, p, p, p, p, p, p, p, p, p,
+                                               ctypes.c_int],
+                "oracle_wkv_backward_rnn": [i64, i64, i64, p, p, p, p, p, p, p, p, p,
+                                            ctypes.c_int],
                 "oracle_scan_rnn": [i64, i64, i64, p, p, p, p, ctypes.c_int],
                 "oracle_scan_direct_points": [i64, i64, i64, p, p, p, i64, p, p, ctypes.c_int],
             }.items():
@@ -376,3 +385,30 @@ def lru_direct_points(nu_log, theta_log, gamma, u, x0, points):
             acc += np.exp((t + 1) * (-nu[d] + 1j * theta[d])) * complex(np.asarray(x0)[b, d])
         out[j] = acc
     return out
+
+
+# ---------------------------------------------------------------------------
+# WKV gradients
+# ---------------------------------------------------------------------------
+def _wkv_backward(name, w, u, k, v, gy, nthreads):
+    B, T, C, w, u, k, v = _wkv_args(w, u, k, v)
+    gy = _f64(gy)
+    if gy.shape != k.shape:
+        raise ValueError("gy must have the shape of k")
+    gk = np.empty_like(k)
+    gv = np.empty_like(k)
+    gw = np.empty(C)
+    gu = np.empty(C)
+    getattr(_get(), name)(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(gy), _ptr(gk),
+                          _ptr(gv), _ptr(gw), _ptr(gu), nthreads)
+    return gk, gv, gw, gu
+
+
+def wkv_backward_direct(w, u, k, v, gy, nthreads: int = 0):
+    """(gk, gv, gw, gu) for upstream gradient gy, by the definition (O(T^2))."""
+    return _wkv_backward("oracle_wkv_backward_direct", w, u, k, v, gy, nthreads)
+
+
+def wkv_backward_rnn(w, u, k, v, gy, nthreads: int = 0):
+    """(gk, gv, gw, gu) by a forward and a reverse recurrence (O(T))."""
+    return _wkv_backward("oracle_wkv_backward_rnn", w, u, k, v, gy, nthreads)

@@ -34,6 +34,7 @@
 #include <stdint.h>
 #include <stddef.h>
 #include <omp.h>
+#include <stdlib.h>
 
 static int pick_threads(int nthreads) {
     return nthreads > 0 ? nthreads : omp_get_max_threads();
@@ -218,6 +219,143 @@ void oracle_wkv_rnn(int64_t B, int64_t T, int64_t C,
                     const double *w, const double *u,
                     const double *k, const double *v, double *y, int nthreads) {
     oracle_wkv_rnn_s(B, T, C, w, u, k, v, NULL, y, NULL, nthreads);
+}
+
+/* ------------------------------------------------------------------------
+ * WKV gradients.  The pages print no gradient formulas; eq. (14) is a
+ * softmax-weighted mean
+ *     y_t = sum_{j<=t} beta_{t,j} v_j,   beta_{t,j} = e^{l_{t,j}} / sum_i e^{l_{t,i}},
+ *     l_{t,j} = -(t-1-j) w + k_j  (j < t),   l_{t,t} = u + k_t,
+ * so with dL/dy_t = g_t, dy_t/dv_j = beta_{t,j} and dy_t/dl_{t,j} =
+ * beta_{t,j} (v_j - y_t), and the logits depend on k_j (slope 1), on u (the
+ * diagonal, slope 1) and on w (slope -(t-1-j) below the diagonal):
+ *     gv_j = sum_{t>=j} g_t beta_{t,j}
+ *     gk_j = sum_{t>=j} g_t beta_{t,j} (v_j - y_t)
+ *     gu   = sum_t g_t beta_{t,t} (v_t - y_t)            (summed over b too)
+ *     gw   = -sum_t sum_{j<t} (t-1-j) g_t beta_{t,j} (v_j - y_t)
+ * Definition form: every beta by its own max-stabilised softmax, O(T^2) per
+ * channel.  gw, gu are [C] sums over batch rows and steps.
+ * ------------------------------------------------------------------------ */
+void oracle_wkv_backward_direct(int64_t B, int64_t T, int64_t C,
+                                const double *w, const double *u,
+                                const double *k, const double *v, const double *gy,
+                                double *gk, double *gv, double *gw, double *gu, int nthreads) {
+    for (int64_t c = 0; c < C; ++c) { gw[c] = 0.0; gu[c] = 0.0; }
+#pragma omp parallel for schedule(dynamic, 1) num_threads(pick_threads(nthreads))
+    for (int64_t c = 0; c < C; ++c) {
+        double gw_c = 0.0, gu_c = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            const double *kb = k + b * T * C + c, *vb = v + b * T * C + c, *gb = gy + b * T * C + c;
+            double *gkb = gk + b * T * C + c, *gvb = gv + b * T * C + c;
+            for (int64_t j = 0; j < T; ++j) { gkb[j * C] = 0.0; gvb[j * C] = 0.0; }
+            for (int64_t t = 0; t < T; ++t) {
+                /* logits of output t and their softmax */
+                double m = u[c] + kb[t * C];
+                for (int64_t j = 0; j < t; ++j) {
+                    double l = -(double)(t - 1 - j) * w[c] + kb[j * C];
+                    if (l > m) m = l;
+                }
+                double den = 0.0, num = 0.0;
+                for (int64_t j = 0; j <= t; ++j) {
+                    double l = j < t ? -(double)(t - 1 - j) * w[c] + kb[j * C] : u[c] + kb[t * C];
+                    double e = exp(l - m);
+                    den += e;
+                    num += e * vb[j * C];
+                }
+                double y = num / den, g = gb[t * C];
+                for (int64_t j = 0; j <= t; ++j) {
+                    double l = j < t ? -(double)(t - 1 - j) * w[c] + kb[j * C] : u[c] + kb[t * C];
+                    double beta = exp(l - m) / den;
+                    double dl = g * beta * (vb[j * C] - y);   /* dL / d logit */
+                    gvb[j * C] += g * beta;
+                    gkb[j * C] += dl;
+                    if (j == t) gu_c += dl;
+                    else gw_c -= (double)(t - 1 - j) * dl;
+                }
+            }
+        }
+        gw[c] = gw_c;
+        gu[c] = gu_c;
+    }
+}
+
+/* ------------------------------------------------------------------------
+ * The same gradients by recurrences, O(T) per channel: a forward sweep keeps
+ * y_t and L_t = ln D_t (D_t the output's denominator, sum_i e^{l_{t,i}}); a
+ * reverse sweep keeps, for the step j being visited, the sums over later
+ * outputs t > j
+ *     P_j  = sum_{t>j} e^{-(t-1-j) w} g_t / D_t,        Q_j  = the same with g_t y_t,
+ *     R_j  = sum_{t>j} (t-1-j) e^{-(t-1-j) w} g_t / D_t, R2_j = the same with g_t y_t,
+ * which obey  P_{j-1} = g_j / D_j + e^{-w} P_j  (Q likewise with g_j y_j) and
+ * R_{j-1} = e^{-w} (R_j + P_j)  (R2 likewise with Q).  Then, since
+ * beta_{t,j} = e^{k_j - (t-1-j) w} / D_t below the diagonal and
+ * beta_{j,j} = e^{u + k_j} / D_j,
+ *     gv_j = e^{u+k_j-L_j} g_j + e^{k_j} P_j
+ *     gk_j = e^{u+k_j-L_j} g_j (v_j - y_j) + e^{k_j} (v_j P_j - Q_j)
+ *     gu  += e^{u+k_j-L_j} g_j (v_j - y_j),   gw -= e^{k_j} (v_j R_j - R2_j).
+ * The four sums share one scale e^{-rho}; rho_{j-1} = min(L_j, rho_j + w)
+ * keeps every exponent <= 0, and rho_j >= k_j, so e^{k_j - rho_j} <= 1.
+ * ------------------------------------------------------------------------ */
+void oracle_wkv_backward_rnn(int64_t B, int64_t T, int64_t C,
+                             const double *w, const double *u,
+                             const double *k, const double *v, const double *gy,
+                             double *gk, double *gv, double *gw, double *gu, int nthreads) {
+    for (int64_t c = 0; c < C; ++c) { gw[c] = 0.0; gu[c] = 0.0; }
+#pragma omp parallel num_threads(pick_threads(nthreads))
+    {
+        double *ys = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        double *Ls = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t c = 0; c < C; ++c) {
+            double gw_c = 0.0, gu_c = 0.0;
+            for (int64_t b = 0; b < B; ++b) {
+                const double *kb = k + b * T * C + c, *vb = v + b * T * C + c;
+                const double *gb = gy + b * T * C + c;
+                double *gkb = gk + b * T * C + c, *gvb = gv + b * T * C + c;
+                /* forward sweep (RNN mode, as oracle_wkv_rnn) keeping y_t, L_t */
+                double a = 0.0, d = 0.0, p = -INFINITY;
+                for (int64_t t = 0; t < T; ++t) {
+                    double kt = kb[t * C], vt = vb[t * C];
+                    double x = u[c] + kt, q = p > x ? p : x;
+                    double ep = exp(p - q), ex = exp(x - q);
+                    double den = ep * d + ex;
+                    ys[t] = (ep * a + ex * vt) / den;
+                    Ls[t] = q + log(den);
+                    double pd = p - w[c], q2 = pd > kt ? pd : kt;
+                    double fo = exp(pd - q2), fn = exp(kt - q2);
+                    a = fo * a + fn * vt;
+                    d = fo * d + fn;
+                    p = q2;
+                }
+                /* reverse sweep */
+                double P = 0.0, Q = 0.0, R = 0.0, R2 = 0.0, rho = INFINITY;
+                for (int64_t j = T - 1; j >= 0; --j) {
+                    double kj = kb[j * C], vj = vb[j * C], gj = gb[j * C];
+                    double diag = exp(u[c] + kj - Ls[j]) * gj;   /* g_j beta_{j,j} */
+                    double sc = exp(kj - rho);                    /* e^{k_j} e^{-rho} */
+                    gvb[j * C] = diag + sc * P;
+                    gkb[j * C] = diag * (vj - ys[j]) + sc * (vj * P - Q);
+                    gu_c += diag * (vj - ys[j]);
+                    gw_c -= sc * (vj * R - R2);
+                    /* sums for step j-1: add output j, decay the rest by e^{-w} */
+                    double r2 = rho + w[c];
+                    double nr = Ls[j] < r2 ? Ls[j] : r2;
+                    double fnew = exp(nr - Ls[j]), fold = exp(nr - r2);
+                    double Pn = fnew * gj + fold * P;
+                    double Qn = fnew * gj * ys[j] + fold * Q;
+                    R = fold * (R + P);
+                    R2 = fold * (R2 + Q);
+                    P = Pn;
+                    Q = Qn;
+                    rho = nr;
+                }
+            }
+            gw[c] = gw_c;
+            gu[c] = gu_c;
+        }
+        free(ys);
+        free(Ls);
+    }
 }
 
 /* ------------------------------------------------------------------------

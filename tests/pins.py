@@ -571,6 +571,125 @@ def run_lru_pins(fn, scan):
 
 
 # ---------------------------------------------------------------------------
+# WKV gradients: fn(w, u, k, v, gy) -> (gk, gv, gw, gu), gw and gu [C]
+# ---------------------------------------------------------------------------
+def grad_worked_example(fn, tol=1e-12):
+    g = read_golden("wkv_grad_worked_example.txt")
+    w = np.array([-np.log(float(g["w_exp_neg"][0]))])
+    u = np.array([np.log(float(g["u_exp"][0]))])
+    k = np.log(np.array([float(x) for x in g["k_exp"]]))[None, :, None]
+    v = np.array([float(x) for x in g["v"]])[None, :, None]
+    gy = np.array([float(x) for x in g["g"]])[None, :, None]
+    gk, gv, gw, gu = fn(w, u, k, v, gy)
+    out = []
+    for name, got in (("gk", gk), ("gv", gv), ("gw", gw), ("gu", gu)):
+        want = np.array([float(x) for x in g[name]])
+        msg = _close(np.asarray(got).reshape(-1), want, tol)
+        if msg: out.append(f"gradient worked example {name}: {msg}")
+    return out
+
+
+def _torch_grads(w, u, k, v, gy):
+    """Reverse-mode autodiff (PyTorch, float64) through eq. (14) written as a
+    masked softmax over the [T, T] logits."""
+    import torch
+    tw, tu, tk, tv = (torch.tensor(np.asarray(x, dtype=np.float64), requires_grad=True)
+                      for x in (w, u, k, v))
+    B, T, C = tk.shape
+    t_idx = torch.arange(T)[:, None]
+    i_idx = torch.arange(T)[None, :]
+    dist = (t_idx - 1 - i_idx).double()
+    logit = -dist[None, :, :, None] * tw[None, None, None, :] + tk[:, None, :, :]
+    diag = (tu[None, None, :] + tk)[:, :, None, :].expand(B, T, T, C)
+    eye = (t_idx == i_idx)[None, :, :, None].expand(B, T, T, C)
+    logit = torch.where(eye, diag, logit)
+    logit = logit.masked_fill((i_idx > t_idx)[None, :, :, None].expand(B, T, T, C), float("-inf"))
+    beta = torch.softmax(logit, dim=2)
+    y = (beta * tv[:, None, :, :]).sum(dim=2)
+    (y * torch.tensor(np.asarray(gy, dtype=np.float64))).sum().backward()
+    return tk.grad.numpy(), tv.grad.numpy(), tw.grad.numpy(), tu.grad.numpy()
+
+
+def grad_autodiff(fn, tol=1e-11):
+    """Against reverse-mode autodiff of the definition on random inputs."""
+    w, u, k, v = _rand_wkv(51, B=2, T=24, C=3)
+    gy = np.random.default_rng(51).normal(0, 1, k.shape)
+    got = fn(w, u, k, v, gy)
+    want = _torch_grads(w, u, k, v, gy)
+    out = []
+    for name, a, b in zip(("gk", "gv", "gw", "gu"), got, want):
+        msg = _close(a, b, tol * max(1.0, float(np.abs(b).max())))
+        if msg: out.append(f"gradient vs autodiff {name}: {msg}")
+    return out
+
+
+def grad_finite_difference(fn, h=1e-6, tol=1e-7):
+    """Central differences of the definition itself (numpy, float64)."""
+    w, u, k, v = _rand_wkv(52, B=1, T=6, C=2, ksig=1.0)
+    gy = np.random.default_rng(52).normal(0, 1, k.shape)
+
+    def loss(w_, u_, k_, v_):
+        T = k_.shape[1]
+        tot = 0.0
+        for c in range(k_.shape[2]):
+            for t in range(T):
+                l = np.array([-(t - 1 - j) * w_[c] + k_[0, j, c] for j in range(t)] + [u_[c] + k_[0, t, c]])
+                e = np.exp(l - l.max())
+                tot += gy[0, t, c] * np.dot(e, v_[0, :t + 1, c]) / e.sum()
+        return tot
+
+    gk, gv, gw, gu = fn(w, u, k, v, gy)
+    out = []
+    for name, arr, grad in (("k", k, gk), ("v", v, gv), ("w", w, gw), ("u", u, gu)):
+        for idx in ([(0, 0, 0), (0, 3, 1), (0, 5, 0)] if arr.ndim == 3 else [(0,), (1,)]):
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += h
+            a2[idx] -= h
+            args1 = {"k": (w, u, a1, v), "v": (w, u, k, a1), "w": (a1, u, k, v), "u": (w, a1, k, v)}[name]
+            args2 = {"k": (w, u, a2, v), "v": (w, u, k, a2), "w": (a2, u, k, v), "u": (w, a2, k, v)}[name]
+            fd = (loss(*args1) - loss(*args2)) / (2 * h)
+            if abs(fd - np.asarray(grad)[idx]) > tol:
+                out.append(f"gradient vs central difference d{name}{idx}: {np.asarray(grad)[idx]} vs {fd}")
+    return out
+
+
+def grad_identities(fn, tol=1e-11):
+    """T = 1: y = v, so gv = gy and the rest vanish.  For any input: the
+    outputs are invariant to shifting k, so sum_j gk_j = 0 per row and
+    channel; and a weighted mean reproduces constants, so sum_j gv_j =
+    sum_t gy_t."""
+    out = []
+    rng = np.random.default_rng(53)
+    w, u, k, v = _rand_wkv(53, B=2, T=1, C=4)
+    gy = rng.normal(0, 1, k.shape)
+    gk, gv, gw, gu = fn(w, u, k, v, gy)
+    msg = (_close(gv, gy, tol) or _close(gk, np.zeros_like(gk), tol) or
+           _close(gw, np.zeros(4), tol) or _close(gu, np.zeros(4), tol))
+    if msg: out.append(f"gradient at T = 1: {msg}")
+    w, u, k, v = _rand_wkv(54, B=2, T=30, C=4)
+    gy = rng.normal(0, 1, k.shape)
+    gk, gv, gw, gu = fn(w, u, k, v, gy)
+    msg = _close(np.asarray(gk).sum(axis=1), np.zeros((2, 4)), tol * 30)
+    if msg: out.append(f"gradient k-shift identity: {msg}")
+    msg = _close(np.asarray(gv).sum(axis=1), gy.sum(axis=1), tol * 30)
+    if msg: out.append(f"gradient constant identity: {msg}")
+    return out
+
+
+GRAD_PINS = [grad_worked_example, grad_autodiff, grad_finite_difference, grad_identities]
+
+
+def run_grad_pins(fn):
+    fails = []
+    for pin in GRAD_PINS:
+        try:
+            fails += pin(fn)
+        except Exception as e:
+            fails.append(f"{pin.__name__} raised {type(e).__name__}: {e}")
+    return fails
+
+
+# ---------------------------------------------------------------------------
 # diagonal scan pins
 # ---------------------------------------------------------------------------
 def scan_worked_example(fn, tol=1e-12):

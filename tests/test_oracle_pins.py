@@ -444,3 +444,64 @@ def test_minlstm_workload_is_a_convex_scan():
     lo = np.minimum(np.minimum.accumulate(x.h_tilde, axis=1), 0.0)
     hi = np.maximum(np.maximum.accumulate(x.h_tilde, axis=1), 0.0)
     assert np.all(h >= lo - 1e-6) and np.all(h <= hi + 1e-6)
+
+
+
+# --- WKV gradients ---------------------------------------------------------
+@pytest.mark.parametrize("fn", [oracle.wkv_backward_direct, oracle.wkv_backward_rnn],
+                         ids=["direct", "rnn"])
+def test_wkv_gradient_oracle_passes_pins(fn):
+    assert pins.run_grad_pins(fn) == []
+
+
+def test_wkv_gradient_forms_agree_under_large_keys():
+    rng = np.random.default_rng(61)
+    B, T, C = 2, 150, 5
+    w = np.concatenate([[0.0, 1e-4, 30.0], np.exp(rng.uniform(-3, 2, C - 3))])
+    u = rng.normal(0, 2, C)
+    k = rng.normal(0, 15, (B, T, C))
+    v = rng.normal(0, 1, (B, T, C))
+    gy = rng.normal(0, 1, (B, T, C))
+    a = oracle.wkv_backward_direct(w, u, k, v, gy)
+    b = oracle.wkv_backward_rnn(w, u, k, v, gy)
+    for x, y in zip(a, b):
+        assert np.all(np.isfinite(y))
+        assert np.max(np.abs(x - y)) <= 1e-10 * max(1.0, np.abs(x).max())
+
+
+C_GRAD_MUTANTS = {
+    "R_without_P": ("R = fold * (R + P);", "R = fold * R;"),
+    "gw_sign": ("gw_c -= sc * (vj * R - R2);", "gw_c += sc * (vj * R - R2);"),
+    "diag_missing_in_gv": ("gvb[j * C] = diag + sc * P;", "gvb[j * C] = sc * P;"),
+    "Q_without_y": ("double Qn = fnew * gj * ys[j] + fold * Q;", "double Qn = fnew * gj + fold * Q;"),
+    "decay_once_more": ("double r2 = rho + w[c];", "double r2 = rho + 2.0 * w[c];"),
+}
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+@pytest.mark.parametrize("name", sorted(C_GRAD_MUTANTS))
+def test_planted_mistake_in_gradient_oracle_is_caught(name, tmp_path):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "wkv_oracle.c")).read()
+    old, new = C_GRAD_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation anchor for {name} not found"
+    mpath = tmp_path / "mut.c"
+    mpath.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-o", str(so),
+                           str(mpath), "-lm"])
+    lib = ctypes.CDLL(str(so))
+    i64, p = ctypes.c_int64, ctypes.c_void_p
+    lib.oracle_wkv_backward_rnn.argtypes = [i64, i64, i64] + [p] * 9 + [ctypes.c_int]
+    lib.oracle_wkv_backward_rnn.restype = None
+
+    def mut(w, u, k, v, gy):
+        k = np.ascontiguousarray(k, float); v = np.ascontiguousarray(v, float)
+        gy = np.ascontiguousarray(gy, float)
+        w = np.ascontiguousarray(w, float).reshape(-1); u = np.ascontiguousarray(u, float).reshape(-1)
+        B, T, C = k.shape
+        gk, gv = np.empty(k.shape), np.empty(k.shape)
+        gw, gu = np.empty(C), np.empty(C)
+        lib.oracle_wkv_backward_rnn(B, T, C, *(x.ctypes.data_as(p) for x in (w, u, k, v, gy, gk, gv, gw, gu)), 1)
+        return gk, gv, gw, gu
+
+    assert pins.run_grad_pins(mut) != []
