@@ -317,9 +317,9 @@ void oracle_wkv_backward_rnn(int64_t B, int64_t T, int64_t C,
                 for (int64_t t = 0; t < T; ++t) {
                     double kt = kb[t * C], vt = vb[t * C];
                     double x = u[c] + kt, q = p > x ? p : x;
-                    double ep = exp(p - q), ex = exp(x - q);
-                    double den = ep * d + ex;
-                    ys[t] = (ep * a + ex * vt) / den;
+                    double e_past = exp(p - q), e_cur = exp(x - q);
+                    double den = e_past * d + e_cur;
+                    ys[t] = (e_past * a + e_cur * vt) / den;
                     Ls[t] = q + log(den);
                     double pd = p - w[c], q2 = pd > kt ? pd : kt;
                     double fo = exp(pd - q2), fn = exp(kt - q2);
