@@ -209,10 +209,22 @@ class DeviceWorkload:
             self.kind = "scan"
             x = workloads.make_scan(name)
             B, T, C = x.a.shape
-            self.dtype, self.es = "f32", 4
-            self.host = {"a": x.a, "b": x.b}
+            bf = spec.dtype == "bf16"
+            self.dtype, self.es = spec.dtype, 2 if bf else 4
+            self.host = {"a": x.a_bits.view(np.int16) if bf else x.a,
+                         "b": x.b_bits.view(np.int16) if bf else x.b}
             self.outputs = {"h": (B, T, C)}
-            alg = 12 * B * T * C
+            alg = 3 * self.es * B * T * C
+        elif isinstance(spec, workloads.LruSpec):
+            self.kind = "lru"
+            x = workloads.make_lru(name)
+            B, T, C = x.u.shape[:3]
+            self.dtype, self.es = "c64", 8
+            self.host = {"u": x.u}
+            for k in ("nu_log", "theta_log", "gamma"):
+                self.consts[k] = torch.from_numpy(getattr(x, k)).to(dev)
+            self.outputs = {"x": (B, T, C, 2)}
+            alg = 16 * B * T * C + 12 * C
         elif isinstance(spec, workloads.ShiftSpec):
             self.kind = "shift"
             x = workloads.make_token_shift(name)
@@ -267,8 +279,10 @@ class DeviceWorkload:
         return t.to(self.dev)
 
     def api(self):
+        if self.kind == "lru":
+            return "lru_scan"
         if self.kind == "scan":
-            return "diag_scan"
+            return "diag_scan_bf16" if self.dtype == "bf16" else "diag_scan"
         bf = "_bf16" if self.dtype == "bf16" else ""
         if self.kind == "shift":
             return "wkv_token_shift" + bf
@@ -285,6 +299,10 @@ class DeviceWorkload:
         fn = getattr(lib, self.api())
         if self.kind == "scan":
             return fn(B, T, C, d["a"].data_ptr(), d["b"].data_ptr(), None, d["h"].data_ptr(), sh)
+        if self.kind == "lru":
+            k = self.consts
+            return fn(B, T, C, k["nu_log"].data_ptr(), k["theta_log"].data_ptr(),
+                      k["gamma"].data_ptr(), d["u"].data_ptr(), None, d["x"].data_ptr(), sh)
         if self.kind == "shift":   # last token handed on in place
             return fn(B, T, C, self.n_mix, d["x"].data_ptr(), d["xp"].data_ptr(),
                       self.consts["mu"].data_ptr(), d["out"].data_ptr(), d["xp"].data_ptr(), sh)
@@ -412,7 +430,8 @@ def e2e_leg(torch, wl, steps):
     outs = {k: torch.empty(shape, dtype=torch.int16 if wl.dtype == "bf16" else torch.float32
                            ).pin_memory() for k, shape in wl.outputs.items()}
     hp = {k: t.cpu().pin_memory() for k, t in wl.consts.items()}
-    host_api = wl.kind == "scan" or (wl.kind == "wkv" and not wl.gated and not wl.has_state)
+    host_api = (wl.kind == "scan" and wl.dtype == "f32") or \
+        (wl.kind == "wkv" and not wl.gated and not wl.has_state)
     if host_api:
         if wl.kind == "scan":
             api = "diag_scan_host"
@@ -492,6 +511,13 @@ def oracle_runner(name, max_elements=None):
         a, b = np.ascontiguousarray(a[:rows]), np.ascontiguousarray(b[:rows])
         fn = lambda: oracle.scan_rnn(a, b, None)   # noqa: E731
         return fn, rows * T * C, f"{rows} of {B} batch rows (all T={T}, D={C})"
+    if isinstance(spec, workloads.LruSpec):
+        x = workloads.make_lru(name)
+        B, T, C = x.u.shape[:3]
+        rows = B if max_elements is None else max(1, min(B, max_elements // (T * C)))
+        u = x.u_complex()[:rows]
+        fn = lambda: oracle.lru_scan(x.nu_log, x.theta_log, x.gamma, u)   # noqa: E731
+        return fn, rows * T * C, f"{rows} of {B} batch rows (all T={T}, D={C} complex)"
     if isinstance(spec, workloads.ShiftSpec):
         x = workloads.make_token_shift(name)
         B, T, C = x.x.shape
@@ -590,9 +616,12 @@ def aggregate_rate(elements_per_rank, world, ms_per_step):
 
 
 def workload_config(spec, name):
+    if isinstance(spec, workloads.LruSpec):
+        return {"workload": name, "op": "lru_scan (complex diagonal recurrence)", "B": spec.B,
+                "T": spec.T, "D": spec.D, "io": "complex64"}
     if isinstance(spec, workloads.ScanSpec):
-        return {"workload": name, "op": "diag_scan", "B": spec.B, "T": spec.T, "D": spec.D,
-                "io": "f32"}
+        return {"workload": name, "op": "diag_scan" + ("_bf16" if spec.dtype == "bf16" else "") +
+                f" ({spec.form} form)", "B": spec.B, "T": spec.T, "D": spec.D, "io": spec.dtype}
     bf = "_bf16" if spec.dtype == "bf16" else ""
     if isinstance(spec, workloads.ShiftSpec):
         return {"workload": name, "op": f"wkv_token_shift{bf} ({spec.n_mix} mixing vectors, "
@@ -608,6 +637,8 @@ def workload_config(spec, name):
 
 
 def metric_for(spec):
+    if isinstance(spec, workloads.LruSpec):
+        return "LRU scan B·T·D complex elems/s and achieved HBM GB/s vs B200 peak (1 GPU)"
     if isinstance(spec, workloads.ShiftSpec):
         return "token shift B·T·C elems/s and achieved HBM GB/s vs B200 peak (1 GPU)"
     return METRIC

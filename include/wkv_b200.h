@@ -197,6 +197,53 @@ WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,
                      const float *a, const float *b, const float *h0, float *h,
                      cudaStream_t stream);
 
+/* Gradients of the fp32 WKV forward (no state in): given gy = dL/dy [B, T, C],
+ * writes gk, gv [B, T, C] and gw, gu [C] (summed over batch rows and steps).
+ * The pages give no gradient formulas; eq. (14) of "RWKV：基于RNN的LLM" is a
+ * softmax-weighted mean of v_0..v_t with logits l_{t,j} = -(t-1-j) w + k_j
+ * (j < t) and l_{t,t} = u + k_t, weights beta_{t,j}, so
+ *     gv_j = sum_{t>=j} gy_t beta_{t,j},   gk_j = sum_{t>=j} gy_t beta_{t,j} (v_j - y_t),
+ *     gu   = sum_t gy_t beta_{t,t} (v_t - y_t),
+ *     gw   = -sum_t sum_{j<t} (t-1-j) gy_t beta_{t,j} (v_j - y_t).
+ * One thread per (row, channel) recomputes the forward pass and runs the
+ * sums over later outputs backwards in time, max-stabilised (every exponent
+ * <= 0 for finite inputs); gw and gu are reduced over rows in a fixed order.
+ * Scratch (8 bytes per element plus 8 per row and channel) is a
+ * library-owned per-stream buffer, allocated on first use like the
+ * look-back workspace (make one call of each size before stream capture).
+ * No output may overlap an input or another output.  Pointers 4-byte
+ * aligned.  B or T = 0 with C > 0 sets gw, gu to 0. */
+WKV_API wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                                const float *k, const float *v, const float *gy, float *gk,
+                                float *gv, float *gw, float *gu, cudaStream_t stream);
+
+/* The LRU's complex diagonal recurrence (review of "Resurrecting Recurrent
+ * Neural Networks for Long Sequences", linear-RNN section), per complex
+ * channel d:
+ *
+ *     x[b,t,d] = lambda_d x[b,t-1,d] + gamma_d u[b,t,d],
+ *     lambda_d = e^{-nu_d + i theta_d},  nu_d = e^{nu_log[d]},  theta_d = e^{theta_log[d]}
+ *
+ * (the page's parameterisation: |lambda| = e^{-nu} <= 1 for any nu_log), with
+ * x[b,-1,d] = x0[b,d] or 0.  u, x: [B, T, D] complex64, i.e. interleaved
+ * (re, im) float pairs, [B, T, D, 2] floats; x0: [B, D] complex64 or NULL;
+ * nu_log, theta_log, gamma: [D] float, gamma NULL = 1 (the page initialises
+ * it to sqrt(1 - |lambda|^2)).  Pointers to complex data must be 8-byte
+ * aligned (TMA path: 16-byte and D even).  lambda^n across chunk boundaries
+ * is evaluated in double precision, so phases n theta of any size stay
+ * exact; inside a chunk the state steps with single-precision lambda.  x must
+ * not overlap an input.  Errors, streams and scratch as diag_scan. */
+WKV_API wkv_status lru_scan(int64_t B, int64_t T, int64_t D, const float *nu_log,
+                            const float *theta_log, const float *gamma, const float *u,
+                            const float *x0, float *x, cudaStream_t stream);
+
+/* Diagonal linear scan with bfloat16 a, b, h (fp32 h0 [B, D] or NULL; the
+ * state is carried in fp32 and each h is rounded to nearest even).  Pointers
+ * must be 2-byte aligned (TMA path: 16-byte and D % 8 == 0). */
+WKV_API wkv_status diag_scan_bf16(int64_t B, int64_t T, int64_t D,
+                                  const wkv_bf16_t *a, const wkv_bf16_t *b, const float *h0,
+                                  wkv_bf16_t *h, cudaStream_t stream);
+
 /* WKV forward, fp32, without allocating any device memory.  The pages this
  * library follows have no counterpart of this entry point: it exists for
  * callers that cannot call cudaMalloc -- code running inside an engine that

@@ -49,6 +49,8 @@ _SIGS = {
     "wkv_token_shift": ([_i64, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_token_shift_bf16": ([_i64, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p], _i32),
     "diag_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
+    "diag_scan_bf16": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
+    "lru_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_bf16_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "diag_scan_host": ([_i64, _i64, _i64, _p, _p, _p, _p], _i32),
@@ -262,10 +264,14 @@ def wkv_forward_noalloc(w, u, k, v, y=None, stream=None):
 
 
 def diag_scan(a, b, h0=None, h=None, stream=None):
-    """h_t = a_t * h_{t-1} + b_t per channel, h_{-1} = h0 (zeros if None)."""
+    """h_t = a_t * h_{t-1} + b_t per channel, h_{-1} = h0 (zeros if None).
+    a, b, h fp32, or all bf16 (fp32 state, bf16 storage); h0 fp32."""
     import torch
-    _need(a, "a", torch.float32, 3)
-    _need(b, "b", torch.float32, 3)
+    io = a.dtype
+    if io not in (torch.float32, torch.bfloat16):
+        raise TypeError("a must be float32 or bfloat16")
+    _need(a, "a", io, 3)
+    _need(b, "b", io, 3)
     if a.shape != b.shape:
         raise ValueError("a and b must have one shape")
     B, T, D = a.shape
@@ -276,13 +282,50 @@ def diag_scan(a, b, h0=None, h=None, stream=None):
     if h is None:
         h = torch.empty_like(a)
     else:
-        _need(h, "h", torch.float32, 3)
+        _need(h, "h", io, 3)
         if h.shape != a.shape:
             raise ValueError("h must have the shape of a")
-    _check(lib.diag_scan(B, T, D, a.data_ptr(), b.data_ptr(),
-                         None if h0 is None else h0.data_ptr(), h.data_ptr(),
-                         _stream_handle(stream)), "diag_scan")
+    fn = "diag_scan" if io == torch.float32 else "diag_scan_bf16"
+    _check(getattr(lib, fn)(B, T, D, a.data_ptr(), b.data_ptr(),
+                            None if h0 is None else h0.data_ptr(), h.data_ptr(),
+                            _stream_handle(stream)), fn)
     return h
+
+
+def lru_scan(nu_log, theta_log, u, gamma=None, x0=None, x=None, stream=None):
+    """The LRU recurrence x_t = lambda x_{t-1} + gamma u_t per complex channel,
+    lambda = e^{-e^{nu_log} + i e^{theta_log}}.  u: complex64 [B, T, D] (or
+    float32 [B, T, D, 2]); nu_log, theta_log, gamma: float32 [D]; x0: complex64
+    [B, D] or None (zeros).  Returns x like u."""
+    import torch
+    as_complex = u.dtype == torch.complex64
+    ur = torch.view_as_real(u) if as_complex else u
+    _need(ur, "u", torch.float32, 4)
+    if ur.shape[-1] != 2:
+        raise ValueError("u must be complex64 [B, T, D] or float32 [B, T, D, 2]")
+    B, T, D, _ = ur.shape
+    for t, name in ((nu_log, "nu_log"), (theta_log, "theta_log"), (gamma, "gamma")):
+        if t is not None:
+            _need(t, name, torch.float32, 1)
+            if t.shape[0] != D:
+                raise ValueError(f"{name} must be [D]")
+    x0r = None
+    if x0 is not None:
+        x0r = torch.view_as_real(x0) if x0.dtype == torch.complex64 else x0
+        _need(x0r, "x0", torch.float32, 3)
+        if tuple(x0r.shape) != (B, D, 2):
+            raise ValueError("x0 must be [B, D] complex")
+    if x is None:
+        x = torch.empty_like(u)
+    xr = torch.view_as_real(x) if x.dtype == torch.complex64 else x
+    _need(xr, "x", torch.float32, 4)
+    if xr.shape != ur.shape:
+        raise ValueError("x must have the shape of u")
+    _check(lib.lru_scan(B, T, D, nu_log.data_ptr(), theta_log.data_ptr(),
+                        None if gamma is None else gamma.data_ptr(), ur.data_ptr(),
+                        None if x0r is None else x0r.data_ptr(), xr.data_ptr(),
+                        _stream_handle(stream)), "lru_scan")
+    return x
 
 
 def _need_host(t, name, dtype, ndim):
@@ -394,6 +437,7 @@ def wkv_set_fault_injection(skip_tile: int = -1, spin_limit: int = 0):
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan",
            "wkv_forward_state", "wkv_forward_bf16_state", "wkv_forward_gated", "token_shift",
+           "lru_scan",
            "wkv_forward_host", "wkv_forward_bf16_host", "diag_scan_host", "wkv_device_status",
            "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
            "wkv_get_tile_steps", "wkv_tile_steps_for", "WkvError", "lib", "LIB_PATH"]

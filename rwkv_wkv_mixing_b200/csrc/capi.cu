@@ -16,8 +16,10 @@
 #include <vector>
 
 #include "chunked_scan.cuh"
+#include "lru_ops.cuh"
 #include "persistent_scan.cuh"
 #include "serial_wkv.cuh"
+#include "wkv_backward.cuh"
 #include "token_shift.cuh"
 #include "wkv_b200.h"
 #include "wkv_ops.cuh"
@@ -144,6 +146,7 @@ wkv_status check_sizes(int64_t B, int64_t T, int64_t C, bool *empty) {
 struct WsEntry {
     int device = -1;
     cudaStream_t stream = nullptr;
+    int kind = 0;  // 0: look-back workspace; 1: gradient scratch
     char *base = nullptr;
     size_t bytes = 0;
 };
@@ -162,15 +165,15 @@ size_t ws_bytes(size_t tiles, size_t channels_per_tile) {
     return round_up(kWsHeader + tiles * channels_per_tile * sizeof(uint4), 256);
 }
 
-WsEntry *find_ws(int dev, cudaStream_t stream) {
+WsEntry *find_ws(int dev, cudaStream_t stream, int kind = 0) {
     for (WsEntry *e : g_ws)
-        if (e->device == dev && e->stream == stream) return e;
+        if (e->device == dev && e->stream == stream && e->kind == kind) return e;
     return nullptr;
 }
 
 // caller holds g_mu
-wkv_status ensure_ws(int dev, cudaStream_t stream, size_t need, WsEntry **out) {
-    WsEntry *e = find_ws(dev, stream);
+wkv_status ensure_ws(int dev, cudaStream_t stream, size_t need, WsEntry **out, int kind = 0) {
+    WsEntry *e = find_ws(dev, stream, kind);
     if (e != nullptr && e->bytes >= need) {
         *out = e;
         return WKV_OK;
@@ -198,6 +201,7 @@ wkv_status ensure_ws(int dev, cudaStream_t stream, size_t need, WsEntry **out) {
         e = new WsEntry;
         e->device = dev;
         e->stream = stream;
+        e->kind = kind;
         g_ws.push_back(e);
     } else if (e->base != nullptr) {
         g_retired.emplace_back(dev, e->base);
@@ -281,12 +285,21 @@ wkv_status make_plan(const typename Op::Args &args, int64_t B, int64_t T, int64_
     std::memset(p->maps, 0, sizeof p->maps);
     g.use_tma = 0;
     if (want_tma) {
-        const void *ptrs[4] = {args.x0, args.x1, args.y, nullptr};
-        int n = 3;
-        if constexpr (Op::NIN == 3) ptrs[n++] = args.x2;
-        g.use_tma = tma_eligible(ptrs, n, sizeof(io_t), T, C) ? 1 : 0;
-        for (int i = 0; i < n && g.use_tma; ++i)
-            if (!make_map(&p->maps[i], ptrs[i], dt, sizeof(io_t), B, T, C, CG, lt)) g.use_tma = 0;
+        // maps: [0] x0, [1] x1 (two or more inputs), [2] y, [3] x2 (three inputs);
+        // an io element is kScalarsPerIo tensor-map elements
+        const void *ptrs[4] = {args.x0, nullptr, args.y, nullptr};
+        if constexpr (Op::NIN >= 2) ptrs[1] = args.x1;
+        if constexpr (Op::NIN == 3) ptrs[3] = args.x2;
+        const void *used[4];
+        int n = 0;
+        for (const void *q : ptrs)
+            if (q != nullptr) used[n++] = q;
+        constexpr int SP = Op::kScalarsPerIo;
+        g.use_tma = tma_eligible(used, n, sizeof(io_t), T, C) ? 1 : 0;
+        for (int i = 0; i < 4 && g.use_tma; ++i)
+            if (ptrs[i] != nullptr &&
+                !make_map(&p->maps[i], ptrs[i], dt, sizeof(io_t) / SP, B, T, C * SP, CG * SP, lt))
+                g.use_tma = 0;
     }
     std::memset(&p->ws, 0, sizeof p->ws);
     if (g.n_seg > 1) {
@@ -417,8 +430,9 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
         if (T <= kSerialMaxSteps && (B * C + kSerialThreads - 1) / kSerialThreads <= INT32_MAX)
             return launch_serial<Op>(args, B, T, C, stream);
     }
-    const void *ptrs[4] = {args.x0, args.x1, args.y, nullptr};
-    int nptr = 3;
+    const void *ptrs[4] = {args.x0, args.y, nullptr, nullptr};
+    int nptr = 2;
+    if constexpr (Op::NIN >= 2) ptrs[nptr++] = args.x1;
     if constexpr (Op::NIN == 3) ptrs[nptr++] = args.x2;
     const bool tma = tma_eligible(ptrs, nptr, sizeof(typename Op::io_t), T, C);
     const int lt = tile_steps_for(B, T, C, 32 * Op::CPT);
@@ -564,6 +578,28 @@ wkv_status shift_common(int64_t B, int64_t T, int64_t C, int64_t n_mix, const IO
     const int nm = static_cast<int>(n_mix);
     return vec4 ? launch_shift<IO, 4>(nm, x, x_prev, mu, out, x_last, B, T, C, stream)
                 : launch_shift<IO, 1>(nm, x, x_prev, mu, out, x_last, B, T, C, stream);
+}
+
+template <typename IO>
+wkv_status scan_common(int64_t B, int64_t T, int64_t D, const IO *a, const IO *b,
+                       const float *h0, IO *h, cudaStream_t stream, CUtensorMapDataType dt) {
+    t_err.clear();
+    bool empty = false;
+    wkv_status st = check_sizes(B, T, D, &empty);
+    if (st != WKV_OK || empty) return st;
+    int dev = 0;
+    if ((st = current_device(&dev)) != WKV_OK) return st;
+    const size_t n = static_cast<size_t>(B) * T * D * sizeof(IO);
+    const size_t n0 = static_cast<size_t>(B) * D * sizeof(float);
+    if ((st = check_buffer(a, n, sizeof(IO), "a", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(b, n, sizeof(IO), "b", dev)) != WKV_OK) return st;
+    if (h0 != nullptr && (st = check_buffer(h0, n0, 4, "h0", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(h, n, sizeof(IO), "h", dev)) != WKV_OK) return st;
+    if (overlaps(h, n, a, n) || overlaps(h, n, b, n) || overlaps(h, n, h0, h0 ? n0 : 0))
+        return fail(WKV_ERR_INVALID_ARG, "h overlaps an input");
+    using Op = ScanOpT<IO, sizeof(IO) == 2 ? 2 : 1>;
+    typename Op::Args args{a, b, h, h0};
+    return dispatch<Op>(args, B, T, D, dt, stream, dev);
 }
 
 // ---- host-buffer entry points: a chunked copy / compute pipeline ------------
@@ -890,24 +926,110 @@ wkv_status wkv_token_shift_bf16(int64_t B, int64_t T, int64_t C, int64_t n_mix,
                             reinterpret_cast<bf *>(x_last), stream);
 }
 
-wkv_status diag_scan(int64_t B, int64_t T, int64_t D, const float *a, const float *b,
-                     const float *h0, float *h, cudaStream_t stream) {
+wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                        const float *k, const float *v, const float *gy, float *gk, float *gv,
+                        float *gw, float *gu, cudaStream_t stream) {
+    t_err.clear();
+    bool empty = false;
+    wkv_status st = check_sizes(B, T, C, &empty);
+    if (st != WKV_OK) return st;
+    if (empty) {
+        if (B == 0 || T == 0) {  // no outputs: gw, gu are empty sums (C may be > 0)
+            if (C > 0) {
+                int dev0 = 0;
+                if ((st = current_device(&dev0)) != WKV_OK) return st;
+                const size_t nc0 = static_cast<size_t>(C) * sizeof(float);
+                if ((st = check_buffer(gw, nc0, 4, "gw", dev0)) != WKV_OK) return st;
+                if ((st = check_buffer(gu, nc0, 4, "gu", dev0)) != WKV_OK) return st;
+                cudaError_t e = cudaMemsetAsync(gw, 0, nc0, stream);
+                if (e == cudaSuccess) e = cudaMemsetAsync(gu, 0, nc0, stream);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(gw, gu)");
+            }
+        }
+        return WKV_OK;
+    }
+    int dev = 0;
+    if ((st = current_device(&dev)) != WKV_OK) return st;
+    const size_t n = static_cast<size_t>(B) * T * C * sizeof(float);
+    const size_t nc = static_cast<size_t>(C) * sizeof(float);
+    const struct { const void *p; size_t bytes; const char *name; } in[] = {
+        {w, nc, "w"}, {u, nc, "u"}, {k, n, "k"}, {v, n, "v"}, {gy, n, "gy"}};
+    const struct { const void *p; size_t bytes; const char *name; } out[] = {
+        {gk, n, "gk"}, {gv, n, "gv"}, {gw, nc, "gw"}, {gu, nc, "gu"}};
+    for (const auto &x : in)
+        if ((st = check_buffer(x.p, x.bytes, 4, x.name, dev)) != WKV_OK) return st;
+    for (const auto &x : out)
+        if ((st = check_buffer(x.p, x.bytes, 4, x.name, dev)) != WKV_OK) return st;
+    for (size_t i = 0; i < 4; ++i) {
+        for (const auto &x : in)
+            if (overlaps(out[i].p, out[i].bytes, x.p, x.bytes))
+                return fail(WKV_ERR_INVALID_ARG, "%s overlaps input %s", out[i].name, x.name);
+        for (size_t j = i + 1; j < 4; ++j)
+            if (overlaps(out[i].p, out[i].bytes, out[j].p, out[j].bytes))
+                return fail(WKV_ERR_INVALID_ARG, "%s overlaps %s", out[i].name, out[j].name);
+    }
+    const int64_t blocks = (B * C + kBwdThreads - 1) / kBwdThreads;
+    if (blocks > INT32_MAX) return fail(WKV_ERR_INVALID_ARG, "B*C too large for one launch");
+    // scratch: y_t, ln D_t per element and per-row gw, gu partials
+    const size_t need = 2 * n + static_cast<size_t>(B) * 2 * C * sizeof(float);
+    WsEntry *e = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if ((st = ensure_ws(dev, stream, need, &e, 1)) != WKV_OK) return st;
+    }
+    float *scratch = reinterpret_cast<float *>(e->base);
+    const size_t ne = static_cast<size_t>(B) * T * C;
+    WkvBwdArgs a{w, u, k, v, gy, gk, gv, scratch, scratch + ne, scratch + 2 * ne, gw, gu};
+    wkv_backward_serial_kernel<<<static_cast<unsigned>(blocks), kBwdThreads, 0, stream>>>(
+        a, static_cast<int>(B), static_cast<int>(T), static_cast<int>(C));
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    wkv_backward_reduce_kernel<<<static_cast<unsigned>((C + kBwdThreads - 1) / kBwdThreads),
+                                 kBwdThreads, 0, stream>>>(a, static_cast<int>(B),
+                                                           static_cast<int>(C));
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
+wkv_status lru_scan(int64_t B, int64_t T, int64_t D, const float *nu_log,
+                    const float *theta_log, const float *gamma, const float *u,
+                    const float *x0, float *x, cudaStream_t stream) {
     t_err.clear();
     bool empty = false;
     wkv_status st = check_sizes(B, T, D, &empty);
     if (st != WKV_OK || empty) return st;
     int dev = 0;
     if ((st = current_device(&dev)) != WKV_OK) return st;
-    const size_t n = static_cast<size_t>(B) * T * D * sizeof(float);
-    const size_t n0 = static_cast<size_t>(B) * D * sizeof(float);
-    if ((st = check_buffer(a, n, 4, "a", dev)) != WKV_OK) return st;
-    if ((st = check_buffer(b, n, 4, "b", dev)) != WKV_OK) return st;
-    if (h0 != nullptr && (st = check_buffer(h0, n0, 4, "h0", dev)) != WKV_OK) return st;
-    if ((st = check_buffer(h, n, 4, "h", dev)) != WKV_OK) return st;
-    if (overlaps(h, n, a, n) || overlaps(h, n, b, n) || overlaps(h, n, h0, h0 ? n0 : 0))
-        return fail(WKV_ERR_INVALID_ARG, "h overlaps an input");
-    ScanOp::Args args{a, b, h, h0};
-    return dispatch<ScanOp>(args, B, T, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, stream, dev);
+    const size_t n = static_cast<size_t>(B) * T * D * 8;   // complex64 elements
+    const size_t n0 = static_cast<size_t>(B) * D * 8;
+    const size_t nd = static_cast<size_t>(D) * 4;
+    if ((st = check_buffer(nu_log, nd, 4, "nu_log", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(theta_log, nd, 4, "theta_log", dev)) != WKV_OK) return st;
+    if (gamma != nullptr && (st = check_buffer(gamma, nd, 4, "gamma", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(u, n, 8, "u", dev)) != WKV_OK) return st;
+    if (x0 != nullptr && (st = check_buffer(x0, n0, 8, "x0", dev)) != WKV_OK) return st;
+    if ((st = check_buffer(x, n, 8, "x", dev)) != WKV_OK) return st;
+    if (overlaps(x, n, u, n) || overlaps(x, n, x0, x0 ? n0 : 0) || overlaps(x, n, nu_log, nd) ||
+        overlaps(x, n, theta_log, nd) || overlaps(x, n, gamma, gamma ? nd : 0))
+        return fail(WKV_ERR_INVALID_ARG, "x overlaps an input");
+    LruOp::Args args{reinterpret_cast<const float2 *>(u), nullptr, reinterpret_cast<float2 *>(x),
+                     nu_log, theta_log, gamma, reinterpret_cast<const float2 *>(x0)};
+    return dispatch<LruOp>(args, B, T, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, stream, dev);
+}
+
+wkv_status diag_scan(int64_t B, int64_t T, int64_t D, const float *a, const float *b,
+                     const float *h0, float *h, cudaStream_t stream) {
+    return scan_common<float>(B, T, D, a, b, h0, h, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+}
+
+wkv_status diag_scan_bf16(int64_t B, int64_t T, int64_t D, const wkv_bf16_t *a,
+                          const wkv_bf16_t *b, const float *h0, wkv_bf16_t *h,
+                          cudaStream_t stream) {
+    using bf = __nv_bfloat16;
+    return scan_common<bf>(B, T, D, reinterpret_cast<const bf *>(a),
+                           reinterpret_cast<const bf *>(b), h0, reinterpret_cast<bf *>(h), stream,
+                           CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
 wkv_status wkv_device_status(cudaStream_t stream) {

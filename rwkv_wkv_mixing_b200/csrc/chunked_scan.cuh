@@ -1,7 +1,7 @@
 // Chunked two-pass time scan over [B, T, C] tensors for sm_100a.
 //
 // One thread block owns one tile: CG consecutive channels x LT consecutive
-// steps of one batch row.  The tile's two input tensors are staged in shared
+// steps of one batch row.  The tile's input tensors (NIN of them) are staged in shared
 // memory once (TMA tile copies, or element-wise copies when the tensor cannot
 // be described by a tensor map), so HBM sees every input element once and
 // every output element once.
@@ -59,8 +59,8 @@ __global__ void __launch_bounds__(NW * 32, 3)
 
     extern __shared__ __align__(128) unsigned char smem[];
     io_t *s_x0 = reinterpret_cast<io_t *>(smem);            // [LT][CG], outputs overwrite it
-    io_t *s_x1 = s_x0 + LT * CG;                            // [LT][CG]
-    io_t *s_x2 = s_x1 + (Op::NIN == 3 ? LT * CG : 0);       // [LT][CG] r, when NIN == 3
+    io_t *s_x1 = s_x0 + (Op::NIN >= 2 ? LT * CG : 0);       // [LT][CG], when NIN >= 2
+    io_t *s_x2 = s_x0 + (Op::NIN == 3 ? 2 * LT * CG : 0);   // [LT][CG] r, when NIN == 3
     float *s_sum = reinterpret_cast<float *>(s_x0 + Op::NIN * LT * CG);  // [NW][NV][CG]
     float *s_carry = s_sum + NW * NV * CG;                   // [NV][CG]
     __shared__ __align__(8) uint64_t s_bar;
@@ -109,9 +109,9 @@ __global__ void __launch_bounds__(NW * 32, 3)
         if (tid == 0) {
             mbar_arrive_expect_tx(&s_bar,
                                   static_cast<uint32_t>(Op::NIN * LT * CG * sizeof(io_t)));
-            tma_load_3d(s_x0, &map_x0, &s_bar, c0, t0, b);
-            tma_load_3d(s_x1, &map_x1, &s_bar, c0, t0, b);
-            if constexpr (Op::NIN == 3) tma_load_3d(s_x2, &map_x2, &s_bar, c0, t0, b);
+            tma_load_3d(s_x0, &map_x0, &s_bar, c0 * Op::kScalarsPerIo, t0, b);
+            if constexpr (Op::NIN >= 2) tma_load_3d(s_x1, &map_x1, &s_bar, c0 * Op::kScalarsPerIo, t0, b);
+            if constexpr (Op::NIN == 3) tma_load_3d(s_x2, &map_x2, &s_bar, c0 * Op::kScalarsPerIo, t0, b);
         }
     } else {
         for (int i = tid; i < LT * CG; i += NW * 32) {
@@ -121,11 +121,11 @@ __global__ void __launch_bounds__(NW * 32, 3)
             if (t < g.T && c < g.C) {
                 const size_t o = (static_cast<size_t>(b) * g.T + t) * g.C + c;
                 a = args.x0[o];
-                bb = args.x1[o];
+                if constexpr (Op::NIN >= 2) bb = args.x1[o];
                 if constexpr (Op::NIN == 3) rr = args.x2[o];
             }
             s_x0[i] = a;
-            s_x1[i] = bb;
+            if constexpr (Op::NIN >= 2) s_x1[i] = bb;
             if constexpr (Op::NIN == 3) s_x2[i] = rr;
         }
     }
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(NW * 32, 3)
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
-            tma_store_3d(&map_y, s_x0, c0, t0, b);  // rows >= T, channels >= C are clipped
+            tma_store_3d(&map_y, s_x0, c0 * Op::kScalarsPerIo, t0, b);  // rows >= T, channels >= C are clipped
             bulk_commit();
             bulk_wait_read_all();
         }

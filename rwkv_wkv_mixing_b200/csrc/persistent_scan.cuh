@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
         // ---------------- producer ----------------
         if (lane == 0) {
             prefetch_tensormap(&map_x0);
-            prefetch_tensormap(&map_x1);
+            if constexpr (Op::NIN >= 2) prefetch_tensormap(&map_x1);
             prefetch_tensormap(&map_y);
             if constexpr (Op::NIN == 3) prefetch_tensormap(&map_x2);
             int sentinels = 0;
@@ -185,11 +185,12 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                     io_t *dst = s_stage + static_cast<size_t>(s) * Op::NIN * Cfg::kTileElems;
                     s_last_it[s] = it;
                     mbar_arrive_expect_tx(&full_bar[s], static_cast<uint32_t>(Cfg::kStageBytes));
-                    tma_load_3d(dst, &map_x0, &full_bar[s], c0, seg * LT, b);
-                    tma_load_3d(dst + Cfg::kTileElems, &map_x1, &full_bar[s], c0, seg * LT, b);
+                    tma_load_3d(dst, &map_x0, &full_bar[s], c0 * Op::kScalarsPerIo, seg * LT, b);
+                    if constexpr (Op::NIN >= 2)
+                        tma_load_3d(dst + Cfg::kTileElems, &map_x1, &full_bar[s], c0 * Op::kScalarsPerIo, seg * LT, b);
                     if constexpr (Op::NIN == 3)
-                        tma_load_3d(dst + 2 * Cfg::kTileElems, &map_x2, &full_bar[s], c0,
-                                    seg * LT, b);
+                        tma_load_3d(dst + 2 * Cfg::kTileElems, &map_x2, &full_bar[s],
+                                    c0 * Op::kScalarsPerIo, seg * LT, b);
                 }
             }
         }
@@ -230,9 +231,10 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             const int t0 = seg * LT;
             const int c0 = (rem - b * g.n_cg) * CG;
             io_t *s_x0 = s_stage + static_cast<size_t>(s) * Op::NIN * Cfg::kTileElems;
-            const io_t *s_x1 = s_x0 + Cfg::kTileElems;
+            // the second input, when there is one; never read otherwise
+            const io_t *s_x1 = Op::NIN >= 2 ? s_x0 + Cfg::kTileElems : s_x0;
             // the third input (r) when there is one; never read otherwise
-            const io_t *s_x2 = Op::NIN == 3 ? s_x1 + Cfg::kTileElems : s_x1;
+            const io_t *s_x2 = Op::NIN == 3 ? s_x0 + 2 * Cfg::kTileElems : s_x1;
 
             Param prm[CPT];
 #pragma unroll
@@ -349,7 +351,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             // store the tile (rows >= T and channels >= C are clipped), then
             // hand the stage back once the store has read it
             if (gtid == 0) {
-                tma_store_3d(&map_y, s_x0, c0, t0, b);
+                tma_store_3d(&map_y, s_x0, c0 * Op::kScalarsPerIo, t0, b);
                 bulk_commit();
                 bulk_wait_read_all();
                 mbar_arrive(&empty_bar[s]);

@@ -58,6 +58,8 @@ __device__ __forceinline__ io_t io_zero();
 template <>
 __device__ __forceinline__ float io_zero<float>() { return 0.f; }
 template <>
+__device__ __forceinline__ float2 io_zero<float2>() { return make_float2(0.f, 0.f); }
+template <>
 __device__ __forceinline__ __nv_bfloat16 io_zero<__nv_bfloat16>() {
     return __float2bfloat16_rn(0.f);
 }

@@ -161,6 +161,7 @@ struct WkvOp {
     static constexpr int CG = 32 * CPT;
     static constexpr int NV = 3;
     static constexpr int NIN = GATED ? 3 : 2;  // input tensors per tile: k, v (, r)
+    static constexpr int kScalarsPerIo = 1;    // tensor-map elements per io_t
     static constexpr bool kGated = GATED;
     static constexpr bool kSerialForm = true;  // has the per-step form of serial_wkv.cuh
     struct Param {
@@ -525,12 +526,14 @@ struct WkvOp {
 // state produced from h = 0); the state h followed by a chunk (A, H) is
 // A h + H.
 // ---------------------------------------------------------------------------
-struct ScanOp {
-    using io_t = float;
-    static constexpr int CPT = 1;
-    static constexpr int CG = 32;
+template <typename IO, int CPT_>
+struct ScanOpT {
+    using io_t = IO;
+    static constexpr int CPT = CPT_;
+    static constexpr int CG = 32 * CPT;
     static constexpr int NV = 2;
     static constexpr int NIN = 2;
+    static constexpr int kScalarsPerIo = 1;
     static constexpr bool kGated = false;
     static constexpr bool kSerialForm = false;
     struct Param {};
@@ -538,10 +541,10 @@ struct ScanOp {
         float A, H;
     };
     struct Args {
-        const float *x0;  // a [B, T, D]
-        const float *x1;  // b [B, T, D]
-        float *y;         // h [B, T, D]
-        const float *h0;  // [B, D] or nullptr
+        const IO *x0;     // a [B, T, D]
+        const IO *x1;     // b [B, T, D]
+        IO *y;            // h [B, T, D]
+        const float *h0;  // [B, D] fp32, or nullptr
     };
     struct Scratch {};
 
@@ -572,46 +575,76 @@ struct ScanOp {
     }
 
     template <int LS>
-    __device__ __forceinline__ static void summarize(const float *p0, const float *p1, int n,
-                                                     const Param (&)[1], State (&out)[1],
-                                                     Scratch (&)[1]) {
-        float A = 1.f, H = 0.f;
-        if (n == LS) {
+    __device__ __forceinline__ static void summarize(const IO *p0, const IO *p1, int n,
+                                                     const Param (&)[CPT], State (&out)[CPT],
+                                                     Scratch (&)[CPT]) {
+        float A[CPT], H[CPT];
 #pragma unroll
-            for (int i = 0; i < LS; ++i) {
-                const float a = p0[i * CG], b = p1[i * CG];
-                H = fmaf(a, H, b);
-                A *= a;
-            }
-        } else {
-            for (int i = 0; i < n; ++i) {
-                const float a = p0[i * CG], b = p1[i * CG];
-                H = fmaf(a, H, b);
-                A *= a;
-            }
+        for (int j = 0; j < CPT; ++j) {
+            A[j] = 1.f;
+            H[j] = 0.f;
         }
-        out[0] = {A, H};
-    }
-
-    template <int LS>
-    __device__ __forceinline__ static void sweep(const State (&carry)[1], const float *p0,
-                                                 const float *p1, const float *, int n,
-                                                 const Param (&)[1], const Scratch (&)[1],
-                                                 float *out, size_t ostride, bool valid) {
-        float H = carry[0].H;
         if (n == LS) {
 #pragma unroll 8
             for (int i = 0; i < LS; ++i) {
-                H = fmaf(p0[i * CG], H, p1[i * CG]);
-                if (valid) out[i * ostride] = H;
+                float a[CPT], b[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, a);
+                Vec<IO, CPT>::load(p1 + i * CG, b);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    H[j] = fmaf(a[j], H[j], b[j]);
+                    A[j] *= a[j];
+                }
             }
         } else {
             for (int i = 0; i < n; ++i) {
-                H = fmaf(p0[i * CG], H, p1[i * CG]);
-                if (valid) out[i * ostride] = H;
+                float a[CPT], b[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, a);
+                Vec<IO, CPT>::load(p1 + i * CG, b);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    H[j] = fmaf(a[j], H[j], b[j]);
+                    A[j] *= a[j];
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) out[j] = {A[j], H[j]};
+    }
+
+    template <int LS>
+    __device__ __forceinline__ static void sweep(const State (&carry)[CPT], const IO *p0,
+                                                 const IO *p1, const IO *, int n,
+                                                 const Param (&)[CPT], const Scratch (&)[CPT],
+                                                 IO *out, size_t ostride, bool valid) {
+        float H[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) H[j] = carry[j].H;
+        if (n == LS) {
+#pragma unroll 8
+            for (int i = 0; i < LS; ++i) {
+                float a[CPT], b[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, a);
+                Vec<IO, CPT>::load(p1 + i * CG, b);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) H[j] = fmaf(a[j], H[j], b[j]);
+                if (valid) Vec<IO, CPT>::store(out + i * ostride, H);
+            }
+        } else {
+            for (int i = 0; i < n; ++i) {
+                float a[CPT], b[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, a);
+                Vec<IO, CPT>::load(p1 + i * CG, b);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) H[j] = fmaf(a[j], H[j], b[j]);
+                if (valid) Vec<IO, CPT>::store(out + i * ostride, H);
             }
         }
     }
 };
+
+// fp32 I/O, one channel per thread; bf16 I/O, two (128-byte tile rows either way)
+using ScanOp = ScanOpT<float, 1>;
+using ScanOpBf16 = ScanOpT<__nv_bfloat16, 2>;
 
 }  // namespace wkvb
