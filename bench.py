@@ -256,6 +256,11 @@ class DeviceWorkload:
             self.outputs = {"y": (B, T, C)}
             alg = self.es * B * T * C * (4 if self.gated else 3) + 8 * C + \
                 (24 * B * C if self.has_state else 0)
+            if x.gy is not None:   # gradients: read k, v, gy; write gk, gv (and gw, gu)
+                self.kind = "bwd"
+                self.host["gy"] = x.gy
+                self.outputs = {"gk": (B, T, C), "gv": (B, T, C), "gw": (C,), "gu": (C,)}
+                alg = 20 * B * T * C + 16 * C
         self.inputs = x
         self.B, self.T, self.C = B, T, C
         self.elements = B * T * C
@@ -279,6 +284,8 @@ class DeviceWorkload:
         return t.to(self.dev)
 
     def api(self):
+        if self.kind == "bwd":
+            return "wkv_backward"
         if self.kind == "lru":
             return "lru_scan"
         if self.kind == "scan":
@@ -307,6 +314,10 @@ class DeviceWorkload:
             return fn(B, T, C, self.n_mix, d["x"].data_ptr(), d["xp"].data_ptr(),
                       self.consts["mu"].data_ptr(), d["out"].data_ptr(), d["xp"].data_ptr(), sh)
         w, u = self.consts["w"].data_ptr(), self.consts["u"].data_ptr()
+        if self.kind == "bwd":
+            return fn(B, T, C, w, u, d["k"].data_ptr(), d["v"].data_ptr(), d["gy"].data_ptr(),
+                      d["gk"].data_ptr(), d["gv"].data_ptr(), d["gw"].data_ptr(),
+                      d["gu"].data_ptr(), sh)
         s = d["s"].data_ptr() if self.has_state else None   # state updated in place
         if self.gated:
             return fn(B, T, C, w, u, d["k"].data_ptr(), d["v"].data_ptr(), d["r"].data_ptr(),
@@ -320,6 +331,8 @@ class DeviceWorkload:
         """The kernel a step launches (the library's dispatch rule)."""
         if self.kind == "shift":
             return "token_shift_kernel"
+        if self.kind == "bwd":
+            return "wkv_backward_serial_kernel"
         if self.kind == "wkv" and self.T <= 16:
             return "wkv_serial_kernel"
         if self.lib.wkv_tile_steps_for(self.B, self.T, self.C, self.es) in (8, 32):
@@ -540,7 +553,10 @@ def oracle_runner(name, max_elements=None):
     w, u = w[:chans], u[:chans]
     s_in = None if x.s_in is None else \
         np.ascontiguousarray(x.s_in[:rows, :, :chans], dtype=np.float64)
-    if x.r is not None:
+    if x.gy is not None:
+        gy = np.ascontiguousarray(x.gy[:rows, :, :chans], dtype=np.float64)
+        fn = lambda: oracle.wkv_backward_rnn(w, u, k, v, gy)   # noqa: E731
+    elif x.r is not None:
         r = np.ascontiguousarray(x.r[:rows, :, :chans], dtype=np.float64)
         fn = lambda: oracle.wkv_gated(w, u, k, v, r, s_in)   # noqa: E731
     elif s_in is not None:
@@ -627,7 +643,9 @@ def workload_config(spec, name):
         return {"workload": name, "op": f"wkv_token_shift{bf} ({spec.n_mix} mixing vectors, "
                 "last token read and written in place)", "B": spec.B, "T": spec.T, "C": spec.C,
                 "io": spec.dtype}
-    if spec.gated:
+    if spec.backward:
+        op = "wkv_backward (gk, gv, gw, gu for an upstream gradient)"
+    elif spec.gated:
         op = f"wkv_forward{bf}_gated (sigma(r) * wkv in one pass)"
     elif spec.state:
         op = f"wkv_forward{bf}_state (state [B,3,C] fp32 read and written in place)"
@@ -637,6 +655,8 @@ def workload_config(spec, name):
 
 
 def metric_for(spec):
+    if isinstance(spec, workloads.WkvSpec) and spec.backward:
+        return "WKV backward B·T·C elems/s and achieved HBM GB/s vs B200 peak (1 GPU)"
     if isinstance(spec, workloads.LruSpec):
         return "LRU scan B·T·D complex elems/s and achieved HBM GB/s vs B200 peak (1 GPU)"
     if isinstance(spec, workloads.ShiftSpec):

@@ -51,6 +51,7 @@ _SIGS = {
     "diag_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "diag_scan_bf16": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "lru_scan": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p], _i32),
+    "wkv_backward": ([_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "wkv_forward_bf16_host": ([_i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
     "diag_scan_host": ([_i64, _i64, _i64, _p, _p, _p, _p], _i32),
@@ -292,6 +293,27 @@ def diag_scan(a, b, h0=None, h=None, stream=None):
     return h
 
 
+def wkv_backward(w, u, k, v, gy, stream=None):
+    """Gradients of wkv_forward (fp32, no state) for upstream gradient gy:
+    returns (gk, gv, gw, gu), gw and gu summed over batch rows and steps."""
+    import torch
+    for t, name in ((k, "k"), (v, "v"), (gy, "gy")):
+        _need(t, name, torch.float32, 3)
+    _need(w, "w", torch.float32, 1)
+    _need(u, "u", torch.float32, 1)
+    if k.shape != v.shape or k.shape != gy.shape:
+        raise ValueError("k, v and gy must have one shape")
+    B, T, C = k.shape
+    if w.shape[0] != C or u.shape[0] != C:
+        raise ValueError("w and u must be [C]")
+    gk, gv = torch.empty_like(k), torch.empty_like(k)
+    gw, gu = torch.empty_like(w), torch.empty_like(u)
+    _check(lib.wkv_backward(B, T, C, w.data_ptr(), u.data_ptr(), k.data_ptr(), v.data_ptr(),
+                            gy.data_ptr(), gk.data_ptr(), gv.data_ptr(), gw.data_ptr(),
+                            gu.data_ptr(), _stream_handle(stream)), "wkv_backward")
+    return gk, gv, gw, gu
+
+
 def lru_scan(nu_log, theta_log, u, gamma=None, x0=None, x=None, stream=None):
     """The LRU recurrence x_t = lambda x_{t-1} + gamma u_t per complex channel,
     lambda = e^{-e^{nu_log} + i e^{theta_log}}.  u: complex64 [B, T, D] (or
@@ -437,7 +459,7 @@ def wkv_set_fault_injection(skip_tile: int = -1, spin_limit: int = 0):
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_noalloc", "diag_scan",
            "wkv_forward_state", "wkv_forward_bf16_state", "wkv_forward_gated", "token_shift",
-           "lru_scan",
+           "lru_scan", "wkv_backward",
            "wkv_forward_host", "wkv_forward_bf16_host", "diag_scan_host", "wkv_device_status",
            "wkv_last_error", "wkv_release_workspaces", "wkv_set_tile_steps",
            "wkv_get_tile_steps", "wkv_tile_steps_for", "WkvError", "lib", "LIB_PATH"]

@@ -1,0 +1,129 @@
+"""WKV gradients on the GPU through the C ABI against the float64 oracle
+(the recurrence form, itself pinned to the definition, autodiff and central
+differences).
+
+Tolerance: each gradient array within 1e-4 of its own largest magnitude
+(fp32 sums over up to T terms of a softmax-weighted mean); gw and gu, sums
+over B T terms, within 2e-4 (1e-3 for keys of N(0, 15)).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def m(cuda_dev):
+    import rwkv_wkv_mixing_b200 as mod
+    return mod
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to("cuda")
+
+
+def check(got, want, rel, what):
+    got = np.asarray(got, np.float64)
+    scale = max(float(np.abs(want).max()), 1e-30)
+    err = np.abs(got - want)
+    i = int(np.argmax(err))
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    assert err.flat[i] <= rel * scale, (f"{what}: max err {err.flat[i]:.3e} > {rel * scale:.3e} "
+                                        f"at {i} (got {got.flat[i]!r}, want {want.flat[i]!r})")
+
+
+def run(m, x, gy):
+    out = m.wkv_backward(dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(gy))
+    torch.cuda.synchronize()
+    return [t.double().cpu().numpy() for t in out]
+
+
+def compare(m, x, gy, what, sums_rel=2e-4):
+    got = run(m, x, gy)
+    want = oracle.wkv_backward_rnn(x.w, x.u, x.k, x.v, gy.astype(np.float32))
+    for name, g, wv, rel in zip(("gk", "gv", "gw", "gu"), got, want,
+                                (1e-4, 1e-4, sums_rel, sums_rel)):
+        check(g, wv, rel, f"{what} {name}")
+
+
+SHAPES = [(1, 1, 4), (2, 5, 32), (2, 64, 40), (3, 300, 33), (1, 1024, 64), (4, 700, 130)]
+
+
+@pytest.mark.parametrize("B,T,C", SHAPES)
+def test_backward_vs_oracle(m, B, T, C):
+    x = workloads.make_wkv("wkv_169m", B=B, T=T, C=C, seed=B * 7 + T + C)
+    gy = np.random.default_rng(T + C).normal(0, 1, x.k.shape).astype(np.float32)
+    compare(m, x, gy, f"backward {B}x{T}x{C}")
+
+
+def test_backward_small_vs_definition(m):
+    """Against the O(T^2) definition form directly."""
+    x = workloads.make_wkv("wkv_tiny", B=2, T=64, C=16, seed=3)
+    gy = np.random.default_rng(3).normal(0, 1, x.k.shape).astype(np.float32)
+    got = run(m, x, gy)
+    want = oracle.wkv_backward_direct(x.w, x.u, x.k, x.v, gy)
+    for name, g, wv in zip(("gk", "gv", "gw", "gu"), got, want):
+        check(g, wv, 1e-4, f"definition {name}")
+
+
+def test_backward_long_keys(m):
+    """wkv_long's distributions (k ~ N(0,3), slow decays) over 4096 steps."""
+    x = workloads.make_wkv("wkv_long", B=1, T=4096, C=64, seed=5)
+    gy = np.random.default_rng(5).normal(0, 1, x.k.shape).astype(np.float32)
+    compare(m, x, gy, "backward long keys")
+
+
+def test_backward_extreme_values(m):
+    rng = np.random.default_rng(6)
+    B, T, C = 2, 400, 32
+    k = rng.normal(0, 15, (B, T, C)).astype(np.float32)
+    v = rng.normal(0, 1, (B, T, C)).astype(np.float32)
+    w = np.concatenate([np.zeros(4), np.full(4, 1e-5), np.full(4, 40.0),
+                        np.exp(rng.uniform(-5, 2, C - 12))]).astype(np.float32)
+    u = rng.normal(0, 3, C).astype(np.float32)
+    gy = rng.normal(0, 1, (B, T, C)).astype(np.float32)
+
+    class X:
+        pass
+    x = X()
+    x.w, x.u, x.k, x.v = w, u, k, v
+    # keys of N(0, 15) let single steps dominate the sums over B T steps in
+    # gw and gu, whose fp32 accumulation then keeps ~1e-3 of their size
+    compare(m, x, gy, "backward extreme", sums_rel=1e-3)
+
+
+def test_backward_identities_at_full_size(m):
+    """wkv_169m (B=8 T=1024 C=768): the k-shift identity sum_j gk_j = 0 and
+    the constant identity sum_j gv_j = sum_t gy_t per row and channel, and
+    sampled channels against the oracle."""
+    x = workloads.make_wkv("wkv_169m")
+    gy = np.random.default_rng(7).normal(0, 1, x.k.shape).astype(np.float32)
+    gk, gv, gw, gu = run(m, x, gy)
+    assert np.max(np.abs(gk.sum(axis=1))) <= 1e-3 * np.abs(gk).max() * np.sqrt(x.spec.T)
+    assert np.allclose(gv.sum(axis=1), gy.astype(np.float64).sum(axis=1),
+                       atol=1e-3 * np.abs(gv).max() * np.sqrt(x.spec.T))
+    chans = np.array([0, 5, 131, 400, 767])
+    sub = lambda a: np.ascontiguousarray(a[:, :, chans])   # noqa: E731
+    want = oracle.wkv_backward_rnn(x.w[chans], x.u[chans], sub(x.k), sub(x.v), sub(gy))
+    for name, g, wv in zip(("gk", "gv", "gw", "gu"), (sub(gk), sub(gv), gw[chans], gu[chans]),
+                           want):
+        check(g, wv, 2e-4, f"full-size sampled channels {name}")
+
+
+def test_backward_argument_errors(m):
+    x = workloads.make_wkv("wkv_169m", B=1, T=10, C=32, seed=1)
+    w, u, k, v = dev(x.w), dev(x.u), dev(x.k), dev(x.v)
+    gy = torch.ones_like(k)
+    gv, gw, gu = torch.empty_like(k), torch.empty_like(w), torch.empty_like(u)
+    st = m.lib.wkv_backward(1, 10, 32, w.data_ptr(), u.data_ptr(), k.data_ptr(), v.data_ptr(),
+                            gy.data_ptr(), k.data_ptr(), gv.data_ptr(), gw.data_ptr(),
+                            gu.data_ptr(), None)   # gk written over k
+    assert st == m.WKV_ERR_INVALID_ARG
+    st = m.lib.wkv_backward(0, 10, 32, w.data_ptr(), u.data_ptr(), None, None, None, None, None,
+                            gw.data_ptr(), gu.data_ptr(), None)
+    torch.cuda.synchronize()
+    assert st == m.WKV_OK and float(gw.abs().max()) == 0.0 and float(gu.abs().max()) == 0.0

@@ -37,6 +37,8 @@ Named workloads (shapes from RWKV-4 models and the minGRU scan form):
   k/v/r/y, B=8 T=4096 C=2560; k, v, w, u as ``wkv_3b_bf16``, then r ~ N(0, 2)
 * ``shift_3b_bf16`` token shift (3 mixing vectors: k, v, r) on bf16 x,
   B=8 T=4096 C=2560; x ~ N(0, 1), mu ~ U(0, 1) (see ``make_token_shift``)
+* ``wkv_169m_bwd`` the WKV gradients at the ``wkv_169m`` shape and
+  distributions, then an upstream gradient gy ~ N(0, 1)
 * ``wkv_decode`` WKV fp32 RNN-mode decoding, one token per sequence: B=1024
   sequences, T=1, C=2560 (RWKV-4-3B width), k, v, w, u as ``wkv_169m``, plus
   a state per (sequence, channel) from ``make_wkv_state``
@@ -77,6 +79,7 @@ class WkvSpec:
     state: bool = False           # the workload starts from a drawn state
     gated: bool = False           # also draws the receptance r ~ N(0, r_sigma)
     r_sigma: float = 2.0
+    backward: bool = False        # gradients: also draws gy ~ N(0, 1)
 
     @property
     def elements(self) -> int:
@@ -112,6 +115,8 @@ WORKLOADS = {
                           0.5, state=True),
     "wkv_3b_gated_bf16": WkvSpec("wkv_3b_gated_bf16", 8, 4096, 2560, "bf16", 1.0, 1.0,
                                  ("uniform", -3.0, 1.0), 0.5, gated=True),
+    "wkv_169m_bwd": WkvSpec("wkv_169m_bwd", 8, 1024, 768, "f32", 1.0, 1.0,
+                            ("uniform", -3.0, 1.0), 0.5, backward=True),
 }
 
 
@@ -178,6 +183,7 @@ class WkvInputs:
     s_in: Optional[np.ndarray] = None   # [B, 3, C] float32 when spec.state
     r: Optional[np.ndarray] = None      # [B, T, C] float32 when spec.gated
     r_bits: Optional[np.ndarray] = None
+    gy: Optional[np.ndarray] = None     # [B, T, C] float32 when spec.backward
 
 
 @dataclasses.dataclass
@@ -217,13 +223,14 @@ def make_wkv(spec, *, B=None, T=None, C=None, seed=None) -> WkvInputs:
     w = np.exp(_draw_log_w(rng, spec.w_log, spec.C)).astype(np.float32)
     u = rng.normal(0.0, spec.u_sigma, size=spec.C).astype(np.float32)
     r = rng.normal(0.0, spec.r_sigma, size=shape).astype(np.float32) if spec.gated else None
+    gy = rng.normal(0.0, 1.0, size=shape).astype(np.float32) if spec.backward else None
     s_in = make_wkv_state(spec.B, spec.C, spec.seed) if spec.state else None
     if spec.dtype == "bf16":
         kb, vb = bf16_bits(k), bf16_bits(v)
         rb = bf16_bits(r) if r is not None else None
         return WkvInputs(spec, w, u, bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), kb, vb, s_in,
                          None if rb is None else bf16_bits_to_f32(rb), rb)
-    return WkvInputs(spec, w, u, k, v, s_in=s_in, r=r)
+    return WkvInputs(spec, w, u, k, v, s_in=s_in, r=r, gy=gy)
 
 
 @dataclasses.dataclass
