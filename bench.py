@@ -332,7 +332,7 @@ class DeviceWorkload:
         if self.kind == "shift":
             return "token_shift_kernel"
         if self.kind == "bwd":
-            return "wkv_backward_serial_kernel"
+            return "wkv_bwd_grads_kernel"
         if self.kind == "wkv" and self.T <= 16:
             return "wkv_serial_kernel"
         if self.lib.wkv_tile_steps_for(self.B, self.T, self.C, self.es) in (8, 32):

@@ -968,26 +968,35 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const f
             if (overlaps(out[i].p, out[i].bytes, out[j].p, out[j].bytes))
                 return fail(WKV_ERR_INVALID_ARG, "%s overlaps %s", out[i].name, out[j].name);
     }
-    const int64_t blocks = (B * C + kBwdThreads - 1) / kBwdThreads;
-    if (blocks > INT32_MAX) return fail(WKV_ERR_INVALID_ARG, "B*C too large for one launch");
-    // scratch: y_t, ln D_t per element and per-row gw, gu partials
-    const size_t need = 2 * n + static_cast<size_t>(B) * 2 * C * sizeof(float);
+    const int64_t S = (T + kSeg - 1) / kSeg;
+    const int64_t seg_threads = B * S * C;
+    if ((seg_threads + kBwdThreads - 1) / kBwdThreads > INT32_MAX)
+        return fail(WKV_ERR_INVALID_ARG, "B*C*T too large for one launch");
+    // scratch: y_t and ln D_t per element; per (row, segment, channel) the
+    // forward (3) and reverse (5) summaries and the gw, gu partials (2)
+    const size_t ne = static_cast<size_t>(B) * T * C;
+    const size_t ns = static_cast<size_t>(B) * S * C;
+    const size_t need = (2 * ne + 10 * ns) * sizeof(float);
     WsEntry *e = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if ((st = ensure_ws(dev, stream, need, &e, 1)) != WKV_OK) return st;
     }
     float *scratch = reinterpret_cast<float *>(e->base);
-    const size_t ne = static_cast<size_t>(B) * T * C;
-    WkvBwdArgs a{w, u, k, v, gy, gk, gv, scratch, scratch + ne, scratch + 2 * ne, gw, gu};
-    wkv_backward_serial_kernel<<<static_cast<unsigned>(blocks), kBwdThreads, 0, stream>>>(
-        a, static_cast<int>(B), static_cast<int>(T), static_cast<int>(C));
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
-    wkv_backward_reduce_kernel<<<static_cast<unsigned>((C + kBwdThreads - 1) / kBwdThreads),
-                                 kBwdThreads, 0, stream>>>(a, static_cast<int>(B),
-                                                           static_cast<int>(C));
-    err = cudaGetLastError();
+    WkvBwdArgs a{w, u, k, v, gy, gk, gv, scratch, scratch + ne, scratch + 2 * ne,
+                 scratch + 2 * ne + 3 * ns, scratch + 2 * ne + 8 * ns, gw, gu,
+                 static_cast<int>(B), static_cast<int>(T), static_cast<int>(C),
+                 static_cast<int>(S)};
+    const unsigned g_seg = static_cast<unsigned>((seg_threads + kBwdThreads - 1) / kBwdThreads);
+    const unsigned g_chan = static_cast<unsigned>((B * C + kBwdThreads - 1) / kBwdThreads);
+    const unsigned g_red = static_cast<unsigned>((C + kBwdThreads - 1) / kBwdThreads);
+    wkv_bwd_fwd_summary_kernel<<<g_seg, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_fwd_carry_kernel<<<g_chan, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_outputs_kernel<<<g_seg, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_rev_carry_kernel<<<g_chan, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_grads_kernel<<<g_seg, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_reduce_kernel<<<g_red, kBwdThreads, 0, stream>>>(a);
+    const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     return WKV_OK;
 }
