@@ -162,6 +162,8 @@ struct WkvOp {
     static constexpr int NV = 3;
     static constexpr int NIN = GATED ? 3 : 2;  // input tensors per tile: k, v (, r)
     static constexpr int kScalarsPerIo = 1;    // tensor-map elements per io_t
+    // two bf16 channels per thread: per-element arithmetic in packed fp32 pairs
+    static constexpr bool kPacked = sizeof(IO) == 2 && CPT == 2;
     static constexpr bool kGated = GATED;
     static constexpr bool kSerialForm = true;  // has the per-step form of serial_wkv.cuh
     struct Param {
@@ -334,6 +336,34 @@ struct WkvOp {
             a[j] = 0.f;
             b[j] = 0.f;
         }
+        if constexpr (kPacked) {
+            // both channels in packed fp32 pairs: one instruction per pair,
+            // each component rounded as the scalar fmaf / fadd
+            const float2 w2 = make_float2(q[0].w, q[1].w), l2e = make_float2(kLog2e, kLog2e);
+            const float2 nref2 = make_float2(-ref2[0], -ref2[1]);
+            float2 a2 = make_float2(0.f, 0.f), b2 = make_float2(0.f, 0.f);
+            const auto one = [&](int i, float ci) {
+                float k[CPT], v[CPT];
+                Vec<IO, CPT>::load(p0 + i * CG, k);
+                Vec<IO, CPT>::load(p1 + i * CG, v);
+                const float2 x = __ffma2_rn(make_float2(ci, ci), w2, make_float2(k[0], k[1]));
+                const float2 arg = __ffma2_rn(x, l2e, nref2);
+                const float2 e = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+                a2 = __ffma2_rn(e, make_float2(v[0], v[1]), a2);
+                b2 = __fadd2_rn(b2, e);
+            };
+            if (n == LS) {
+#pragma unroll 8
+                for (int i = 0; i < LS; ++i) one(i, static_cast<float>(i - (LS - 1)));
+            } else {
+                for (int i = 0; i < n; ++i) one(i, static_cast<float>(i - (n - 1)));
+            }
+            a[0] = a2.x;
+            a[1] = a2.y;
+            b[0] = b2.x;
+            b[1] = b2.y;
+            return;
+        }
         if (n == LS) {
 #pragma unroll 8
             for (int i = 0; i < LS; ++i) {
@@ -464,6 +494,12 @@ struct WkvOp {
                 carry[j].b >= 1.f && carry[j].p - M[j] - static_cast<float>(n) * q[j].w >= -69.f;
             fast = fast && (by_token || by_carry) && q[j].u <= 44.f;
         }
+        if constexpr (kPacked) {
+            if (fast) {
+                packed_sweep<LS>(p0, p1, p2, n, q, M2, A, Bs, out, ostride, valid);
+                return;
+            }
+        }
         if (fast) {
             if (n == LS) {
 #pragma unroll 8
@@ -497,6 +533,46 @@ struct WkvOp {
         Vec<IO, CPT>::load(pr, r);
 #pragma unroll
         for (int j = 0; j < CPT; ++j) y[j] *= gate_sigmoid(r[j]);
+    }
+
+    // the fixed-reference steps of sweep for two channels in packed fp32 pairs
+    // (same per-component arithmetic as fast_step)
+    template <int LS>
+    __device__ __forceinline__ static void packed_sweep(const IO *p0, const IO *p1, const IO *p2,
+                                                        int n, const Param (&q)[CPT],
+                                                        const float (&M2)[CPT], float (&A)[CPT],
+                                                        float (&Bs)[CPT], IO *out, size_t ostride,
+                                                        bool valid) {
+        const float2 l2e = make_float2(kLog2e, kLog2e), nM2 = make_float2(-M2[0], -M2[1]);
+        const float2 U = make_float2(q[0].U, q[1].U), D = make_float2(q[0].D, q[1].D);
+        float2 a = make_float2(A[0], A[1]), bs = make_float2(Bs[0], Bs[1]);
+        const auto one = [&](int i) {
+            float k[CPT], v[CPT];
+            Vec<IO, CPT>::load(p0 + i * CG, k);
+            Vec<IO, CPT>::load(p1 + i * CG, v);
+            const float2 v2 = make_float2(v[0], v[1]);
+            const float2 arg = __ffma2_rn(make_float2(k[0], k[1]), l2e, nM2);
+            const float2 e = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+            // v + (A - Bs v) / (Bs + e U), as wkv_output
+            const float2 t = __ffma2_rn(make_float2(-bs.x, -bs.y), v2, a);
+            const float2 d = __ffma2_rn(e, U, bs);
+            const float2 y2 = __ffma2_rn(t, make_float2(rcp_approx(d.x), rcp_approx(d.y)), v2);
+            a = __ffma2_rn(a, D, __fmul2_rn(e, v2));
+            bs = __ffma2_rn(bs, D, e);
+            float y[CPT] = {y2.x, y2.y};
+            if constexpr (GATED) apply_gate(p2 + i * CG, y);
+            if (valid) Vec<IO, CPT>::store(out + i * ostride, y);
+        };
+        if (n == LS) {
+#pragma unroll 8
+            for (int i = 0; i < LS; ++i) one(i);
+        } else {
+            for (int i = 0; i < n; ++i) one(i);
+        }
+        A[0] = a.x;
+        A[1] = a.y;
+        Bs[0] = bs.x;
+        Bs[1] = bs.y;
     }
 
     __device__ __forceinline__ static void fast_step(const IO *pk, const IO *pv, const IO *pr,
