@@ -205,7 +205,7 @@ WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,
  *     gv_j = sum_{t>=j} gy_t beta_{t,j},   gk_j = sum_{t>=j} gy_t beta_{t,j} (v_j - y_t),
  *     gu   = sum_t gy_t beta_{t,t} (v_t - y_t),
  *     gw   = -sum_t sum_{j<t} (t-1-j) gy_t beta_{t,j} (v_j - y_t).
- * Time-parallel over segments of 64 steps (six launches: forward segment
+ * Time-parallel over segments of 32 steps (six launches: forward segment
  * summaries, forward carries, outputs and reverse segment summaries, reverse
  * carries, gradients, the gw/gu reduction), recomputing the forward pass and
  * running the sums over later outputs backwards in time, max-stabilised

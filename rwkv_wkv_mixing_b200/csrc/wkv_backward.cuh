@@ -41,7 +41,7 @@
 namespace wkvb {
 
 constexpr int kBwdThreads = 128;
-constexpr int kSeg = 64;  // steps per segment
+constexpr int kSeg = 32;  // steps per segment (32: more threads in flight; 16 lengthens the carries)
 
 struct WkvBwdArgs {
     const float *w, *u;       // [C]
