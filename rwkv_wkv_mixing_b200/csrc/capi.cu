@@ -616,6 +616,7 @@ struct HostPipe {
     cudaStream_t s[kPipeStreams] = {};
     char *stage = nullptr;  // kPipeStreams slices of `slice` bytes
     size_t slice = 0;
+    int *status = nullptr;  // pinned host copies of each stream's device status word
 };
 
 std::mutex g_pipe_mu;  // serialises host-buffer calls (and guards g_pipes)
@@ -637,6 +638,15 @@ wkv_status get_pipe(int dev, size_t slice, HostPipe **out) {
                 return cuda_fail(e, "cudaStreamCreate");
             }
         }
+        void *h = nullptr;
+        cudaError_t e = cudaHostAlloc(&h, kPipeStreams * sizeof(int), cudaHostAllocDefault);
+        if (e != cudaSuccess) {
+            for (int j = 0; j < kPipeStreams; ++j) cudaStreamDestroy(p->s[j]);
+            delete p;
+            cudaGetLastError();
+            return fail(WKV_ERR_OOM, "host-pipeline status words: %s", cudaGetErrorName(e));
+        }
+        p->status = static_cast<int *>(h);
         g_pipes.push_back(p);
     }
     if (p->slice < slice) {
@@ -771,6 +781,21 @@ wkv_status run_host(int64_t B, int64_t T, int64_t C, const void *x0, const void 
         if (st != WKV_OK) break;
         e = copy_chunk(y, dy, ch, T, C, es, false, sc);
     }
+    // each stream's device status word (a device-side wait that gave up)
+    // comes back with the stream's last copy, not through a blocking copy
+    WsEntry *ws_of[kPipeStreams] = {};
+    {
+        std::lock_guard<std::mutex> lk2(g_mu);
+        for (int i = 0; i < kPipeStreams; ++i) {
+            pipe->status[i] = 0;
+            WsEntry *w = find_ws(dev, pipe->s[i]);
+            if (w == nullptr || w->base == nullptr) continue;
+            ws_of[i] = w;
+            cudaError_t ce = cudaMemcpyAsync(&pipe->status[i], w->base + 16, sizeof(int),
+                                             cudaMemcpyDeviceToHost, pipe->s[i]);
+            if (e == cudaSuccess) e = ce;
+        }
+    }
     // whatever happened, nothing may still be using the staging on return
     for (int i = 0; i < kPipeStreams; ++i) {
         cudaError_t se = cudaStreamSynchronize(pipe->s[i]);
@@ -778,16 +803,10 @@ wkv_status run_host(int64_t B, int64_t T, int64_t C, const void *x0, const void 
     }
     if (st != WKV_OK) return st;
     if (e != cudaSuccess) return cuda_fail(e, "host-buffer pipeline");
-    // a device-side wait that gave up on any internal stream
-    std::lock_guard<std::mutex> lk2(g_mu);
     for (int i = 0; i < kPipeStreams; ++i) {
-        WsEntry *w = find_ws(dev, pipe->s[i]);
-        if (w == nullptr || w->base == nullptr) continue;
-        int code = 0;
-        if (cudaMemcpy(&code, w->base + 16, sizeof code, cudaMemcpyDeviceToHost) != cudaSuccess)
-            return cuda_fail(cudaGetLastError(), "cudaMemcpy(status)");
-        if (code != 0) {
-            cudaMemset(w->base + 16, 0, sizeof code);
+        const int code = pipe->status[i];
+        if (code != 0 && ws_of[i] != nullptr) {
+            cudaMemset(ws_of[i]->base + 16, 0, sizeof code);
             return fail(static_cast<wkv_status>(code),
                         "a device-side wait gave up; the affected outputs are NaN");
         }

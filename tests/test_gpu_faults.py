@@ -21,7 +21,7 @@ def m(cuda_dev):
     import rwkv_wkv_mixing_b200 as mod
     yield mod
     mod.wkv_set_fault_injection(-1, 0)
-    mod.wkv_set_tile_steps(128)
+    mod.wkv_set_tile_steps(0)
 
 
 @pytest.mark.parametrize("steps", [128, 32])   # persistent pipeline, block per tile
@@ -59,3 +59,22 @@ def test_fault_injection_arguments_are_checked(m):
     assert m.lib.wkv_set_fault_injection(-2, 0) == m.WKV_ERR_INVALID_ARG
     assert m.lib.wkv_set_fault_injection(0, -1) == m.WKV_ERR_INVALID_ARG
     assert m.lib.wkv_set_fault_injection(-1, 0) == m.WKV_OK
+
+
+def test_host_entry_point_reports_a_timeout(m):
+    """The host-buffer entry point reads each internal stream's status word
+    back with the stream's work and returns WKV_ERR_TIMEOUT for the call
+    whose wait gave up; the next call is correct again."""
+    B, T, C = 1, 1024, 64            # one chunk: the tile numbering of a direct call
+    x = workloads.make_wkv("wkv_169m", B=B, T=T, C=C, seed=102)
+    h = lambda a: torch.from_numpy(np.ascontiguousarray(a))   # noqa: E731
+    w, u, k, v = h(x.w), h(x.u), h(x.k), h(x.v)
+    want = oracle.wkv_rnn(x.w, x.u, x.k, x.v)
+    m.wkv_set_tile_steps(128)
+    m.wkv_set_fault_injection(4, 4096)
+    with pytest.raises(m.WkvError) as err:
+        m.wkv_forward_host(w, u, k, v)
+    assert err.value.status == m.WKV_ERR_TIMEOUT
+    m.wkv_set_fault_injection(-1, 0)
+    y = m.wkv_forward_host(w, u, k, v)
+    assert np.abs(y.double().numpy() - want).max() <= 1e-5 * float(np.abs(x.v).max())
