@@ -146,7 +146,7 @@ wkv_status check_sizes(int64_t B, int64_t T, int64_t C, bool *empty) {
 struct WsEntry {
     int device = -1;
     cudaStream_t stream = nullptr;
-    int kind = 0;  // 0: look-back workspace; 1: gradient scratch
+    int kind = 0;  // 0: look-back workspace; 1: gradient scratch; 2: gradient sum counters
     char *base = nullptr;
     size_t bytes = 0;
 };
@@ -991,30 +991,37 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const f
     const int64_t seg_threads = B * S * C;
     if ((seg_threads + kBwdThreads - 1) / kBwdThreads > INT32_MAX)
         return fail(WKV_ERR_INVALID_ARG, "B*C*T too large for one launch");
-    // scratch: y_t and ln D_t per element; per (row, segment, channel) the
-    // forward (3) and reverse (5) summaries and the gw, gu partials (2)
-    const size_t ne = static_cast<size_t>(B) * T * C;
+    // scratch per (row, segment, channel): the forward (3) and reverse (5)
+    // summaries, then carries, and the gw, gu partials (2); then the
+    // first-level sums of gw, gu.  The sum's counters, one per 32 channels,
+    // have a workspace of their own: zero when allocated, and every launch
+    // leaves them at zero.
+    const int64_t n_cg = (C + 31) / 32;
     const size_t ns = static_cast<size_t>(B) * S * C;
-    const size_t need = (2 * ne + 10 * ns) * sizeof(float);
-    WsEntry *e = nullptr;
+    const size_t nred = static_cast<size_t>(kReduceParts) * 2 * C;
+    WsEntry *e = nullptr, *ce = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if ((st = ensure_ws(dev, stream, need, &e, 1)) != WKV_OK) return st;
+        if ((st = ensure_ws(dev, stream, (10 * ns + nred) * sizeof(float), &e, 1)) != WKV_OK)
+            return st;
+        if ((st = ensure_ws(dev, stream, static_cast<size_t>(n_cg) * sizeof(unsigned), &ce, 2)) !=
+            WKV_OK)
+            return st;
     }
     float *scratch = reinterpret_cast<float *>(e->base);
-    WkvBwdArgs a{w, u, k, v, gy, gk, gv, scratch, scratch + ne, scratch + 2 * ne,
-                 scratch + 2 * ne + 3 * ns, scratch + 2 * ne + 8 * ns, gw, gu,
+    WkvBwdArgs a{w, u, k, v, gy, gk, gv, scratch, scratch + 3 * ns, scratch + 8 * ns, gw, gu,
+                 scratch + 10 * ns, reinterpret_cast<unsigned *>(ce->base),
                  static_cast<int>(B), static_cast<int>(T), static_cast<int>(C),
                  static_cast<int>(S)};
     const unsigned g_seg = static_cast<unsigned>((seg_threads + kBwdThreads - 1) / kBwdThreads);
-    const unsigned g_chan = static_cast<unsigned>((B * C + kBwdThreads - 1) / kBwdThreads);
-    const unsigned g_red = static_cast<unsigned>((C + kBwdThreads - 1) / kBwdThreads);
+    const unsigned g_chan = static_cast<unsigned>(B * n_cg);
+    const unsigned g_red = static_cast<unsigned>(n_cg * kReduceParts);
     wkv_bwd_fwd_summary_kernel<<<g_seg, kBwdThreads, 0, stream>>>(a);
-    wkv_bwd_fwd_carry_kernel<<<g_chan, kBwdThreads, 0, stream>>>(a);
-    wkv_bwd_outputs_kernel<<<g_seg, kBwdThreads, 0, stream>>>(a);
-    wkv_bwd_rev_carry_kernel<<<g_chan, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_fwd_carry_kernel<<<g_chan, 32 * kCarryWarps, 0, stream>>>(a);
+    wkv_bwd_rev_summary_kernel<<<g_seg, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_rev_carry_kernel<<<g_chan, 32 * kCarryWarps, 0, stream>>>(a);
     wkv_bwd_grads_kernel<<<g_seg, kBwdThreads, 0, stream>>>(a);
-    wkv_bwd_reduce_kernel<<<g_red, kBwdThreads, 0, stream>>>(a);
+    wkv_bwd_reduce_kernel<<<g_red, 32 * kReduceWarps, 0, stream>>>(a);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     return WKV_OK;

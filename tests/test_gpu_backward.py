@@ -50,7 +50,8 @@ def compare(m, x, gy, what, sums_rel=2e-4):
         check(g, wv, rel, f"{what} {name}")
 
 
-SHAPES = [(1, 1, 4), (2, 5, 32), (2, 64, 40), (3, 300, 33), (1, 1024, 64), (4, 700, 130)]
+SHAPES = [(1, 1, 4), (2, 5, 32), (2, 64, 40), (3, 300, 33), (1, 1024, 64), (4, 700, 130),
+          (1, 4100, 40), (2, 257, 96)]
 
 
 @pytest.mark.parametrize("B,T,C", SHAPES)
