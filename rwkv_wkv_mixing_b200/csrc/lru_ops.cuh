@@ -8,12 +8,14 @@
 // per complex channel, u and x stored as interleaved (re, im) float pairs.
 // lambda does not change with t, so a chunk of n steps is summarised by its
 // state from zero alone (its transition is lambda^n), and a state followed by
-// a chunk of n steps is lambda^n x + H.  lambda^n for a chunk length comes
-// from the exponent n (-nu + i theta) evaluated in double precision: the
-// phase n theta reaches 10^6 radians for long sequences, far beyond what
-// single precision can reduce.  Inside a sub-chunk the state steps with the
-// single-precision lambda (at most a tile's worth of steps).  nu and theta
-// themselves are kept in double: a phase n theta is only as exact as theta.
+// a chunk of n steps is lambda^n x + H.  lambda^n = e^{-n nu} e^{i n theta}:
+// the phase n theta reaches 10^6 radians for long sequences, far beyond what
+// single precision can reduce, so n theta and its reduction to [-pi, pi]
+// (subtracting the nearest multiple of 2 pi) are done in double precision and
+// only the reduced phase and the magnitude go through single-precision
+// functions.  Inside a sub-chunk the state steps with the single-precision
+// lambda (at most a tile's worth of steps).  nu and theta themselves are kept
+// in double: a phase n theta is only as exact as theta.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -49,16 +51,23 @@ struct LruOp {
     };
     struct Scratch {};
 
+    // e^{i phase} for a phase given in double: reduced to [-pi, pi] in double
+    __device__ __forceinline__ static void unit_phase(double phase, float &c, float &s) {
+        constexpr double kTwoPi = 6.283185307179586, kInvTwoPi = 0.15915494309189535;
+        const double red = fma(-kTwoPi, rint(phase * kInvTwoPi), phase);
+        sincosf(static_cast<float>(red), &s, &c);
+    }
+
     __device__ __forceinline__ static Param param(const Args &args, int c, int C) {
         Param q{0.f, 0.f, 1.f, 0.0, 0.0};
         if (c < C) {
             q.nu = exp(static_cast<double>(args.nu_log[c]));
             q.theta = exp(static_cast<double>(args.theta_log[c]));
-            const double r = exp(-q.nu);
-            double s, co;
-            sincos(q.theta, &s, &co);
-            q.lr = static_cast<float>(r * co);
-            q.li = static_cast<float>(r * s);
+            const float r = expf(-static_cast<float>(q.nu));
+            float co, si;
+            unit_phase(q.theta, co, si);
+            q.lr = r * co;
+            q.li = r * si;
             q.g = args.gamma != nullptr ? args.gamma[c] : 1.f;
         }
         return q;
@@ -85,15 +94,15 @@ struct LruOp {
     __device__ __forceinline__ static State unpack(float x, float y, uint32_t) { return {x, y}; }
 
     // l followed by a chunk of n steps whose state from zero is r:
-    // lambda^n l + r, lambda^n = e^{n (-nu + i theta)} in double precision
+    // lambda^n l + r, lambda^n = e^{-n nu} e^{i n theta}
     __device__ __forceinline__ static State combine(const State &l, const State &r, float n,
                                                     const Param &q) {
         if (n == 0.f) return {l.r + r.r, l.i + r.i};
         const double nn = static_cast<double>(n);
-        const double mag = exp(-nn * q.nu);
-        double s, c;
-        sincos(nn * q.theta, &s, &c);
-        const float pr = static_cast<float>(mag * c), pi = static_cast<float>(mag * s);
+        const float mag = expf(-static_cast<float>(nn * q.nu));
+        float c, s;
+        unit_phase(nn * q.theta, c, s);
+        const float pr = mag * c, pi = mag * s;
         return {fmaf(pr, l.r, fmaf(-pi, l.i, r.r)), fmaf(pr, l.i, fmaf(pi, l.r, r.i))};
     }
 
