@@ -240,6 +240,15 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
 #pragma unroll
             for (int j = 0; j < CPT; ++j) prm[j] = Op::param(args, c0 + lane * CPT + j, g.C);
 
+            // the carry warps load the record their look-back reads first now:
+            // the tile before this one in time was handed out well before it,
+            // so its state is usually published already and lands during pass 1
+            const bool lb = chained && seg > 0;
+            ChannelPrefetch<1> pf;
+#pragma unroll
+            for (int j = 0; j < CPT; ++j)
+                if (wg == j && lb) lookback_prefetch_channel<Op>(ws, g, tile, lane, j, pf);
+
             // pass 1
             const int s0 = wg * LS;
             const int nval = max(0, min(LS, g.T - (t0 + s0)));
@@ -257,73 +266,53 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             }
             named_bar_sync(bar_id, NWG * 32);
 
-            // carry into the tile (the group's first warp)
-            if (wg == 0) {
-                // the look-back's first records are loaded now and land while the
-                // warp folds and publishes this tile's aggregate
-                LookbackPrefetch<Op> pf;
-                const bool lb = chained && seg > 0;
-                if (lb) lookback_prefetch<Op>(ws, g, tile, lane, pf);
-                State agg[CPT], X[CPT];
+            // carry into the tile: channel j of every lane by the group's warp
+            // j, so a lane's CPT channels resolve in parallel
+            static_assert(CPT <= NWG, "one carry warp per channel of a lane");
 #pragma unroll
-                for (int j = 0; j < CPT; ++j) {
-                    // fold the warps' summaries in time order; each slot is
-                    // overwritten with its warp's exclusive prefix (the fold of
-                    // the sub-chunks before it) for pass 2
-                    agg[j] = Op::identity();
-                    for (int w = 0; w < NWG; ++w) {
-                        float vals[NV];
-                        float *slot = g_sum + w * NV * CG + lane * CPT + j;
+            for (int j = 0; j < CPT; ++j) {  // j is a constant in each copy: prm[j] stays in registers
+                if (wg != j) continue;
+                // fold the warps' summaries in time order; each slot is
+                // overwritten with its warp's exclusive prefix (the fold of the
+                // sub-chunks before it) for pass 2
+                State agg = Op::identity();
+                for (int w = 0; w < NWG; ++w) {
+                    float vals[NV];
+                    float *slot = g_sum + w * NV * CG + lane * CPT + j;
 #pragma unroll
-                        for (int q = 0; q < NV; ++q) vals[q] = slot[q * CG];
+                    for (int q = 0; q < NV; ++q) vals[q] = slot[q * CG];
 #pragma unroll
-                        for (int q = 0; q < NV; ++q) slot[q * CG] = Op::get(agg[j], q);
-                        const int len = max(0, min(LS, g.T - (t0 + w * LS)));
-                        agg[j] = Op::combine(agg[j], Op::make(vals), static_cast<float>(len), prm[j]);
-                    }
-                    // the state before step 0 seeds the first segment only
-                    X[j] = seg == 0 ? Op::carry0(args, b, c0 + lane * CPT + j, g.C)
-                                    : Op::identity();
+                    for (int q = 0; q < NV; ++q) slot[q * CG] = Op::get(agg, q);
+                    const int len = max(0, min(LS, g.T - (t0 + w * LS)));
+                    agg = Op::combine(agg, Op::make(vals), static_cast<float>(len), prm[j]);
                 }
+                // the state before step 0 seeds the first segment only
+                State X = seg == 0 ? Op::carry0(args, b, c0 + lane * CPT + j, g.C)
+                                   : Op::identity();
                 if (chained) {
                     const bool last = seg == g.n_seg - 1;
                     if (seg == 0) {
-                        State inc[CPT];
-#pragma unroll
-                        for (int j = 0; j < CPT; ++j)
-                            inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                        publish<Op, CG>(ws, g, tile, inc, kFlagIncl, epoch, lane);
+                        publish_channel<Op, CG>(ws, g, tile,
+                                                Op::combine(X, agg, static_cast<float>(LT), prm[j]),
+                                                j, kFlagIncl, epoch, lane);
                     } else {
-                        if (!last)
-                            publish<Op, CG>(ws, g, tile, agg, kFlagAgg, epoch, lane);
-                        State run[CPT];
-                        if (!lookback<Op, LT>(ws, g, tile, epoch, prm, lane, run, lb ? &pf : nullptr)) {
+                        if (!last) publish_channel<Op, CG>(ws, g, tile, agg, j, kFlagAgg, epoch, lane);
+                        if (!lookback_channel<Op, LT>(ws, g, tile, epoch, prm[j], lane, j, X,
+                                                      lb ? &pf : nullptr)) {
                             atomicExch(ws.status, kStatusTimeout);  // this lane gave up
-#pragma unroll
-                            for (int j = 0; j < CPT; ++j) run[j] = Op::nan_state();
+                            X = Op::nan_state();
                         }
-#pragma unroll
-                        for (int j = 0; j < CPT; ++j) X[j] = run[j];
-                        if (!last) {
-                            State inc[CPT];
-#pragma unroll
-                            for (int j = 0; j < CPT; ++j)
-                                inc[j] = Op::combine(X[j], agg[j], static_cast<float>(LT), prm[j]);
-                            publish<Op, CG>(ws, g, tile, inc, kFlagIncl, epoch, lane);
-                        }
+                        if (!last)
+                            publish_channel<Op, CG>(
+                                ws, g, tile, Op::combine(X, agg, static_cast<float>(LT), prm[j]), j,
+                                kFlagIncl, epoch, lane);
                     }
                 }
-                if (seg == g.n_seg - 1) {  // the state after the last step
-                    const float len = static_cast<float>(min(LT, g.T - t0));
+                if (seg == g.n_seg - 1)  // the state after the last step
+                    Op::store_final(args, b, c0 + lane * CPT + j, g.C,
+                                    Op::combine(X, agg, static_cast<float>(min(LT, g.T - t0)), prm[j]));
 #pragma unroll
-                    for (int j = 0; j < CPT; ++j)
-                        Op::store_final(args, b, c0 + lane * CPT + j, g.C,
-                                        Op::combine(X[j], agg[j], len, prm[j]));
-                }
-#pragma unroll
-                for (int j = 0; j < CPT; ++j)
-#pragma unroll
-                    for (int q = 0; q < NV; ++q) g_carry[q * CG + lane * CPT + j] = Op::get(X[j], q);
+                for (int q = 0; q < NV; ++q) g_carry[q * CG + lane * CPT + j] = Op::get(X, q);
             }
             named_bar_sync(bar_id, NWG * 32);
 

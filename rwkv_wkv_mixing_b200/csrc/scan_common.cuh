@@ -68,26 +68,32 @@ __device__ __forceinline__ unsigned long long epoch_of(const Workspace &ws) {
     return ld_relaxed_gpu_u64(ws.epoch) & ((1ull << kEpochBits) - 1ull);
 }
 
-// Publish this lane's CPT channels of `tile` with the given flag.  (The
-// fault-injection test hook can name one tile that never publishes, so that
-// the look-back waits behind it run out.)
+// Publish channel j of this lane's CPT channels of `tile` with the given
+// flag.  (The fault-injection test hook can name one tile that never
+// publishes, so that the look-back waits behind it run out.)
+template <class Op, int CG>
+__device__ __forceinline__ void publish_channel(const Workspace &ws, const Geometry &g, int tile,
+                                                const typename Op::State &val, int j,
+                                                uint32_t flag, unsigned long long epoch,
+                                                int lane) {
+    if (tile == g.skip_publish) return;
+    uint4 *dst = ws.records + static_cast<size_t>(tile) * CG + lane * Op::CPT + j;
+    float x, y;
+    uint32_t bits16;
+    Op::pack(val, x, y, bits16);
+    const unsigned long long tag =
+        (epoch << 18) | (static_cast<unsigned long long>(bits16 & 0xffffu) << 2) | flag;
+    st_relaxed_gpu_v4(dst, make_uint4(__float_as_uint(x), __float_as_uint(y),
+                                      static_cast<uint32_t>(tag), static_cast<uint32_t>(tag >> 32)));
+}
+
+// all CPT channels of this lane
 template <class Op, int CG>
 __device__ __forceinline__ void publish(const Workspace &ws, const Geometry &g, int tile,
                                         const typename Op::State (&val)[Op::CPT], uint32_t flag,
                                         unsigned long long epoch, int lane) {
-    if (tile == g.skip_publish) return;
-    uint4 *dst = ws.records + static_cast<size_t>(tile) * CG + lane * Op::CPT;
 #pragma unroll
-    for (int j = 0; j < Op::CPT; ++j) {
-        float x, y;
-        uint32_t bits16;
-        Op::pack(val[j], x, y, bits16);
-        const unsigned long long tag =
-            (epoch << 18) | (static_cast<unsigned long long>(bits16 & 0xffffu) << 2) | flag;
-        st_relaxed_gpu_v4(dst + j, make_uint4(__float_as_uint(x), __float_as_uint(y),
-                                              static_cast<uint32_t>(tag),
-                                              static_cast<uint32_t>(tag >> 32)));
-    }
+    for (int j = 0; j < Op::CPT; ++j) publish_channel<Op, CG>(ws, g, tile, val[j], j, flag, epoch, lane);
 }
 
 __device__ __forceinline__ unsigned long long record_tag(uint4 r) {
@@ -117,93 +123,110 @@ __device__ __forceinline__ void finish_launch(const Workspace &ws, bool chained,
 // The first records a tile's look-back will read, loaded ahead of time: the
 // look-back does not depend on the tile's own data, so the carry warp issues
 // these loads before it folds and publishes its own aggregate, and they land
-// while it does.
+// while it does.  H hops of one channel.
+template <int H>
+struct ChannelPrefetch {
+    static constexpr int kHops = H;
+    uint4 rec[H];
+};
+
+template <class Op, int H>
+__device__ __forceinline__ void lookback_prefetch_channel(const Workspace &ws, const Geometry &g,
+                                                          int tile, int lane, int j,
+                                                          ChannelPrefetch<H> &pf) {
+    constexpr int CPT = Op::CPT, CG = 32 * CPT;
+    const long long S = g.tiles_per_seg;
+#pragma unroll
+    for (int i = 0; i < H; ++i) {
+        const long long q = static_cast<long long>(tile) - (i + 1) * S;
+        pf.rec[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (q >= 0) pf.rec[i] = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
+    }
+}
+
+// every channel of this lane, 4 records in all
 template <class Op>
 struct LookbackPrefetch {
-    static constexpr int kHops = 4 / Op::CPT;
-    uint4 rec[Op::CPT][kHops];
+    ChannelPrefetch<4 / Op::CPT> ch[Op::CPT];
 };
 
 template <class Op>
 __device__ __forceinline__ void lookback_prefetch(const Workspace &ws, const Geometry &g, int tile,
                                                   int lane, LookbackPrefetch<Op> &pf) {
-    constexpr int CPT = Op::CPT, CG = 32 * CPT;
-    const long long S = g.tiles_per_seg;
 #pragma unroll
-    for (int j = 0; j < CPT; ++j)
-#pragma unroll
-        for (int i = 0; i < LookbackPrefetch<Op>::kHops; ++i) {
-            const long long q = static_cast<long long>(tile) - (i + 1) * S;
-            pf.rec[j][i] = make_uint4(0u, 0u, 0u, 0u);
-            if (q >= 0) pf.rec[j][i] = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
-        }
+    for (int j = 0; j < Op::CPT; ++j) lookback_prefetch_channel<Op>(ws, g, tile, lane, j, pf.ch[j]);
 }
 
-// Decoupled look-back for one tile, each lane for its own CPT channels.  The
-// tiles before this one in time are tile - S, tile - 2S, ... (S = tiles per
-// time segment).  A lane folds its channel's records newest first -- a tile
-// aggregate moves the fold one tile further back, a state-after-tile ends it
-// -- prefetching several hops' records with independent loads.  Lanes may
-// stop at different hops; each ends with the state before this tile.
-// Returns false (in every lane that gave up) if a record never appeared
-// within the poll budget.
+// Decoupled look-back for one tile, channel j of this lane's CPT channels.
+// The tiles before this one in time are tile - S, tile - 2S, ... (S = tiles
+// per time segment).  The lane folds its channel's records newest first -- a
+// tile aggregate moves the fold one tile further back, a state-after-tile
+// ends it -- prefetching several hops' records with independent loads.
+// Lanes may stop at different hops; each ends with the state before this
+// tile.  Returns false if a record never appeared within the poll budget.
+template <class Op, int LT, int H>
+__device__ __forceinline__ bool lookback_channel(const Workspace &ws, const Geometry &g, int tile,
+                                                 unsigned long long epoch,
+                                                 const typename Op::Param &prm, int lane, int j,
+                                                 typename Op::State &run,
+                                                 const ChannelPrefetch<H> *pre) {
+    constexpr int CPT = Op::CPT, CG = 32 * CPT, HB = 4;  // hops per batch of loads
+    const long long S = g.tiles_per_seg;
+    run = Op::identity();
+    float run_len = 0.f;
+    long long base = tile;
+    bool first = true;
+    for (;;) {
+        uint4 rec[HB];
+#pragma unroll
+        for (int i = 0; i < HB; ++i) {
+            const long long q = base - (i + 1) * S;
+            rec[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (first && pre != nullptr && i < H)
+                rec[i] = pre->rec[i];   // possibly stale: re-polled below if not ready
+            else if (q >= 0)
+                rec[i] = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
+        }
+        first = false;
+#pragma unroll
+        for (int i = 0; i < HB; ++i) {
+            const long long q = base - (i + 1) * S;
+            if (q < 0) return false;  // cannot happen: first-segment tiles always end the fold
+            uint4 r = rec[i];
+            long long polls = 0;
+            while (((record_tag(r) >> 18) != epoch) || (record_tag(r) & 3u) == 0u) {
+                if (++polls > g.spin_limit) return false;
+                __nanosleep(32);
+                r = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
+            }
+            const unsigned long long tag = record_tag(r);
+            const typename Op::State val = Op::unpack(
+                __uint_as_float(r.x), __uint_as_float(r.y), static_cast<uint32_t>(tag >> 2) & 0xffffu);
+            run = Op::combine(val, run, run_len, prm);
+            run_len += static_cast<float>(LT);
+            if ((tag & 3u) == kFlagIncl) return true;
+        }
+        base -= HB * S;
+    }
+}
+
+// all CPT channels of this lane, one after another; false (in every lane
+// that gave up) if a record never appeared within the poll budget
 template <class Op, int LT>
 __device__ __forceinline__ bool lookback(const Workspace &ws, const Geometry &g, int tile,
                                          unsigned long long epoch,
                                          const typename Op::Param (&prm)[Op::CPT], int lane,
                                          typename Op::State (&run)[Op::CPT],
                                          const LookbackPrefetch<Op> *pre = nullptr) {
-    constexpr int CPT = Op::CPT, CG = 32 * CPT, HB = 4;  // hops per batch of loads
-    constexpr int PH = LookbackPrefetch<Op>::kHops;
-    const long long S = g.tiles_per_seg;
     bool ok = true;
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) {
-        run[j] = Op::identity();
-        float run_len = 0.f;
-        long long base = tile;
-        bool done = false;
-        bool first = true;
-        while (!done && ok) {
-            uint4 rec[HB];
-#pragma unroll
-            for (int i = 0; i < HB; ++i) {
-                const long long q = base - (i + 1) * S;
-                rec[i] = make_uint4(0u, 0u, 0u, 0u);
-                if (first && pre != nullptr && i < PH)
-                    rec[i] = pre->rec[j][i];   // possibly stale: re-polled below if not ready
-                else if (q >= 0)
-                    rec[i] = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
-            }
-            first = false;
-#pragma unroll
-            for (int i = 0; i < HB; ++i) {
-                if (done || !ok) break;
-                const long long q = base - (i + 1) * S;
-                if (q < 0) {  // cannot happen: first-segment tiles always end the fold
-                    ok = false;
-                    break;
-                }
-                uint4 r = rec[i];
-                long long polls = 0;
-                while (((record_tag(r) >> 18) != epoch) || (record_tag(r) & 3u) == 0u) {
-                    if (++polls > g.spin_limit) {
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(32);
-                    r = ld_relaxed_gpu_v4(ws.records + q * CG + lane * CPT + j);
-                }
-                if (!ok) break;
-                const unsigned long long tag = record_tag(r);
-                const typename Op::State val = Op::unpack(
-                    __uint_as_float(r.x), __uint_as_float(r.y), static_cast<uint32_t>(tag >> 2) & 0xffffu);
-                run[j] = Op::combine(val, run[j], run_len, prm[j]);
-                run_len += static_cast<float>(LT);
-                done = (tag & 3u) == kFlagIncl;
-            }
-            base -= HB * S;
+    for (int j = 0; j < Op::CPT; ++j) {
+        if (!ok) {
+            run[j] = Op::identity();
+            continue;
         }
+        ok = lookback_channel<Op, LT>(ws, g, tile, epoch, prm[j], lane, j, run[j],
+                                      pre != nullptr ? &pre->ch[j] : nullptr);
     }
     return ok;
 }
