@@ -656,8 +656,9 @@ def grad_finite_difference(fn, h=1e-6, tol=1e-7):
 def grad_identities(fn, tol=1e-11):
     """T = 1: y = v, so gv = gy and the rest vanish.  For any input: the
     outputs are invariant to shifting k, so sum_j gk_j = 0 per row and
-    channel; and a weighted mean reproduces constants, so sum_j gv_j =
-    sum_t gy_t."""
+    channel; a weighted mean reproduces constants, so sum_j gv_j =
+    sum_t gy_t; and the decay's gradient is the keys' first moment less the
+    bonus's, gw = sum_j j gk_j - gu."""
     out = []
     rng = np.random.default_rng(53)
     w, u, k, v = _rand_wkv(53, B=2, T=1, C=4)
@@ -673,6 +674,16 @@ def grad_identities(fn, tol=1e-11):
     if msg: out.append(f"gradient k-shift identity: {msg}")
     msg = _close(np.asarray(gv).sum(axis=1), gy.sum(axis=1), tol * 30)
     if msg: out.append(f"gradient constant identity: {msg}")
+    # w enters the logits of output t as j w - (t-1) w for j < t and not at
+    # all in the diagonal u + k_t.  A softmax ignores a constant added to a
+    # whole row, so moving the row's -(t-1) w onto every logit of the row
+    # leaves the weight j on l_{t,j} (j < t) and t - 1 on l_{t,t}; k_j enters
+    # l_{t,j} with weight 1 and u the diagonal only, hence
+    # gw = sum_j j gk_j - gu (summed over rows; j counted from 0).
+    j = np.arange(k.shape[1])[None, :, None]
+    moment = (j * np.asarray(gk)).sum(axis=(0, 1)) - np.asarray(gu)
+    msg = _close(moment, np.asarray(gw), tol * 30 * max(1.0, float(np.abs(gw).max())))
+    if msg: out.append(f"gradient w-shift identity: {msg}")
     return out
 
 
