@@ -205,15 +205,16 @@ WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,
  *     gv_j = sum_{t>=j} gy_t beta_{t,j},   gk_j = sum_{t>=j} gy_t beta_{t,j} (v_j - y_t),
  *     gu   = sum_t gy_t beta_{t,t} (v_t - y_t),
  *     gw   = -sum_t sum_{j<t} (t-1-j) gy_t beta_{t,j} (v_j - y_t).
- * Time-parallel over segments of 32 steps (six launches: forward segment
- * summaries, forward carries, outputs and reverse segment summaries, reverse
- * carries, gradients, the gw/gu reduction), recomputing the forward pass and
- * running the sums over later outputs backwards in time, max-stabilised
- * (every exponent <= 0 for finite inputs); gw and gu are reduced over rows
- * and segments in a fixed order, so results do not depend on timing.
- * Scratch (8 bytes per element plus 40 per row, segment and channel) is a
- * library-owned per-stream buffer, allocated on first use like the
- * look-back workspace (make one call of each size before stream capture).
+ * Time-parallel over segments of 16 steps (six launches: forward segment
+ * summaries, forward carries, reverse segment summaries, reverse carries,
+ * gradients, the gw/gu reduction), recomputing the forward outputs per
+ * segment and running the sums over later outputs backwards in time,
+ * max-stabilised (every exponent <= 0 for finite inputs); gw and gu are
+ * reduced over rows and segments in a fixed order, so results do not depend
+ * on timing.  Scratch (40 bytes per row, segment and channel, plus 64 bytes
+ * per channel and a counter per 32 channels) is library-owned per-stream
+ * memory, allocated on first use like the look-back workspace (make one call
+ * of each size before stream capture).
  * No output may overlap an input or another output.  Pointers 4-byte
  * aligned.  B or T = 0 with C > 0 sets gw, gu to 0. */
 WKV_API wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
