@@ -6,8 +6,9 @@
 
 One step is one pass of the hot path over one batch of synthetic input
 already resident in HBM: a WKV forward (or, for ``--workload scan_mingru``,
-a diagonal scan).  The default workload is the RWKV-4-169M-shaped WKV forward
-(fp32, B=8, T=1024, C=768).  W untimed warm-up steps and a short untimed soak
+a diagonal scan).  The default workload is the largest single-GPU WKV
+forward: the long-sequence one (fp32, B=1, T=131072, C=1024, keys of
+standard deviation 3, slow decays); ``--workload`` selects the others.  W untimed warm-up steps and a short untimed soak
 run first; then exactly K steps are timed with CUDA events on the launching
 stream, bracketed by a barrier and a device synchronisation, and the maximum
 over ranks is taken.  Inputs rotate over enough buffer sets that the data a
@@ -19,7 +20,10 @@ Printed (rank 0): one JSON line with the metric, the roofline of the kernel
 HBM peak), the float64 CPU oracle timed on this host's cores, an end-to-end
 number through the C ABI with host buffers (host->device copies, the call,
 device->host copy of the result, every step), SM clocks sampled during the
-timed region, and the number of library kernel launches timed.
+timed region (NVML queries every fraction of a millisecond while the timed
+steps run; null when none landed inside it), and the number of library
+kernel launches timed.  The CPU oracle is timed on all of this host's cores
+and on one core.
 
 ``--impl reference`` times the CPU oracle instead (the only reference this
 project has: a plain float64 implementation of the pages' definition), on a
@@ -60,12 +64,12 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
-    ap.add_argument("--workload", default="wkv_169m", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="wkv_long", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="untimed steps before the timed region, so clocks settle")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="budget of the CPU-oracle baseline (rank 0, N=1)")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="budget of each CPU-oracle leg, all cores and one core (rank 0, N=1)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -135,28 +139,78 @@ def cpu_model():
 
 
 class ClockSampler:
-    """nvidia-smi SM clock / throttle-reason samples every 100 ms."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons, read-only, sampled from a
+    background thread: NVML queries every `fast_s` seconds while `fast()` is
+    on (around the timed region, so even a few milliseconds of timed steps
+    get samples), every 100 ms otherwise; `nvidia-smi -lms 100` when NVML
+    cannot be loaded.  Nothing is ever set."""
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id=None):
-        self.samples = []
+    def __init__(self, gpu_uuid=None, fast_s=0.0002):
+        self.samples = []          # (time, sm_mhz, sm_max_mhz, [reason names])
         self.proc = None
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+        self.source = None
+        self._fast = False
+        self._stop = False
+        self.fast_s = fast_s
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            if gpu_uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.nvml, self.handle = pynvml, h
+            self.bits = (pynvml.nvmlClocksEventReasonHwSlowdown,
+                         pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                         pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                         pynvml.nvmlClocksEventReasonSwPowerCap)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.nvml = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits",
                "-lms", "100"]
-        if gpu_id:
-            cmd += ["-i", gpu_id]
+        if gpu_uuid:
+            cmd += ["-i", gpu_uuid]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
         except Exception:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi"
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
+    def _poll_nvml(self):
+        nv, h = self.nvml, self.handle
+        try:
+            reasons_fn = nv.nvmlDeviceGetCurrentClocksEventReasons
+        except AttributeError:
+            reasons_fn = nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop:
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = int(reasons_fn(h))
+                self.samples.append((time.time(), sm, self.max_mhz,
+                                     [n for n, b in zip(self.NAMES, self.bits) if r & b]))
+            except Exception:
+                pass
+            time.sleep(self.fast_s if self._fast else 0.1)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
@@ -165,30 +219,45 @@ class ClockSampler:
                 sm, smax = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            self.samples.append((time.time(), sm, smax, parts[2], parts[4:8]))
+            self.samples.append((time.time(), sm, smax,
+                                 [n for n, r in zip(self.NAMES, parts[4:8])
+                                  if r.lower().startswith("active")]))
+
+    def fast(self, on):
+        self._fast = bool(on)
 
     def stop(self):
+        self._stop = True
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        if self.nvml is not None:
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
 
-    def summary(self, t0, t1):
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    def summary(self, t0, t1, timed_ms=None):
+        """Samples taken inside [t0, t1] only; sm_mhz is null when none
+        landed there.  `mhz_x_ms` is the timed milliseconds times the median
+        SM clock, to compare runs at different clocks."""
         win = [s for s in self.samples if t0 <= s[0] <= t1]
-        window = "timed"
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": len(win),
+               "window": "timed", "source": self.source}
         if not win:
-            win = self.samples
-            window = "run"
-        if not win:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        reasons = sorted({names[i] for s in win for i, r in enumerate(s[4])
-                          if r.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(s[1] for s in win),
-                "sm_max_mhz": max(s[2] for s in win), "reasons": reasons,
-                "samples": len(win), "window": window}
+            return out
+        med = statistics.median(s[1] for s in win)
+        out.update({"sm_mhz": med, "sm_min_mhz": min(s[1] for s in win),
+                    "sm_max_mhz": max(s[2] for s in win),
+                    "reasons": sorted({n for s in win for n in s[3]})})
+        if timed_ms is not None:
+            out["mhz_x_ms"] = med * timed_ms
+        return out
 
 
 # ---------------------------------------------------------------------------
@@ -523,9 +592,11 @@ def e2e_leg(torch, wl, steps):
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline / reference arm)
 # ---------------------------------------------------------------------------
-def oracle_runner(name, max_elements=None):
+def oracle_runner(name, max_elements=None, nthreads=0):
     """A callable running the float64 oracle once over a sample of the
-    workload, and the sample's element count and description."""
+    workload, and the sample's element count and description.  `nthreads`
+    (0: all) is passed to the C oracle's OpenMP loops; the numpy oracles
+    (gate, token shift, LRU) run on one thread either way."""
     import oracle
     spec = workloads.WORKLOADS[name]
     if isinstance(spec, workloads.ScanSpec):
@@ -534,7 +605,7 @@ def oracle_runner(name, max_elements=None):
         B, T, C = a.shape
         rows = B if max_elements is None else max(1, min(B, max_elements // (T * C)))
         a, b = np.ascontiguousarray(a[:rows]), np.ascontiguousarray(b[:rows])
-        fn = lambda: oracle.scan_rnn(a, b, None)   # noqa: E731
+        fn = lambda: oracle.scan_rnn(a, b, None, nthreads)   # noqa: E731
         return fn, rows * T * C, f"{rows} of {B} batch rows (all T={T}, D={C})"
     if isinstance(spec, workloads.LruSpec):
         x = workloads.make_lru(name)
@@ -567,32 +638,49 @@ def oracle_runner(name, max_elements=None):
         np.ascontiguousarray(x.s_in[:rows, :, :chans], dtype=np.float64)
     if x.gy is not None:
         gy = np.ascontiguousarray(x.gy[:rows, :, :chans], dtype=np.float64)
-        fn = lambda: oracle.wkv_backward_rnn(w, u, k, v, gy)   # noqa: E731
+        fn = lambda: oracle.wkv_backward_rnn(w, u, k, v, gy, nthreads)   # noqa: E731
     elif x.r is not None:
         r = np.ascontiguousarray(x.r[:rows, :, :chans], dtype=np.float64)
         fn = lambda: oracle.wkv_gated(w, u, k, v, r, s_in)   # noqa: E731
     elif s_in is not None:
-        fn = lambda: oracle.wkv_rnn_state(w, u, k, v, s_in)   # noqa: E731
+        fn = lambda: oracle.wkv_rnn_state(w, u, k, v, s_in, nthreads)   # noqa: E731
     else:
-        fn = lambda: oracle.wkv_rnn(w, u, k, v)   # noqa: E731
+        fn = lambda: oracle.wkv_rnn(w, u, k, v, nthreads)   # noqa: E731
     return fn, rows * T * chans, f"{rows} of {B} batch rows x {chans} of {C} channels (all T={T})"
 
 
-def cpu_baseline(name, seconds):
+def _time_oracle(name, seconds, nthreads):
+    """Run the oracle over a sample of `name` for about `seconds`; elements
+    per second, the thread count used and the sample's description."""
     import oracle
-    fn, n, desc = oracle_runner(name, max_elements=None)
+    fn, n, desc = oracle_runner(name, max_elements=None, nthreads=nthreads)
     t0 = time.perf_counter(); fn(); one = time.perf_counter() - t0
     if one > seconds:   # a smaller sample of the same workload
-        fn, n, desc = oracle_runner(name, max_elements=max(1, int(n * seconds / one / 2)))
+        fn, n, desc = oracle_runner(name, max_elements=max(1, int(n * seconds / one / 2)),
+                                    nthreads=nthreads)
         t0 = time.perf_counter(); fn(); one = time.perf_counter() - t0
     reps = max(1, int(seconds / max(one, 1e-6)))
     t0 = time.perf_counter()
     for _ in range(reps):
         fn()
     dt = time.perf_counter() - t0
-    return {"value": n * reps / dt, "unit": "elem/s", "cores": oracle.max_threads(),
-            "kind": "oracle", "sample": f"{desc}, {reps} passes, float64 RNN-mode oracle",
-            "seconds": dt, "cpu": cpu_model()}
+    spec = workloads.WORKLOADS[name]
+    numpy_only = isinstance(spec, (workloads.LruSpec, workloads.ShiftSpec)) or \
+        (isinstance(spec, workloads.WkvSpec) and spec.gated)
+    cores = 1 if (nthreads == 1 or numpy_only) else oracle.max_threads()
+    return {"value": n * reps / dt, "cores": cores,
+            "sample": f"{desc}, {reps} passes, float64 RNN-mode oracle", "seconds": dt}
+
+
+def cpu_baseline(name, seconds):
+    """The float64 oracle on all of this host's cores, and on one core."""
+    allc = _time_oracle(name, seconds, 0)
+    one = _time_oracle(name, seconds, 1)
+    return {"value": allc["value"], "unit": "elem/s", "cores": allc["cores"],
+            "kind": "oracle", "sample": allc["sample"], "seconds": allc["seconds"],
+            "cpu": cpu_model(),
+            "one_core": {"value": one["value"], "unit": "elem/s", "cores": 1,
+                         "sample": one["sample"], "seconds": one["seconds"]}}
 
 
 def run_reference(args):
@@ -741,15 +829,18 @@ def main(argv=None):
     host_us = host_overhead_us(torch, wl)
 
     barrier()
+    if sampler is not None:
+        sampler.fast(True)
+        time.sleep(0.01)
     t_timed0 = time.time()
     if graphs is not None:
         total_ms, per = graphs.run()
     else:
         total_ms, per = time_steps(torch, wl, args.steps)
-    barrier()
     t_timed1 = time.time()
+    barrier()
     if sampler is not None:
-        time.sleep(0.25)
+        sampler.fast(False)
         sampler.stop()
     wkv.wkv_device_status()   # raises if a device-side wait gave up
 
@@ -804,7 +895,8 @@ def main(argv=None):
         "e2e": e2e,
         "gpu_launches": args.steps * wl.launches_per_step(),
         "host_us_per_call": host_us,
-        "clocks": sampler.summary(t_timed0, t_timed1) if sampler is not None else None,
+        "clocks": (sampler.summary(t_timed0, t_timed1, total_ms) if sampler is not None
+                   else None),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -36,17 +36,22 @@
  *           computes in fp32 and rounds y to nearest even; w, u stay fp32.
  * Sizes     B, T, C (D) >= 0; an empty tensor (any size 0) is a no-op.
  *           B*T*C must be < 2^62.
- * Scratch   inputs with T longer than one tile (256 steps) carry state between
- *           thread blocks through a small library-owned device workspace, one
- *           per (device, stream), allocated with cudaMalloc on first use and
- *           grown when a larger problem needs it.  Make one call of each size
- *           before capturing a stream into a CUDA graph.  Calls on different
- *           streams use different workspaces and may run concurrently.
- * Rounding  results match the operator to fp32 rounding; they are bitwise
+ * Scratch   inputs with T longer than one tile carry state between thread
+ *           blocks through a small library-owned device workspace, one per
+ *           (device, stream), allocated with cudaMalloc on first use and
+ *           grown when a larger problem needs it.  The tile length is chosen
+ *           per call (wkv_tile_steps_for() below returns it; unless
+ *           wkv_set_tile_steps() fixed it): 128 steps, or 256 for sequences
+ *           longer than 4096 steps with fewer than 64 tiles per time
+ *           segment.  Make one call of each size before capturing a stream
+ *           into a CUDA graph.  Calls on different streams use different
+ *           workspaces and may run concurrently.
+ * Rounding  results match the operator to fp32 rounding.  They are bitwise
  *           reproducible from run to run when T spans at most two tiles
- *           (256 steps).  Beyond that the carry between tiles may fold a
- *           different, equivalent set of partial results, which can move the
- *           last bits.
+ *           (256 steps at the 128-step default, 512 where the call takes
+ *           256-step tiles).  Beyond that the carry between tiles may fold
+ *           a different, equivalent set of partial results, which can move
+ *           the last bits.
  * Errors    argument errors are detected on the host before anything is
  *           launched and return a non-zero wkv_status; wkv_last_error()
  *           then describes the problem (thread-local, valid until the next

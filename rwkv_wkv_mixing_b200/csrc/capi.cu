@@ -193,6 +193,12 @@ wkv_status ensure_ws(int dev, cudaStream_t stream, size_t need, WsEntry **out, i
         return fail(WKV_ERR_OOM, "workspace of %zu bytes: %s", nb, cudaGetErrorName(err));
     }
     err = cudaMemsetAsync(p, 0, nb, stream);
+    if (err == cudaSuccess && e != nullptr && e->base != nullptr && kind == 0)
+        // a timeout recorded in the buffer being retired (and not yet read by
+        // wkv_device_status) carries over: the status word moves, in stream
+        // order, after every launch that used the old buffer
+        err = cudaMemcpyAsync(static_cast<char *>(p) + 16, e->base + 16, sizeof(int),
+                              cudaMemcpyDeviceToDevice, stream);
     if (err != cudaSuccess) {
         cudaFree(p);
         return cuda_fail(err, "cudaMemsetAsync(workspace)");

@@ -78,3 +78,29 @@ def test_host_entry_point_reports_a_timeout(m):
     m.wkv_set_fault_injection(-1, 0)
     y = m.wkv_forward_host(w, u, k, v)
     assert np.abs(y.double().numpy() - want).max() <= 1e-5 * float(np.abs(x.v).max())
+
+
+def test_a_timeout_survives_the_workspace_growing(m):
+    """A timeout recorded on a stream, then a larger call on the same stream
+    that needs a larger look-back workspace (the old one is retired): the
+    status word moves to the new workspace, so wkv_device_status still
+    reports the timeout, once."""
+    s = torch.cuda.Stream()
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to("cuda")   # noqa: E731
+    small = workloads.make_wkv("wkv_169m", B=1, T=1024, C=64, seed=103)
+    big = workloads.make_wkv("wkv_169m", B=8, T=4096, C=1024, seed=104)  # > 1 MiB of records
+    m.wkv_set_tile_steps(128)
+    with torch.cuda.stream(s):
+        m.wkv_set_fault_injection(4, 4096)
+        m.wkv_forward(d(small.w), d(small.u), d(small.k), d(small.v), stream=s)
+        m.wkv_set_fault_injection(-1, 0)
+        y = m.wkv_forward(d(big.w), d(big.u), d(big.k), d(big.v), stream=s)
+    with pytest.raises(m.WkvError) as err:
+        m.wkv_device_status(s)
+    assert err.value.status == m.WKV_ERR_TIMEOUT
+    m.wkv_device_status(s)            # read and cleared
+    # the larger call itself was not affected
+    sl = lambda a: np.ascontiguousarray(a[:, :, :64])   # noqa: E731
+    want = oracle.wkv_rnn(big.w[:64], big.u[:64], sl(big.k), sl(big.v))
+    got = y[:, :, :64].double().cpu().numpy()
+    assert np.abs(got - want).max() <= 1e-5 * float(np.abs(big.v).max())

@@ -141,6 +141,11 @@ def test_gated_full_size_3b_bf16(m):
     pts = np.concatenate([rng.integers(0, x.k.size, 1500), [0, x.k.size - 1]])
     want = oracle.sigmoid(x.r.reshape(-1)[pts]) * oracle.wkv_direct_points(x.w, x.u, x.k, x.v, pts)
     assert_close(got.reshape(-1)[pts], want, 2e-2 * scale(x.v), "gated 3b bf16 points")
+    # every output against sigma(r) times the float64 recurrence, one batch row at a time
+    for b in range(x.k.shape[0]):
+        row = lambda a: np.ascontiguousarray(a[b:b + 1])   # noqa: E731
+        want_row, _ = oracle.wkv_gated(x.w, x.u, row(x.k), row(x.v), row(x.r))
+        assert_close(got[b:b + 1], want_row, 2e-2 * scale(x.v), f"gated 3b bf16 row {b}")
 
 
 def test_gated_argument_errors(m):

@@ -3,9 +3,10 @@
 Element by element on seeded inputs at sizes the oracle finishes in seconds
 (spanning several tiles, with ragged tails and odd channel counts that take
 the element-wise copy path), and at the full workload sizes in the launch
-configuration the benchmark times: sampled outputs against the definition
-(eq. (14) of the RWKV page, or the unrolled scan sum) plus invariants checked
-over every output.
+configuration the benchmark times: every output against the float64
+recurrence (the RNN-mode form, pinned to the definition on the CPU), sampled
+outputs against the definition itself (eq. (14) of the RWKV page, or the
+unrolled scan sum), and invariants checked over every output.
 
 Tolerances: WKV fp32 max|err| <= 1e-5 max|v| (1e-4 max|v| for T >= 65536);
 WKV bf16 <= 2e-2 max|v| and, tighter, within one bf16 ulp of the oracle plus
@@ -56,6 +57,22 @@ def run_scan(m, a, b, h0):
     h = m.diag_scan(dev(a), dev(b), None if h0 is None else dev(h0))
     torch.cuda.synchronize()
     return h.double().cpu().numpy()
+
+
+def assert_full_wkv(got, x, tol, what, bf16=False, chans_per_pass=128):
+    """Every output of a [B, T, C] WKV result against oracle.wkv_rnn, a slice
+    of channels at a time so the float64 arrays stay a few hundred MB."""
+    B, T, C = x.k.shape
+    vmax = float(np.abs(x.v).max())
+    for c0 in range(0, C, chans_per_pass):
+        c1 = min(C, c0 + chans_per_pass)
+        sl = lambda a: np.ascontiguousarray(a[:, :, c0:c1])   # noqa: E731
+        want = oracle.wkv_rnn(x.w[c0:c1], x.u[c0:c1], sl(x.k), sl(x.v))
+        g = np.asarray(got[:, :, c0:c1], dtype=np.float64)
+        assert_close(g, want, tol, f"{what} channels {c0}:{c1}")
+        if bf16:   # one bf16 rounding (half an ulp) on top of the fp32 bound
+            assert np.all(np.abs(g - want) <= np.abs(want) * 2.0 ** -8 + 1e-5 * vmax), \
+                f"{what} channels {c0}:{c1}: beyond one bf16 rounding"
 
 
 def assert_close(got, want, tol, what):
@@ -354,6 +371,8 @@ def test_wkv_full_size_workload(m, name):
              torch.from_numpy(chans[cidx]).cuda()].double().cpu().numpy()
     tol = 2e-2 * vmax if x.spec.dtype == "bf16" else wkv_tol(T, vmax)
     assert_close(got, want, tol, name)
+    # every output against the float64 recurrence
+    assert_full_wkv(yf.cpu().numpy(), x, tol, name, bf16=x.spec.dtype == "bf16")
 
 
 def test_scan_full_size_workload(m):
@@ -376,6 +395,10 @@ def test_scan_full_size_workload(m):
     got = h[torch.from_numpy(b).cuda(), torch.from_numpy(t).cuda(),
             torch.from_numpy(d).cuda()].double().cpu().numpy()
     assert_close(got, want, 1e-5 * hmax, "scan_mingru")
+    # every output against the float64 recurrence
+    want_full = oracle.scan_rnn(x.a, x.b, None)
+    assert_close(h.double().cpu().numpy(), want_full, 1e-5 * float(np.abs(want_full).max()),
+                 "scan_mingru every output")
 
 
 # ---------------------------------------------------------------------------

@@ -83,6 +83,9 @@ def test_scan_bf16_full_size(m):
     want = oracle.scan_direct_points(x.a, x.b, None, pts)
     scale = float(np.abs(x.h_tilde).max())
     assert_close(got.reshape(-1)[pts], want, 2.0 ** -8 * scale, "scan bf16 full-size points")
+    # every output against the float64 recurrence over the bf16-rounded inputs
+    want_full = oracle.scan_rnn(x.a, x.b, None)
+    assert_close(got, want_full, 2.0 ** -8 * scale, "scan bf16 full-size every output")
 
 
 # ---------------------------------------------------------------------------
@@ -110,6 +113,9 @@ def test_minlstm_full_size(m):
     want = oracle.scan_direct_points(x.a, x.b, None, pts)
     assert_close(got.reshape(-1)[pts], want, 1e-5 * float(np.abs(x.h_tilde).max()),
                  "minlstm full-size points")
+    want_full = oracle.scan_rnn(x.a, x.b, None)
+    assert_close(got, want_full, 1e-5 * float(np.abs(want_full).max()),
+                 "minlstm full-size every output")
     lo = np.minimum(np.minimum.accumulate(x.h_tilde, axis=1), 0.0)
     hi = np.maximum(np.maximum.accumulate(x.h_tilde, axis=1), 0.0)
     tol = 1e-5 * float(np.abs(x.h_tilde).max())
@@ -179,6 +185,12 @@ def test_lru_full_size(m):
     want = oracle.lru_direct_points(x.nu_log, x.theta_log, x.gamma, x.u_complex(), None, pts)
     assert_close(got.reshape(-1)[pts], want, 1e-5 * float(np.abs(want).max()) + 1e-6,
                  "lru full-size points")
+    # every output against the complex128 recurrence, eight batch rows at a time
+    uc = x.u_complex()
+    for b0 in range(0, uc.shape[0], 8):
+        want_full = oracle.lru_scan(x.nu_log, x.theta_log, x.gamma, uc[b0:b0 + 8])
+        assert_close(got[b0:b0 + 8], want_full, 1e-5 * float(np.abs(want).max()) + 1e-6,
+                     f"lru full-size every output, rows {b0}:{b0 + 8}")
 
 
 def test_lru_argument_errors(m):

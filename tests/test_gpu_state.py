@@ -249,8 +249,9 @@ def test_full_size_wkv_long_from_a_state(m):
     want = oracle.wkv_direct_points(x.w, x.u, x.k, x.v, pts, s_in=s_in)
     tol = 1e-4 * scale(x.v, s_in)
     assert_close(y.reshape(-1)[pts], want, tol, "wkv_long state points")
-    _, want_s = oracle.wkv_rnn_state(x.w, x.u, x.k, x.v, s_in)
+    want_y, want_s = oracle.wkv_rnn_state(x.w, x.u, x.k, x.v, s_in)
     assert_state_close(s_out, want_s, tol, "wkv_long final")
+    assert_close(y, want_y, tol, "wkv_long state every output")
 
 
 def test_decode_workload_vs_oracle(m):

@@ -4,10 +4,12 @@ a plugin interface that hands an operator only its inputs and outputs, a
 latency-critical path that must not pay for cudaMalloc or the synchronisation
 it can cause).  Its scratch is a fixed device array shared by every call.
 
-Checked through the C ABI against the allocating entry point, wkv_forward, on
-two calls in a row (the second call must clean up after the first).  Named to
-be collected last, and written to pass both alone in a fresh process and after
-the other tests.
+Checked through the C ABI on two calls in a row (the second call must clean
+up after the first), each against the float64 oracle (the RNN-mode
+recurrence of eq. (14) of "RWKV：基于RNN的LLM") at the fp32 tolerance
+1e-5 * max|v|, and against the allocating entry point, wkv_forward, at the
+same tolerance.  Named to be collected last, and written to pass both alone
+in a fresh process and after the other tests.
 """
 import ctypes
 
@@ -15,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
 
 pytestmark = pytest.mark.gpu
@@ -37,9 +40,10 @@ def _dev(a):
 @pytest.mark.parametrize("B,T,C", [(2, 1000, 96),    # chained tiles, TMA path
                                    (3, 700, 33),     # chained tiles, element-wise path
                                    (1, 100, 64)])    # one tile in time, no scratch
-def test_noalloc_matches_allocating_entry_point_twice(lib, B, T, C):
+def test_noalloc_matches_oracle_and_allocating_entry_point_twice(lib, B, T, C):
     x = workloads.make_wkv("wkv_169m", B=B, T=T, C=C, seed=B * 7 + T + C)
     w, u, k, v = _dev(x.w), _dev(x.u), _dev(x.k), _dev(x.v)
+    want = oracle.wkv_rnn(x.w, x.u, x.k, x.v)   # float64, computed on the CPU
     ref = lib.wkv_forward(w, u, k, v)
     torch.cuda.synchronize()
     tol = 1e-5 * float(np.abs(x.v).max())
@@ -51,8 +55,11 @@ def test_noalloc_matches_allocating_entry_point_twice(lib, B, T, C):
                                          ctypes.c_void_p(stream.cuda_stream))
         assert st == lib.WKV_OK, lib.wkv_last_error()
         torch.cuda.synchronize()
+        got = y.double().cpu().numpy()
+        err = float(np.abs(got - want).max())
+        assert err <= tol, f"call {call}: max err vs the oracle {err} > {tol}"
         err = float((y.double() - ref.double()).abs().max())
-        assert err <= tol, f"call {call}: max err {err} > {tol}"
+        assert err <= tol, f"call {call}: max err vs wkv_forward {err} > {tol}"
 
 
 def test_noalloc_rejects_a_problem_beyond_its_scratch(lib):
