@@ -155,6 +155,8 @@ class ClockSampler:
         self.source = None
         self._fast = False
         self._stop = False
+        self._wake = threading.Event()   # set to cut a slow-mode sleep short
+        self._took = threading.Event()   # set by the poller after each sample
         self.fast_s = fast_s
         self.thread = None
         try:
@@ -208,7 +210,12 @@ class ClockSampler:
                                      [n for n, b in zip(self.NAMES, self.bits) if r & b]))
             except Exception:
                 pass
-            time.sleep(self.fast_s if self._fast else 0.1)
+            self._took.set()
+            if self._fast:
+                time.sleep(self.fast_s)
+            else:
+                self._wake.wait(0.1)
+                self._wake.clear()
 
     def _read_smi(self):
         for line in self.proc.stdout:
@@ -224,10 +231,17 @@ class ClockSampler:
                                   if r.lower().startswith("active")]))
 
     def fast(self, on):
+        """Switch to (or from) sampling every `fast_s`; switching on returns
+        once the poller has taken a sample in fast mode."""
         self._fast = bool(on)
+        if on and self.source == "nvml":
+            self._took.clear()
+            self._wake.set()
+            self._took.wait(1.0)
 
     def stop(self):
         self._stop = True
+        self._wake.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -831,7 +845,6 @@ def main(argv=None):
     barrier()
     if sampler is not None:
         sampler.fast(True)
-        time.sleep(0.01)
     t_timed0 = time.time()
     if graphs is not None:
         total_ms, per = graphs.run()

@@ -18,6 +18,7 @@
 #include "chunked_scan.cuh"
 #include "lru_ops.cuh"
 #include "persistent_scan.cuh"
+#include "persistent_wkv.cuh"
 #include "serial_wkv.cuh"
 #include "wkv_backward.cuh"
 #include "token_shift.cuh"
@@ -307,6 +308,10 @@ wkv_status make_plan(const typename Op::Args &args, int64_t B, int64_t T, int64_
                 !make_map(&p->maps[i], ptrs[i], dt, sizeof(io_t) / SP, B, T, C * SP, CG * SP, lt))
                 g.use_tma = 0;
     }
+    g.params_staged = 0;
+    if constexpr (StagesParams<Op>::value)
+        g.params_staged = reinterpret_cast<uintptr_t>(args.u) % 16 == 0 &&
+                          reinterpret_cast<uintptr_t>(args.w) % 16 == 0;
     std::memset(&p->ws, 0, sizeof p->ws);
     if (g.n_seg > 1) {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -391,6 +396,93 @@ wkv_status launch_persistent(const typename Op::Args &args, int64_t B, int64_t T
     return WKV_OK;
 }
 
+// fp32 WKV forward (with or without the gate) with register-resident
+// sub-chunks; shapes a tensor map describes.  Same plan and workspace as
+// launch_persistent.
+template <bool GATED, int LT, int NWG, int NC, int NSTAGE>
+wkv_status launch_persistent_wkv(const typename WkvOp<float, 1, GATED>::Args &ga, int64_t B,
+                                 int64_t T, int64_t C, CUtensorMapDataType dt, cudaStream_t stream,
+                                 int dev) {
+    using Cfg = RegWkvCfg<LT, NWG, NC, NSTAGE, GATED>;
+    using GOp = WkvOp<float, 1, GATED>;  // its Args carry r for the plan's maps
+    Plan p;
+    wkv_status st = make_plan<GOp>(ga, B, T, C, LT, dt, stream, dev, true, &p);
+    if (st != WKV_OK) return st;
+    if (!p.g.use_tma)  // a tensor map could not be made after all
+        return launch_chunked<GOp, LT, 8>(ga, B, T, C, dt, stream, dev);
+    const WkvOp<float, 1>::Args args{ga.x0, ga.x1, ga.y, ga.w, ga.u, ga.s_in, ga.s_out, ga.x2};
+    auto kern = persistent_wkv_kernel<LT, NWG, NC, NSTAGE, GATED>;
+    static std::atomic<uint64_t> configured{0};
+    if ((st = configure_once(kern, Cfg::kSmemBytes, dev, configured)) != WKV_OK) return st;
+    const int grid = std::min(p.g.tiles, sm_count(dev));
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaGetLastError();
+    cudaError_t err =
+        cudaLaunchKernelEx(&cfg, kern, p.maps[0], p.maps[1], p.maps[2], p.maps[3], args, p.g, p.ws);
+    if (err == cudaSuccess) err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
+// Compute warps per group, groups and ring stages of the register-resident
+// WKV kernel for each tile length (build-time tuning parameters; each group
+// also has a carry warp, and the block a producer warp).
+#ifndef WKV_REG_F32_64
+#define WKV_REG_F32_64 4, 3, 10
+#endif
+#ifndef WKV_REG_F32_128
+#define WKV_REG_F32_128 4, 3, 5
+#endif
+#ifndef WKV_REG_F32_256
+#define WKV_REG_F32_256 8, 1, 2
+#endif
+#ifndef WKV_REG_GATED_F32_64
+#define WKV_REG_GATED_F32_64 4, 3, 7
+#endif
+#ifndef WKV_REG_GATED_F32_128
+#define WKV_REG_GATED_F32_128 4, 3, 3
+#endif
+
+// The register-resident kernel is the faster one for fp32 problems of few
+// time segments (it measured ~6 % faster on B=8 T=1024 C=768); for bf16 and
+// for long chains of tiles the stage-resident kernel is (its four consumer
+// groups hide the carry between tiles better).
+constexpr int64_t kRegKernelMaxSegments = 16;
+
+template <bool GATED>
+wkv_status dispatch_reg_wkv(const typename WkvOp<float, 1, GATED>::Args &args, int64_t B,
+                            int64_t T, int64_t C, int lt, CUtensorMapDataType dt,
+                            cudaStream_t stream, int dev) {
+    if constexpr (GATED) {
+        switch (lt) {
+            case 64: return launch_persistent_wkv<true, 64, WKV_REG_GATED_F32_64>(args, B, T, C, dt, stream, dev);
+            default: return launch_persistent_wkv<true, 128, WKV_REG_GATED_F32_128>(args, B, T, C, dt, stream, dev);
+        }
+    } else {
+        switch (lt) {
+            case 64: return launch_persistent_wkv<false, 64, WKV_REG_F32_64>(args, B, T, C, dt, stream, dev);
+            case 256: return launch_persistent_wkv<false, 256, WKV_REG_F32_256>(args, B, T, C, dt, stream, dev);
+            default: return launch_persistent_wkv<false, 128, WKV_REG_F32_128>(args, B, T, C, dt, stream, dev);
+        }
+    }
+}
+
+// 1: the WKV forward takes the register-resident kernel (persistent_wkv.cuh)
+// where a tensor map describes the problem; 0: the stage-resident one
+#ifndef WKV_USE_REG_KERNEL
+#define WKV_USE_REG_KERNEL 1
+#endif
+
 // Steps per tile: the knob's value, or when it is 0, 128 unless a time
 // segment holds too few tiles to keep the SMs' consumer groups fed -- long
 // sequences over few rows and channels -- where 256-step tiles halve the
@@ -442,6 +534,16 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
     if constexpr (Op::NIN == 3) ptrs[nptr++] = args.x2;
     const bool tma = tma_eligible(ptrs, nptr, sizeof(typename Op::io_t), T, C);
     const int lt = tile_steps_for(B, T, C, 32 * Op::CPT);
+    if constexpr (Op::kSerialForm && sizeof(typename Op::io_t) == 4 && WKV_USE_REG_KERNEL) {
+        // the fp32 WKV forward (with or without the gate) over few time
+        // segments: register-resident sub-chunks (u and w staged with each
+        // tile by 16-byte bulk copies; three 256-step input tiles per stage
+        // do not fit twice in shared memory, so the gate keeps 64 and 128)
+        const auto al16 = [](const void *p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+        if (tma && lt >= 64 && (T + lt - 1) / lt <= kRegKernelMaxSegments && al16(args.u) &&
+            al16(args.w) && !(Op::kGated && lt == 256))
+            return dispatch_reg_wkv<Op::kGated>(args, B, T, C, lt, dt, stream, dev);
+    }
     if constexpr (Op::NIN == 3) {
         // a third input tile per stage: fewer stages and groups fit in shared memory
         switch (lt) {

@@ -25,6 +25,7 @@
 
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "scan_common.cuh"
@@ -33,18 +34,36 @@ namespace wkvb {
 
 constexpr unsigned long long kBarrierWaitNs = 4000000000ull;  // 4 s
 
+// stage waits: 0 = suspend in mbarrier try_wait; N > 0 = poll with
+// mbarrier test_wait, N ns apart
+#ifndef WKV_FILL_POLL
+#define WKV_FILL_POLL 0
+#endif
+
+// Ops whose per-channel parameters are the two fp32 arrays args.u and
+// args.w (the WKV ops) can have them staged with each tile
+template <class Op, class = void>
+struct StagesParams : std::false_type {};
+template <class Op>
+struct StagesParams<Op, std::void_t<decltype(Op::kSerialForm)>>
+    : std::bool_constant<Op::kSerialForm> {};
+
 template <class Op, int LT, int NWG, int NC, int NSTAGE>
 struct PersistentCfg {
     static constexpr int CPT = Op::CPT, NV = Op::NV, CG = 32 * CPT, LS = LT / NWG;
     static constexpr int kThreads = (1 + NC * NWG) * 32;
     static constexpr size_t kTileElems = static_cast<size_t>(LT) * CG;
-    static constexpr size_t kStageBytes = Op::NIN * kTileElems * sizeof(typename Op::io_t);
+    static constexpr bool kStaged = StagesParams<Op>::value;
+    // a stage: NIN input tiles, then (WKV) the tile's u and w, [CG] fp32 each
+    static constexpr size_t kParamOffset = Op::NIN * kTileElems * sizeof(typename Op::io_t);
+    static constexpr size_t kStageBytes = kParamOffset + (kStaged ? 2 * CG * sizeof(float) : 0);
     static constexpr size_t kSmemBytes =
         NSTAGE * kStageBytes + static_cast<size_t>(NC) * (NWG + 1) * NV * CG * sizeof(float);
     static_assert(LT % NWG == 0, "tile length must split evenly over a group's warps");
     static_assert(LT <= 256, "TMA box rows are limited to 256");
     static_assert(NSTAGE > NC, "one stage per group plus at least one being loaded");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
+    static_assert(kStageBytes % 128 == 0, "stage alignment");
     static_assert(2 + NC <= 16, "named barrier ids: 0, one per group, one for all consumers");
 };
 
@@ -82,10 +101,17 @@ __device__ __forceinline__ bool wait_fill(uint64_t *bar, const int *fill_it, int
         // (or a time limit passes), so waiting costs no issue slots; a
         // completed phase whose stamp is not ours is an older fill of the
         // stage: back off until the producer re-arms it for this iteration
+#if WKV_FILL_POLL
+        if (mbar_test_wait(bar, parity)) {
+            if (*stamp == it) return true;
+        }
+        __nanosleep(WKV_FILL_POLL);
+#else
         if (mbar_try_wait(bar, parity)) {
             if (*stamp == it) return true;
             __nanosleep(64);
         }
+#endif
         if ((n & 63u) == 63u) {
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > kBarrierWaitNs) {
@@ -111,7 +137,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
     constexpr int CPT = Cfg::CPT, NV = Cfg::NV, CG = Cfg::CG, LS = Cfg::LS;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    io_t *s_stage = reinterpret_cast<io_t *>(smem);  // [NSTAGE][NIN][LT][CG]
+    unsigned char *s_stage = smem;  // [NSTAGE] x (NIN tiles [LT][CG], then u[CG], w[CG])
     float *s_sum = reinterpret_cast<float *>(smem + NSTAGE * Cfg::kStageBytes);  // [NC][NWG][NV][CG]
     float *s_carry = s_sum + NC * NWG * NV * CG;                                   // [NC][NV][CG]
     __shared__ __align__(8) uint64_t full_bar[NSTAGE];
@@ -182,9 +208,25 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                     const int rem = tile - seg * g.tiles_per_seg;
                     const int b = rem / g.n_cg;
                     const int c0 = (rem - b * g.n_cg) * CG;
-                    io_t *dst = s_stage + static_cast<size_t>(s) * Op::NIN * Cfg::kTileElems;
+                    io_t *dst = reinterpret_cast<io_t *>(s_stage + static_cast<size_t>(s) * Cfg::kStageBytes);
                     s_last_it[s] = it;
-                    mbar_arrive_expect_tx(&full_bar[s], static_cast<uint32_t>(Cfg::kStageBytes));
+                    // the tile's u and w, channels c0 .. c0 + CG clipped to C
+                    // (C * 4 bytes is a multiple of 16 on the TMA path)
+                    uint32_t pbytes = 0;
+                    if constexpr (Cfg::kStaged)
+                        if (g.params_staged)
+                            pbytes = static_cast<uint32_t>(min(CG, g.C - c0)) *
+                                     static_cast<uint32_t>(sizeof(float));
+                    mbar_arrive_expect_tx(&full_bar[s],
+                                          static_cast<uint32_t>(Cfg::kParamOffset) + 2 * pbytes);
+                    if constexpr (Cfg::kStaged) {
+                        if (pbytes > 0) {
+                            float *dp = reinterpret_cast<float *>(
+                                s_stage + static_cast<size_t>(s) * Cfg::kStageBytes + Cfg::kParamOffset);
+                            bulk_load(dp, args.u + c0, pbytes, &full_bar[s]);
+                            bulk_load(dp + CG, args.w + c0, pbytes, &full_bar[s]);
+                        }
+                    }
                     tma_load_3d(dst, &map_x0, &full_bar[s], c0 * Op::kScalarsPerIo, seg * LT, b);
                     if constexpr (Op::NIN >= 2)
                         tma_load_3d(dst + Cfg::kTileElems, &map_x1, &full_bar[s], c0 * Op::kScalarsPerIo, seg * LT, b);
@@ -230,15 +272,36 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             const int b = rem / g.n_cg;
             const int t0 = seg * LT;
             const int c0 = (rem - b * g.n_cg) * CG;
-            io_t *s_x0 = s_stage + static_cast<size_t>(s) * Op::NIN * Cfg::kTileElems;
+            io_t *s_x0 = reinterpret_cast<io_t *>(s_stage + static_cast<size_t>(s) * Cfg::kStageBytes);
             // the second input, when there is one; never read otherwise
             const io_t *s_x1 = Op::NIN >= 2 ? s_x0 + Cfg::kTileElems : s_x0;
             // the third input (r) when there is one; never read otherwise
             const io_t *s_x2 = Op::NIN == 3 ? s_x0 + 2 * Cfg::kTileElems : s_x1;
 
             Param prm[CPT];
+            if constexpr (Cfg::kStaged) {
+                if (g.params_staged) {
+                    // staged with the tile: no global-memory round trip
+                    const float *sp = reinterpret_cast<const float *>(
+                        s_stage + static_cast<size_t>(s) * Cfg::kStageBytes + Cfg::kParamOffset);
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) prm[j] = Op::param(args, c0 + lane * CPT + j, g.C);
+                    for (int j = 0; j < CPT; ++j) {
+                        prm[j] = Param{0.f, 0.f, 1.f, 1.f};
+                        if (c0 + lane * CPT + j < g.C) {
+                            prm[j].u = sp[lane * CPT + j];
+                            prm[j].w = sp[CG + lane * CPT + j];
+                            prm[j].U = expf(prm[j].u);
+                            prm[j].D = expf(-prm[j].w);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < CPT; ++j) prm[j] = Op::param(args, c0 + lane * CPT + j, g.C);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) prm[j] = Op::param(args, c0 + lane * CPT + j, g.C);
+            }
 
             // the carry warps load the record their look-back reads first now:
             // the tile before this one in time was handed out well before it,

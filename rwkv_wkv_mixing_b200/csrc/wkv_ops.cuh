@@ -148,7 +148,7 @@ __device__ __forceinline__ float gate_sigmoid(float r) {
 // a <- a D + e v,  b <- b D + e  with per-channel constants U = e^u,
 // D = e^{-w}.  The loop-carried dependency is one FMA.  This is exact
 // arithmetic reordered; it is used when a bound shows every denominator stays
-// above 2^-100 (so nothing that matters is flushed to zero) and U is below
+// above e^-69 (so nothing that matters is flushed to zero) and U is below
 // 2^64.  Otherwise the sub-chunk takes the per-step max-stabilised update,
 // whose every exponent is <= 0 for any finite input.
 // ---------------------------------------------------------------------------
@@ -488,8 +488,10 @@ struct WkvOp {
             const float s = fast_exp(carry[j].p - M[j]);
             A[j] = carry[j].a * s;
             Bs[j] = carry[j].b * s;
-            // den_t >= e^{u + k_t - M}, and den_t >= b_in e^{p_in - M - t w}
-            const bool by_token = sc[j].kmin + q[j].u - M[j] >= -69.f;
+            // den_t >= e^{u + k_t - M} once e^{k_t - M}, evaluated on its own
+            // before the multiplication by e^u, cannot flush to zero (so
+            // k_t - M >= -69 as well when u >= 0); and den_t >= b_in e^{p_in - M - t w}
+            const bool by_token = sc[j].kmin + fminf(q[j].u, 0.f) - M[j] >= -69.f;
             const bool by_carry =
                 carry[j].b >= 1.f && carry[j].p - M[j] - static_cast<float>(n) * q[j].w >= -69.f;
             fast = fast && (by_token || by_carry) && q[j].u <= 44.f;

@@ -187,6 +187,37 @@ def test_wkv_f32_extreme_values(m):
 
 
 @pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
+def test_wkv_large_bonus_with_a_key_far_below_the_chunk_max(m, bf16):
+    """A bonus u between 18 and 44 with a sub-chunk whose first key sits 98
+    below its largest: e^{u + k - M} = e^-68 is a fine weight, but e^{k - M}
+    on its own (before the multiplication by e^u) would flush to zero, so the
+    first step of the sequence (empty past) must not take the fixed-reference
+    sweep.  Outputs finite and matching the oracle; y_0 = v_0."""
+    rng = np.random.default_rng(41)
+    B, T, C = 2, 700, 64
+    k = rng.normal(0, 1, (B, T, C))
+    k[:, ::16, :] = -68.0         # the first step of every 16- and 32-step sub-chunk
+    k[:, 1::16, :] = 30.0         # and the largest key right after it
+    v = rng.normal(0, 1, (B, T, C))
+    w = np.exp(rng.uniform(-3, 1, C))
+    u = np.concatenate([np.full(32, 30.0), rng.uniform(18, 44, C - 32)])
+    kf, vf = k.astype(np.float32), v.astype(np.float32)
+    wf, uf = w.astype(np.float32), u.astype(np.float32)
+    if bf16:
+        kb, vb = workloads.bf16_bits(kf), workloads.bf16_bits(vf)
+        y = m.wkv_forward_bf16(dev(wf), dev(uf), bf16_dev(kb), bf16_dev(vb))
+        kf, vf = workloads.bf16_bits_to_f32(kb), workloads.bf16_bits_to_f32(vb)
+    else:
+        y = m.wkv_forward(dev(wf), dev(uf), dev(kf), dev(vf))
+    torch.cuda.synchronize()
+    got = y.float().double().cpu().numpy()
+    want = oracle.wkv_rnn(wf, uf, kf, vf)
+    vmax = float(np.abs(vf).max())
+    assert_close(got, want, (2e-2 if bf16 else 1e-5) * vmax, "large bonus, far key")
+    assert np.array_equal(got[:, 0, :], vf[:, 0, :].astype(np.float64))
+
+
+@pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
 def test_wkv_chunk_whose_largest_key_decays_away(m, bf16):
     """Sub-chunks whose largest key comes first and is decayed far below the
     rest (w = 10, one key of +30 among keys of -30): summed against max k

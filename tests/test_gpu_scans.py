@@ -185,12 +185,17 @@ def test_lru_full_size(m):
     want = oracle.lru_direct_points(x.nu_log, x.theta_log, x.gamma, x.u_complex(), None, pts)
     assert_close(got.reshape(-1)[pts], want, 1e-5 * float(np.abs(want).max()) + 1e-6,
                  "lru full-size points")
-    # every output against the complex128 recurrence, eight batch rows at a time
+    # every output against the complex128 recurrence, eight batch rows at a
+    # time; the tolerance scales with the largest |x| of the whole output
     uc = x.u_complex()
+    errs, scale = [], 0.0
     for b0 in range(0, uc.shape[0], 8):
         want_full = oracle.lru_scan(x.nu_log, x.theta_log, x.gamma, uc[b0:b0 + 8])
-        assert_close(got[b0:b0 + 8], want_full, 1e-5 * float(np.abs(want).max()) + 1e-6,
-                     f"lru full-size every output, rows {b0}:{b0 + 8}")
+        assert np.all(np.isfinite(got[b0:b0 + 8])), f"rows {b0}:{b0 + 8}: non-finite output"
+        errs.append(float(np.abs(got[b0:b0 + 8] - want_full).max()))
+        scale = max(scale, float(np.abs(want_full).max()))
+    tol = 1e-5 * scale + 1e-6
+    assert max(errs) <= tol, f"lru full-size every output: max err {max(errs):.3e} > {tol:.3e}"
 
 
 def test_lru_argument_errors(m):
