@@ -78,6 +78,9 @@ def parse_args(argv=None):
                     help="steps per tile (8, 32, 64, 128, 256); 0 keeps the library default")
     ap.add_argument("--launch", default="graph", choices=["graph", "direct"],
                     help="replay the K steps from CUDA graphs (default) or call directly")
+    ap.add_argument("--shape", default=None,
+                    help="B,T,C (B,T,D for scans): the workload's distributions at another "
+                         "shape, for small profiler captures of the same kernel")
     return ap.parse_args(argv)
 
 
@@ -94,8 +97,8 @@ def read_peaks():
 # the sources the tiled WKV / scan kernels are built from (their dispatch
 # included); a recorded DRAM-traffic figure is only reported while these are
 # unchanged
-TILED_KERNEL_SOURCES = ("capi.cu", "persistent_scan.cuh", "chunked_scan.cuh", "scan_common.cuh",
-                        "wkv_ops.cuh", "ptx.cuh")
+TILED_KERNEL_SOURCES = ("capi.cu", "persistent_scan.cuh", "persistent_wkv.cuh", "chunked_scan.cuh",
+                        "scan_common.cuh", "wkv_ops.cuh", "ptx.cuh")
 
 
 def src_hash():
@@ -285,8 +288,9 @@ class DeviceWorkload:
     receptance gate), "scan" (diagonal scan), "shift" (token shift, the
     saved last token read and written in place)."""
 
-    def __init__(self, name, torch, lib, l2_bytes):
+    def __init__(self, name, torch, lib, l2_bytes, shape=None):
         self.name = name
+        sB, sT, sC = shape if shape is not None else (None, None, None)
         self.spec = spec = workloads.WORKLOADS[name]
         self.torch = torch
         self.lib = lib
@@ -296,7 +300,7 @@ class DeviceWorkload:
         self.has_state = self.gated = False
         if isinstance(spec, workloads.ScanSpec):
             self.kind = "scan"
-            x = workloads.make_scan(name)
+            x = workloads.make_scan(name, B=sB, T=sT, D=sC)
             B, T, C = x.a.shape
             bf = spec.dtype == "bf16"
             self.dtype, self.es = spec.dtype, 2 if bf else 4
@@ -306,7 +310,7 @@ class DeviceWorkload:
             alg = 3 * self.es * B * T * C
         elif isinstance(spec, workloads.LruSpec):
             self.kind = "lru"
-            x = workloads.make_lru(name)
+            x = workloads.make_lru(name, B=sB, T=sT, D=sC)
             B, T, C = x.u.shape[:3]
             self.dtype, self.es = "c64", 8
             self.host = {"u": x.u}
@@ -316,7 +320,7 @@ class DeviceWorkload:
             alg = 16 * B * T * C + 12 * C
         elif isinstance(spec, workloads.ShiftSpec):
             self.kind = "shift"
-            x = workloads.make_token_shift(name)
+            x = workloads.make_token_shift(name, B=sB, T=sT, C=sC)
             B, T, C = x.x.shape
             bf = spec.dtype == "bf16"
             self.dtype, self.es = spec.dtype, 2 if bf else 4
@@ -328,7 +332,7 @@ class DeviceWorkload:
             alg = self.es * B * T * C * (1 + self.n_mix) + 2 * self.es * B * C + 4 * self.n_mix * C
         else:
             self.kind = "wkv"
-            x = workloads.make_wkv(name)
+            x = workloads.make_wkv(name, B=sB, T=sT, C=sC)
             B, T, C = x.k.shape
             bf = spec.dtype == "bf16"
             self.dtype, self.es = spec.dtype, 2 if bf else 4
@@ -430,8 +434,12 @@ class DeviceWorkload:
             return "wkv_bwd_* (six kernels per step, timed together)"
         if self.kind == "wkv" and self.T <= 16:
             return "wkv_serial_kernel"
-        if self.lib.wkv_tile_steps_for(self.B, self.T, self.C, self.es) in (8, 32):
+        lt = self.lib.wkv_tile_steps_for(self.B, self.T, self.C, min(self.es, 4))
+        if lt in (8, 32):
             return "chunked_scan_kernel"
+        if self.kind == "wkv" and self.dtype == "f32" and -(-self.T // lt) <= 16 and \
+                not (self.gated and lt == 256):
+            return "persistent_wkv_kernel"
         return "persistent_scan_kernel"
 
     def step(self, i):
@@ -808,7 +816,10 @@ def main(argv=None):
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
     if args.tile_steps:
         wkv.wkv_set_tile_steps(args.tile_steps)
-    wl = DeviceWorkload(args.workload, torch, wkv.lib, l2)
+    shape = tuple(int(v) for v in args.shape.split(",")) if args.shape else None
+    if shape is not None and len(shape) != 3:
+        raise SystemExit("--shape takes three integers: B,T,C")
+    wl = DeviceWorkload(args.workload, torch, wkv.lib, l2, shape)
 
     def barrier():
         torch.cuda.synchronize()
@@ -883,6 +894,9 @@ def main(argv=None):
 
     spec = wl.spec
     cfg = workload_config(spec, args.workload)
+    if shape is not None:
+        cfg.update({"B": wl.B, "T": wl.T, ("D" if "D" in cfg else "C"): wl.C,
+                    "shape": "overridden by --shape (not the named workload's size)"})
     cfg.update({"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                 "l2": (f"inputs rotate over {wl.n_sets} buffer sets "
                        f"({wl.n_sets * wl.set_bytes / 1e6:.0f} MB > L2 "
