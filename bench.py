@@ -421,17 +421,20 @@ class DeviceWorkload:
         return fn(B, T, C, w, u, d["k"].data_ptr(), d["v"].data_ptr(), d["y"].data_ptr(), sh)
 
     def launches_per_step(self):
-        """Kernels one step launches: the gradient path runs six (segment
-        summaries, carries, outputs, reverse carries, gradients, reduction),
+        """Kernels one step launches: the gradient path runs four when a
+        tensor map describes its rows (forward states and reverse segment
+        summaries, reverse carries, gradients, reduction), six otherwise;
         every other path one."""
-        return 6 if self.kind == "bwd" else 1
+        if self.kind == "bwd":
+            return 4 if (self.C * 4) % 16 == 0 else 6
+        return 1
 
     def kernel(self):
         """The dominant kernel a step launches (the library's dispatch rule)."""
         if self.kind == "shift":
             return "token_shift_kernel"
         if self.kind == "bwd":
-            return "wkv_bwd_* (six kernels per step, timed together)"
+            return ("wkv_bwd_* (%d kernels per step, timed together)" % self.launches_per_step())
         if self.kind == "wkv" and self.T <= 16:
             return "wkv_serial_kernel"
         lt = self.lib.wkv_tile_steps_for(self.B, self.T, self.C, min(self.es, 4))

@@ -210,13 +210,21 @@ WKV_API wkv_status diag_scan(int64_t B, int64_t T, int64_t D,
  *     gv_j = sum_{t>=j} gy_t beta_{t,j},   gk_j = sum_{t>=j} gy_t beta_{t,j} (v_j - y_t),
  *     gu   = sum_t gy_t beta_{t,t} (v_t - y_t),
  *     gw   = -sum_t sum_{j<t} (t-1-j) gy_t beta_{t,j} (v_j - y_t).
- * Time-parallel over segments of 16 steps (six launches: forward segment
- * summaries, forward carries, reverse segment summaries, reverse carries,
- * gradients, the gw/gu reduction), recomputing the forward outputs per
+ * Time-parallel over segments of steps, recomputing the forward outputs per
  * segment and running the sums over later outputs backwards in time,
- * max-stabilised (every exponent <= 0 for finite inputs); gw and gu are
- * reduced over rows and segments in a fixed order, so results do not depend
- * on timing.  Scratch (40 bytes per row, segment and channel, plus 64 bytes
+ * max-stabilised (every exponent <= 0 for finite inputs).  When every
+ * pointer is 16-byte aligned and C is a multiple of 4 (rows a tensor map
+ * can describe): 32-step segments in four launches (forward states and
+ * reverse segment summaries, with the forward state carried between
+ * 128-step tiles by the decoupled look-back of the forward kernel; reverse
+ * carries; gradients; the gw/gu reduction), k, v, gy read twice.  Otherwise
+ * 16-step segments in six launches (forward segment summaries, forward
+ * carries, reverse segment summaries, reverse carries, gradients, the
+ * reduction), k, v read three times.  gw and gu are reduced over rows and
+ * segments in a fixed order.  Results are bitwise reproducible on the
+ * six-launch path and, on the four-launch path, up to two 128-step tiles;
+ * beyond that reproducible to rounding (the look-back may fold the forward
+ * carry from different predecessors from run to run).  Scratch (40 bytes per row, segment and channel, plus 64 bytes
  * per channel and a counter per 32 channels) is library-owned per-stream
  * memory, allocated on first use like the look-back workspace (make one call
  * of each size before stream capture).

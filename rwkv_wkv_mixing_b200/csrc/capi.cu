@@ -17,6 +17,7 @@
 
 #include "chunked_scan.cuh"
 #include "lru_ops.cuh"
+#include "persistent_bwd.cuh"
 #include "persistent_scan.cuh"
 #include "persistent_wkv.cuh"
 #include "serial_wkv.cuh"
@@ -477,6 +478,20 @@ wkv_status dispatch_reg_wkv(const typename WkvOp<float, 1, GATED>::Args &args, i
     }
 }
 
+// Warps per group, groups and ring stages of the stage-resident kernel for
+// 128-step tiles of two inputs (build-time tuning parameters): bf16 WKV (two
+// channels a thread), everything else
+#ifndef WKV_PS_128_BF16
+#define WKV_PS_128_BF16 4, 4, 6
+#endif
+#ifndef WKV_PS_128
+#define WKV_PS_128 4, 4, 6
+#endif
+template <class Op, class = void>
+struct PackedIo : std::false_type {};
+template <class Op>
+struct PackedIo<Op, std::void_t<decltype(Op::kPacked)>> : std::bool_constant<Op::kPacked> {};
+
 // 1: the WKV forward takes the register-resident kernel (persistent_wkv.cuh)
 // where a tensor map describes the problem; 0: the stage-resident one
 #ifndef WKV_USE_REG_KERNEL
@@ -570,8 +585,12 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
                 return tma ? launch_persistent<Op, 256, 8, 2, 3>(args, B, T, C, dt, stream, dev)
                            : launch_chunked<Op, 256, 8>(args, B, T, C, dt, stream, dev);
             default:
-                return tma ? launch_persistent<Op, 128, 4, 4, 6>(args, B, T, C, dt, stream, dev)
-                           : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
+                if constexpr (PackedIo<Op>::value)
+                    return tma ? launch_persistent<Op, 128, WKV_PS_128_BF16>(args, B, T, C, dt, stream, dev)
+                               : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
+                else
+                    return tma ? launch_persistent<Op, 128, WKV_PS_128>(args, B, T, C, dt, stream, dev)
+                               : launch_chunked<Op, 128, 8>(args, B, T, C, dt, stream, dev);
         }
     }
 }
@@ -953,6 +972,119 @@ wkv_status wkv_host_common(int64_t B, int64_t T, int64_t C, const float *w, cons
     return run_host<Op>(B, T, C, k, v, y, w, u, nullptr, dt, &wkv_host_args<IO>);
 }
 
+// ---- WKV gradients on the tiled path (persistent_bwd.cuh) -------------------------
+// 1: shapes a tensor map describes take the tiled gradient kernels; 0: every
+// shape takes the per-segment kernels of wkv_backward.cuh
+#ifndef WKV_BWD_TILED
+#define WKV_BWD_TILED 1
+#endif
+// states kernel: 128-step tiles, three groups of four compute warps (one
+// 32-step segment each) and a carry warp, three stages; gradients kernel:
+// eleven compute warps (168 registers: three warps per SM sub-partition),
+// sixteen 32-step stages of k, v and gy
+#ifndef WKV_BWD_STATES_CFG
+#define WKV_BWD_STATES_CFG 128, 4, 3, 3
+#endif
+#ifndef WKV_BWD_GRADS_CFG
+#define WKV_BWD_GRADS_CFG 11, 16
+#endif
+using BwdStates = BwdStatesCfg<WKV_BWD_STATES_CFG>;
+using BwdGrads = BwdGradsCfg<WKV_BWD_GRADS_CFG>;
+constexpr int kBwdStatesLT = BwdStates::kLT;
+
+Geometry bwd_geometry(int64_t B, int64_t T, int64_t C, int lt) {
+    Geometry g{};
+    g.B = static_cast<int>(B);
+    g.T = static_cast<int>(T);
+    g.C = static_cast<int>(C);
+    g.n_cg = static_cast<int>((C + 31) / 32);
+    g.n_seg = static_cast<int>((T + lt - 1) / lt);
+    g.tiles_per_seg = static_cast<int>(B * g.n_cg);
+    g.tiles = g.n_seg * g.tiles_per_seg;
+    g.use_tma = 1;
+    g.spin_limit = g_fault_spin_limit.load() > 0 ? g_fault_spin_limit.load() : kSpinLimit;
+    g.skip_publish = g_fault_skip_tile.load();
+    g.params_staged = 1;
+    return g;
+}
+
+template <typename K, typename... A>
+wkv_status launch_pdl(K kern, int grid, int threads, size_t smem, cudaStream_t stream, A... args) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaGetLastError();
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (err == cudaSuccess) err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
+// The four launches of one gradient step on the tiled path, or *done = false
+// (nothing launched) when a tensor map cannot be made for these buffers.
+wkv_status launch_bwd_tiled(const WkvBwdArgs &a, int64_t B, int64_t T, int64_t C,
+                            cudaStream_t stream, int dev, bool *done) {
+    *done = false;
+    const auto dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    // [0..2] k, v, gy in 128-step boxes (states kernel); [3..7] k, v, gy, gk,
+    // gv in 32-step boxes (gradients kernel)
+    CUtensorMap m[8];
+    std::memset(m, 0, sizeof m);
+    const void *src[8] = {a.k, a.v, a.gy, a.k, a.v, a.gy, a.gk, a.gv};
+    for (int i = 0; i < 8; ++i)
+        if (!make_map(&m[i], src[i], dt, sizeof(float), B, T, C, 32,
+                      i < 3 ? kBwdStatesLT : kBwdSegSteps))
+            return WKV_OK;
+    const Geometry gs = bwd_geometry(B, T, C, kBwdStatesLT);
+    Geometry gg = bwd_geometry(B, T, C, kBwdSegSteps);
+    gg.skip_publish = -1;
+    // the look-back workspace of this stream (its status word reports the
+    // timeouts of both persistent kernels)
+    Workspace ws;
+    std::memset(&ws, 0, sizeof ws);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        WsEntry *e = nullptr;
+        wkv_status st = ensure_ws(dev, stream, ws_bytes(static_cast<size_t>(gs.tiles), 32), &e);
+        if (st != WKV_OK) return st;
+        ws.ticket = reinterpret_cast<unsigned int *>(e->base);
+        ws.done = reinterpret_cast<unsigned int *>(e->base + 4);
+        ws.epoch = reinterpret_cast<unsigned long long *>(e->base + 8);
+        ws.status = reinterpret_cast<int *>(e->base + 16);
+        ws.records = reinterpret_cast<uint4 *>(e->base + kWsHeader);
+    }
+    const BwdTileArgs ta{a.w, a.u, a.k, a.v, a.fwd, a.rev, a.partial, a.S};
+    auto ks = wkv_bwd_states_kernel<WKV_BWD_STATES_CFG>;
+    auto kg = wkv_bwd_grads_tiles_kernel<WKV_BWD_GRADS_CFG>;
+    static std::atomic<uint64_t> conf_s{0}, conf_g{0};
+    wkv_status st = configure_once(ks, BwdStates::kSmemBytes, dev, conf_s);
+    if (st == WKV_OK) st = configure_once(kg, BwdGrads::kSmemBytes, dev, conf_g);
+    if (st != WKV_OK) return st;
+    *done = true;
+    const int sms = sm_count(dev);
+    if ((st = launch_pdl(ks, std::min(gs.tiles, sms), BwdStates::kThreads, BwdStates::kSmemBytes,
+                         stream, m[0], m[1], m[2], ta, gs, ws)) != WKV_OK)
+        return st;
+    const int64_t n_cg = (C + 31) / 32;
+    wkv_bwd_rev_carry_kernel<<<static_cast<unsigned>(B * n_cg), 32 * kCarryWarps, 0, stream>>>(a);
+    if ((st = launch_pdl(kg, std::min(gg.tiles, sms), BwdGrads::kThreads, BwdGrads::kSmemBytes,
+                         stream, m[3], m[4], m[5], m[6], m[7], ta, gg, ws)) != WKV_OK)
+        return st;
+    wkv_bwd_reduce_kernel<<<static_cast<unsigned>(n_cg * kReduceParts), 32 * kReduceWarps, 0,
+                            stream>>>(a);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return WKV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1095,8 +1227,14 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const f
             if (overlaps(out[i].p, out[i].bytes, out[j].p, out[j].bytes))
                 return fail(WKV_ERR_INVALID_ARG, "%s overlaps %s", out[i].name, out[j].name);
     }
-    const int64_t S = (T + kSeg - 1) / kSeg;
-    const int64_t seg_threads = B * S * C;
+    // tiled path: every buffer 16-byte aligned, rows of a multiple of 16 bytes
+    const void *tptrs[7] = {k, v, gy, gk, gv, u, w};
+    const bool tiled = WKV_BWD_TILED && tma_eligible(tptrs, 7, sizeof(float), T, C);
+    // segments of kSeg steps for the per-segment kernels, kBwdSegSteps on the
+    // tiled path; the scratch is sized for the shorter ones, so a call that
+    // meant to go tiled can still take the per-segment kernels
+    const int64_t S16 = (T + kSeg - 1) / kSeg;
+    const int64_t seg_threads = B * S16 * C;
     if ((seg_threads + kBwdThreads - 1) / kBwdThreads > INT32_MAX)
         return fail(WKV_ERR_INVALID_ARG, "B*C*T too large for one launch");
     // scratch per (row, segment, channel): the forward (3) and reverse (5)
@@ -1105,7 +1243,7 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const f
     // have a workspace of their own: zero when allocated, and every launch
     // leaves them at zero.
     const int64_t n_cg = (C + 31) / 32;
-    const size_t ns = static_cast<size_t>(B) * S * C;
+    const size_t ns = static_cast<size_t>(B) * S16 * C;
     const size_t nred = static_cast<size_t>(kReduceParts) * 2 * C;
     WsEntry *e = nullptr, *ce = nullptr;
     {
@@ -1120,7 +1258,15 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float *w, const f
     WkvBwdArgs a{w, u, k, v, gy, gk, gv, scratch, scratch + 3 * ns, scratch + 8 * ns, gw, gu,
                  scratch + 10 * ns, reinterpret_cast<unsigned *>(ce->base),
                  static_cast<int>(B), static_cast<int>(T), static_cast<int>(C),
-                 static_cast<int>(S)};
+                 static_cast<int>(S16), kSeg};
+    if (tiled) {
+        WkvBwdArgs at = a;
+        at.L = kBwdSegSteps;
+        at.S = static_cast<int>((T + kBwdSegSteps - 1) / kBwdSegSteps);
+        bool done = false;
+        if ((st = launch_bwd_tiled(at, B, T, C, stream, dev, &done)) != WKV_OK || done) return st;
+        // no tensor map for these buffers after all: the per-segment kernels
+    }
     const unsigned g_seg = static_cast<unsigned>((seg_threads + kBwdThreads - 1) / kBwdThreads);
     const unsigned g_chan = static_cast<unsigned>(B * n_cg);
     const unsigned g_red = static_cast<unsigned>(n_cg * kReduceParts);

@@ -41,6 +41,12 @@
 // (A single-pass form, segments chained by a decoupled look-back in each
 // direction, measured slower at these segment lengths: the look-back's
 // latency outweighs a 16- or 32-step segment's work.)
+//
+// These six kernels serve the shapes a TMA tensor map cannot describe.  The
+// others take persistent_bwd.cuh: 32-step segments whose forward states and
+// reverse summaries come from one pass over TMA-staged 128-step tiles, then
+// the reverse carries and the reduction below (segment length a.L), then
+// one TMA-staged gradient pass (k, v, gy read twice instead of three times).
 #pragma once
 
 #include "wkv_ops.cuh"
@@ -62,7 +68,8 @@ struct WkvBwdArgs {
     float *gw, *gu;           // [C]
     float *red;               // scratch [kReduceParts, 2, C]: first-level sums of gw, gu
     unsigned *red_done;       // [ceil(C / 32)] counters, zero between launches
-    int B, T, C, S;           // S = ceil(T / kSeg) segments per row
+    int B, T, C, S;           // S = ceil(T / L) segments per row
+    int L;                    // steps per segment: kSeg here, 32 on the tiled path
 };
 
 // forward state: (num, den) = (a, d) e^p of the sums over the steps before
@@ -131,7 +138,7 @@ __device__ __forceinline__ bool seg_thread(const WkvBwdArgs &a, int &b, int &s, 
 }
 
 __device__ __forceinline__ int seg_len(const WkvBwdArgs &a, int s) {
-    return min(a.T, (s + 1) * kSeg) - s * kSeg;
+    return min(a.T, (s + 1) * a.L) - s * a.L;
 }
 
 // one reverse step over output j: (P, Q) take g_j / D_j and g_j y_j / D_j,
@@ -240,7 +247,7 @@ __device__ __forceinline__ void carry_range(const WkvBwdArgs &a, int &lo, int &h
     const int wi = threadIdx.x / 32;
     lo = static_cast<int>(static_cast<long long>(a.S) * wi / kCarryWarps);
     hi = static_cast<int>(static_cast<long long>(a.S) * (wi + 1) / kCarryWarps);
-    steps = hi > lo ? min(a.T, hi * kSeg) - lo * kSeg : 0;
+    steps = hi > lo ? min(a.T, hi * a.L) - lo * a.L : 0;
 }
 
 // 2. the forward state before each segment

@@ -50,8 +50,13 @@ def compare(m, x, gy, what, sums_rel=2e-4):
         check(g, wv, rel, f"{what} {name}")
 
 
+# C = 33 and 130 (rows not a multiple of 16 bytes) take the per-segment
+# kernels; the others the tiled ones (128-step tiles, 32-step segments):
+# one segment, one partial tile, several tiles with ragged tails in time
+# and channels, long chains
 SHAPES = [(1, 1, 4), (2, 5, 32), (2, 64, 40), (3, 300, 33), (1, 1024, 64), (4, 700, 130),
-          (1, 4100, 40), (2, 257, 96)]
+          (1, 4100, 40), (2, 257, 96), (1, 31, 8), (2, 129, 36), (1, 128, 32), (3, 2000, 100),
+          (2, 4129, 64)]
 
 
 @pytest.mark.parametrize("B,T,C", SHAPES)
