@@ -42,9 +42,11 @@ namespace wkvb {
 constexpr int kBwdSegSteps = 32;  // steps per segment: one compute warp's share of a tile
 
 // 1: a gradients warp hands a stage back after its next tile's stores are
-// issued; 0: it waits for its stores to read the stage at once
+// issued; 0: it waits for its stores to read the stage at once (measured
+// faster: 62 against 67 us a gradient step on B=8 T=1024 C=768 -- a warp
+// holding two stages of the in-order ring stalls the producer)
 #ifndef WKV_BWD_DEFER_RELEASE
-#define WKV_BWD_DEFER_RELEASE 1
+#define WKV_BWD_DEFER_RELEASE 0
 #endif
 
 struct BwdTileArgs {
@@ -92,58 +94,102 @@ struct BwdStatesCfg {
     static_assert(2 + kBarsPerGroup * NC <= 16, "named barrier ids: 0, per group, one for all");
 };
 
-// y_t and ln D_t of the segment from the state before it, in place of the
-// weights and values in R (R.e[i] <- y_i, R.v[i] <- ln D_i).  The fixed
-// reference M = max(p_in, max k) of the forward kernel's pass 2 when its
-// bound holds (D_t = (b_t + e_t e^u) e^M with every denominator above
-// e^-69); otherwise the per-step max-stabilised form, keys and values read
-// back from global memory (kp[i * C], vp[i * C]; zeros when the channel does
-// not exist).
+// The reverse sums over a segment's own outputs can run at the forward
+// pass's fixed reference M: with D_t = den_t e^M, each output enters them as
+// g_t e^{-L_t} = g_t r_t e^{-M}, r_t = 1 / den_t, so sums kept in units of
+// e^{-M} need no exponential at all.  Safe when every den_t >= e^-30 (the
+// forward bound at that floor): then r_t <= e^30 and no sum of a segment's
+// terms can overflow for |g|, |v| below 1e15.
+constexpr float kRevFixedFloor = -30.f;
+
+// y_t of the segment from the state before it, in place of the weights in R
+// (R.e[i] <- y_i).  Returns true when the segment takes the fixed reference
+// M = max(p_in, max k) of the forward kernel's pass 2 with every denominator
+// above e^-30: then R.v[i] <- r_i = 1 / den_i.  Otherwise R.v[i] <- ln D_i:
+// at the same reference when the forward kernel's own bound (e^-69) holds,
+// else from the per-step max-stabilised form, keys and values read back from
+// global memory (batch row b, rows t.., channel c; zeros when the channel
+// does not exist).
 template <int LS, bool FULL>
-__device__ __forceinline__ void rows_forward_outputs(LaneRows<LS> &R,
+__device__ __forceinline__ bool rows_forward_outputs(LaneRows<LS> &R,
                                                      const WkvOp<float, 1>::State &cin, int n,
                                                      const WkvOp<float, 1>::Param &q,
-                                                     const float *kp, const float *vp, size_t C,
-                                                     bool cvalid) {
-    const float M = fmaxf(cin.p, R.kmax);
+                                                     const BwdTileArgs &a, const Geometry &g,
+                                                     int b, int t, int c, float &M) {
+    M = fmaxf(cin.p, R.kmax);
     if (sweep_is_safe(R.kmin, M, cin, q, n)) {
+        const bool rev_fixed = sweep_is_safe(R.kmin, M, cin, q, n, kRevFixedFloor);
         const float s = fast_exp(R.kmax - M), f = fast_exp(cin.p - M);
         float A = cin.a * f, Bs = cin.b * f;
+        if (rev_fixed) {
 #pragma unroll
-        for (int i = 0; i < LS; ++i)
-            if (FULL || i < n) {
-                const float e = R.e[i] * s, v = R.v[i];
-                const float den = fmaf(e, q.U, Bs);
-                const float y = v + fmaf(-Bs, v, A) * rcp_approx(den);
-                A = fmaf(A, q.D, e * v);
-                Bs = fmaf(Bs, q.D, e);
-                R.e[i] = y;
-                R.v[i] = M + __logf(den);
-            }
-    } else {
-        FwdState st{cin.a, cin.b, cin.p};
+            for (int i = 0; i < LS; ++i)
+                if (FULL || i < n) {
+                    const float e = R.e[i] * s, v = R.v[i];
+                    const float r = rcp_approx(fmaf(e, q.U, Bs));
+                    R.e[i] = v + fmaf(-Bs, v, A) * r;
+                    R.v[i] = r;
+                    A = fmaf(A, q.D, e * v);
+                    Bs = fmaf(Bs, q.D, e);
+                }
+        } else {
 #pragma unroll
-        for (int i = 0; i < LS; ++i)
-            if (FULL || i < n) {
-                const float k = cvalid ? kp[i * C] : 0.f, v = cvalid ? vp[i * C] : 0.f;
-                const Pair f = max_pair(st.p, q.u + k);
-                const float den = fmaf(f.fx, st.d, f.fy);  // in [1, T + 1]
-                R.e[i] = fmaf(f.fx, st.a, f.fy * v) * __fdividef(1.f, den);
-                R.v[i] = f.q + __logf(den);
-                fwd_step(st, k, v, q.w);
-            }
+            for (int i = 0; i < LS; ++i)
+                if (FULL || i < n) {
+                    const float e = R.e[i] * s, v = R.v[i];
+                    const float den = fmaf(e, q.U, Bs);
+                    R.e[i] = v + fmaf(-Bs, v, A) * rcp_approx(den);
+                    R.v[i] = M + __logf(den);
+                    A = fmaf(A, q.D, e * v);
+                    Bs = fmaf(Bs, q.D, e);
+                }
+        }
+        return rev_fixed;
     }
+    // the rare path: keys and values of rows t.. of batch row b, channel c
+    const size_t C = static_cast<size_t>(g.C);
+    const bool cvalid = c < g.C;
+    const size_t row0 = (static_cast<size_t>(b) * g.T + t) * C + (cvalid ? c : 0);
+    const float *kp = a.k + row0, *vp = a.v + row0;
+    FwdState st{cin.a, cin.b, cin.p};
+#pragma unroll
+    for (int i = 0; i < LS; ++i)
+        if (FULL || i < n) {
+            const float k = cvalid ? kp[i * C] : 0.f, v = cvalid ? vp[i * C] : 0.f;
+            const Pair f = max_pair(st.p, q.u + k);
+            const float den = fmaf(f.fx, st.d, f.fy);  // in [1, T + 1]
+            R.e[i] = fmaf(f.fx, st.a, f.fy * v) * __fdividef(1.f, den);
+            R.v[i] = f.q + __logf(den);
+            fwd_step(st, k, v, q.w);
+        }
+    return false;
 }
 
-// the segment's reverse summary from the zero state: R holds y_t, ln D_t,
-// gp[i * 32] the upstream gradient g_t
+// The segment's reverse summary from the zero state: R holds y_t and, at the
+// fixed reference M, r_t (the sums come out in units of e^{-M}: rho = M);
+// otherwise ln D_t, and the per-step min-stabilised steps.  gp[i * 32]: the
+// upstream gradient g_t.
 template <int LS, bool FULL>
 __device__ __forceinline__ RevState rows_reverse_summary(const LaneRows<LS> &R, const float *gp,
-                                                         int n, float w) {
+                                                         int n, const WkvOp<float, 1>::Param &q,
+                                                         bool fixed, float M) {
+    if (fixed) {
+        float P = 0.f, Q = 0.f, Rs = 0.f, R2 = 0.f;
+#pragma unroll
+        for (int i = LS - 1; i >= 0; --i)
+            if (FULL || i < n) {
+                const float gr = gp[i * 32] * R.v[i];
+                Rs = q.D * (Rs + P);
+                R2 = q.D * (R2 + Q);
+                P = fmaf(q.D, P, gr);
+                Q = fmaf(q.D, Q, gr * R.e[i]);
+            }
+        return {P, Q, Rs, R2, M};
+    }
     RevState z{0.f, 0.f, 0.f, 0.f, -kNoScale};
 #pragma unroll
     for (int i = LS - 1; i >= 0; --i)
-        if (FULL || i < n) rev_step(z, gp[i * 32], R.e[i], R.v[i], w);
+        if (FULL || i < n) rev_step(z, gp[i * 32], R.e[i], R.v[i], q.w);
     return z;
 }
 
@@ -435,27 +481,28 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
                 // pass 2: the forward state before the segment, y_t and ln D_t,
                 // and the segment's reverse summary, to the scratch
                 if (nval > 0) {
-                    const bool cvalid = c < g.C;
-                    const size_t C = static_cast<size_t>(g.C);
-                    const size_t bs = static_cast<size_t>(b) * a.S + (t0 + s0) / LS;
-                    if (cvalid) {
-                        float *f = a.fwd + bs * 3 * C + c;
+                    // segment (b, (t0 + s0) / LS) of the scratch
+                    const int segi = b * a.S + (t0 + s0) / LS;
+                    if (c < g.C) {
+                        const size_t C = static_cast<size_t>(g.C);
+                        float *f = a.fwd + static_cast<size_t>(segi) * 3 * C + c;
                         f[0] = cur.a;
                         f[C] = cur.b;
                         f[2 * C] = cur.p;
                     }
-                    const size_t row0 = (static_cast<size_t>(b) * g.T + t0 + s0) * C + c;
-                    const float *kp = a.k + row0, *vp = a.v + row0;
                     const float *pg = g_gy + s0 * CG + lane;
                     RevState z;
+                    float M;
                     if (nval == LS) {
-                        rows_forward_outputs<LS, true>(R, cur, nval, prm, kp, vp, C, cvalid);
-                        z = rows_reverse_summary<LS, true>(R, pg, nval, prm.w);
+                        const bool fx = rows_forward_outputs<LS, true>(R, cur, nval, prm, a, g, b,
+                                                                       t0 + s0, c, M);
+                        z = rows_reverse_summary<LS, true>(R, pg, nval, prm, fx, M);
                     } else {
-                        rows_forward_outputs<LS, false>(R, cur, nval, prm, kp, vp, C, cvalid);
-                        z = rows_reverse_summary<LS, false>(R, pg, nval, prm.w);
+                        const bool fx = rows_forward_outputs<LS, false>(R, cur, nval, prm, a, g, b,
+                                                                        t0 + s0, c, M);
+                        z = rows_reverse_summary<LS, false>(R, pg, nval, prm, fx, M);
                     }
-                    if (cvalid) store_rev(a.rev + bs * 5 * C + c, g.C, z);
+                    if (c < g.C) store_rev(a.rev + static_cast<size_t>(segi) * 5 * g.C + c, g.C, z);
                 }
             }
         }
@@ -495,77 +542,160 @@ struct BwdGradsCfg {
     static_assert(kStageBytes % 128 == 0, "stage alignment");
 };
 
-// y_t and ln D_t of the tile's n steps from the forward state before it; sk,
-// sv: this lane's column of the staged k and v tiles.
-// Fixed reference M = max(p_in, max k) when the forward kernel's bound holds,
-// else the per-step max-stabilised form.
+// Per-step values of one lane's tile for the reverse pass, in registers:
+// at the fixed reference M, E = e^{k_t - M}, X = r_t = 1 / den_t and Y = y_t;
+// otherwise E = beta_{t,t}, X = ln D_t and Y = y_t.
+// WKV_BWD_KEEP_E 0: E is not held; the reverse pass evaluates it again from
+// the staged key (one more exponential a step, 32 fewer registers: eleven
+// compute warps without spills, as fast as seven holding it)
+#ifndef WKV_BWD_KEEP_E
+#define WKV_BWD_KEEP_E 0
+#endif
+template <int LT>
+struct TileRows {
+#if WKV_BWD_KEEP_E
+    float E[LT];
+#endif
+    float X[LT], Y[LT];
+};
+
+// The forward pass over the tile's n steps from the state before it (sk, sv:
+// this lane's column of the staged k and v) and the state after it, z.  A
+// full tile whose forward kernel bound holds takes the fixed reference
+// M = max(p_in, max k); it returns true, with E, X, Y at M, when every
+// denominator is also above e^-30 and z's scale e^{M - rho} below e^30 (the
+// reverse pass then runs at M too).  Every other tile ends in the per-step
+// form's values and returns false.
 template <int LT, bool FULL>
-__device__ __forceinline__ void grads_forward(const float *sk, const float *sv, int n,
-                                              const FwdState &cin,
-                                              const WkvOp<float, 1>::Param &q, float (&ys)[LT],
-                                              float (&Ls)[LT]) {
+__device__ __forceinline__ bool grads_forward(const float *sk, const float *sv, int n,
+                                              const FwdState &cin, const RevState &z,
+                                              const WkvOp<float, 1>::Param &q, TileRows<LT> &R,
+                                              float &M) {
     constexpr int CG = 32;
-    float kx = kNoScale, kn = -kNoScale;
+    M = 0.f;
+    if constexpr (FULL) {
+        float kx = kNoScale, kn = -kNoScale;
 #pragma unroll
-    for (int i = 0; i < LT; ++i)
-        if (FULL || i < n) {
+        for (int i = 0; i < LT; ++i) {
             const float k = sk[i * CG];
             kx = fmaxf(kx, k);
             kn = fminf(kn, k);
         }
-    const WkvOp<float, 1>::State cs{cin.a, cin.d, cin.p};
-    const float M = fmaxf(cin.p, kx);
-    if (sweep_is_safe(kn, M, cs, q, n)) {
-        const float f = fast_exp(cin.p - M);
-        float A = cin.a * f, Bs = cin.d * f;
+        const WkvOp<float, 1>::State cs{cin.a, cin.d, cin.p};
+        M = fmaxf(cin.p, kx);
+        if (sweep_is_safe(kn, M, cs, q, n)) {
+            const bool rev_fixed =
+                sweep_is_safe(kn, M, cs, q, n, kRevFixedFloor) && M - z.rho <= 30.f;
+            const float f = fast_exp(cin.p - M);
+            float A = cin.a * f, Bs = cin.d * f;
+            if (rev_fixed) {
 #pragma unroll
-        for (int i = 0; i < LT; ++i)
-            if (FULL || i < n) {
-                const float k = sk[i * CG], v = sv[i * CG];
-                const float e = ex2_approx((k - M) * kLog2e);
-                const float den = fmaf(e, q.U, Bs);
-                ys[i] = v + fmaf(-Bs, v, A) * rcp_approx(den);
-                Ls[i] = M + __logf(den);
-                A = fmaf(A, q.D, e * v);
-                Bs = fmaf(Bs, q.D, e);
-            }
-    } else {
-        FwdState st = cin;
+                for (int i = 0; i < LT; ++i) {
+                    const float k = sk[i * CG], v = sv[i * CG];
+                    const float e = ex2_approx((k - M) * kLog2e);
+                    const float r = rcp_approx(fmaf(e, q.U, Bs));
+#if WKV_BWD_KEEP_E
+                    R.E[i] = e;
+#endif
+                    R.X[i] = r;
+                    R.Y[i] = v + fmaf(-Bs, v, A) * r;
+                    A = fmaf(A, q.D, e * v);
+                    Bs = fmaf(Bs, q.D, e);
+                }
+            } else {
 #pragma unroll
-        for (int i = 0; i < LT; ++i)
-            if (FULL || i < n) {
-                const float k = sk[i * CG], v = sv[i * CG];
-                const Pair f = max_pair(st.p, q.u + k);
-                const float den = fmaf(f.fx, st.d, f.fy);  // in [1, T + 1]
-                ys[i] = fmaf(f.fx, st.a, f.fy * v) * __fdividef(1.f, den);
-                Ls[i] = f.q + __logf(den);
-                fwd_step(st, k, v, q.w);
+                for (int i = 0; i < LT; ++i) {
+                    const float k = sk[i * CG], v = sv[i * CG];
+                    const float e = ex2_approx((k - M) * kLog2e);
+                    const float den = fmaf(e, q.U, Bs);
+                    const float r = rcp_approx(den);
+#if WKV_BWD_KEEP_E
+                    R.E[i] = q.U * e * r;  // beta_{t,t}
+#endif
+                    R.X[i] = M + __logf(den);
+                    R.Y[i] = v + fmaf(-Bs, v, A) * r;
+                    A = fmaf(A, q.D, e * v);
+                    Bs = fmaf(Bs, q.D, e);
+                }
             }
+            return rev_fixed;
+        }
     }
+    FwdState st = cin;
+#pragma unroll
+    for (int i = 0; i < LT; ++i)
+        if (FULL || i < n) {
+            const float k = sk[i * CG], v = sv[i * CG];
+            const Pair f = max_pair(st.p, q.u + k);
+            const float den = fmaf(f.fx, st.d, f.fy);  // in [1, T + 1]
+            const float rden = __fdividef(1.f, den);
+            R.Y[i] = fmaf(f.fx, st.a, f.fy * v) * rden;
+            R.X[i] = f.q + __logf(den);
+#if WKV_BWD_KEEP_E
+            R.E[i] = f.fy * rden;
+#endif
+            fwd_step(st, k, v, q.w);
+        }
+    return false;
 }
 
 // The reverse pass from the state after the tile: gk over sk, gv over sv,
-// and the tile's gw, gu.  beta_{j,j} = e^{u + k_j - ln D_j} (<= 1) is
-// evaluated again here rather than held from the forward pass.
+// and the tile's gw, gu.  At the fixed reference M the four sums run in
+// units of e^{-M} (z converted by e^{M - rho} <= e^30; far below 1 it
+// flushes to 0, the carried sums then weighing less than e^-87 of theirs)
+// and e^{k_j} times a sum is E_j times it: no exponential per step.
+// Otherwise the per-step min-stabilised steps, e^{k_j - rho} <= 1 from the
+// staged key.
 template <int LT, bool FULL>
 __device__ __forceinline__ void grads_reverse(float *sk, float *sv, const float *sg, int n,
-                                              RevState z, float u, float w, const float (&ys)[LT],
-                                              const float (&Ls)[LT], float &gw, float &gu) {
+                                              RevState z, const WkvOp<float, 1>::Param &q,
+                                              const TileRows<LT> &R, bool fixed, float M,
+                                              float &gw, float &gu) {
     constexpr int CG = 32;
     gw = 0.f;
     gu = 0.f;
+    if (fixed) {
+        const float f = fast_exp(M - z.rho);
+        float P = z.P * f, Q = z.Q * f, Rs = z.R * f, R2 = z.R2 * f;
+#pragma unroll
+        for (int i = LT - 1; i >= 0; --i)
+            if (FULL || i < n) {
+                const float vj = sv[i * CG], gj = sg[i * CG];
+#if WKV_BWD_KEEP_E
+                const float e = R.E[i];
+#else
+                const float e = ex2_approx((sk[i * CG] - M) * kLog2e);
+#endif
+                const float gr = gj * R.X[i], y = R.Y[i];
+                const float diag = q.U * gr;  // g_j beta_{j,j} / e_j
+                const float dv = vj - y;
+                sv[i * CG] = e * (diag + P);
+                sk[i * CG] = e * fmaf(diag, dv, fmaf(vj, P, -Q));
+                gu = fmaf(e * diag, dv, gu);
+                gw = fmaf(-e, fmaf(vj, Rs, -R2), gw);
+                Rs = q.D * (Rs + P);
+                R2 = q.D * (R2 + Q);
+                P = fmaf(q.D, P, gr);
+                Q = fmaf(q.D, Q, gr * y);
+            }
+        return;
+    }
 #pragma unroll
     for (int i = LT - 1; i >= 0; --i)
         if (FULL || i < n) {
             const float kj = sk[i * CG], vj = sv[i * CG], gj = sg[i * CG];
-            const float sc = fast_exp(kj - z.rho);              // e^{k_j - rho}, <= 1
-            const float diag = fast_exp(u + kj - Ls[i]) * gj;  // g_j beta_{j,j}
-            const float dv = vj - ys[i];
+            const float sc = fast_exp(kj - z.rho);  // e^{k_j - rho}, <= 1
+#if WKV_BWD_KEEP_E
+            const float diag = R.E[i] * gj;         // g_j beta_{j,j}
+#else
+            const float diag = fast_exp(q.u + kj - R.X[i]) * gj;
+#endif
+            const float dv = vj - R.Y[i];
             sv[i * CG] = fmaf(sc, z.P, diag);
             sk[i * CG] = fmaf(diag, dv, sc * fmaf(vj, z.P, -z.Q));
             gu = fmaf(diag, dv, gu);
             gw = fmaf(-sc, fmaf(vj, z.R, -z.R2), gw);
-            rev_step(z, gj, ys[i], Ls[i], w);
+            rev_step(z, gj, R.Y[i], R.X[i], q.w);
         }
 }
 
@@ -679,16 +809,16 @@ __global__ void __launch_bounds__(BwdGradsCfg<NCW, NSTAGE>::kThreads, 1)
             float *st_k = reinterpret_cast<float *>(smem + static_cast<size_t>(s) * Cfg::kStageBytes);
             float *st_v = st_k + Cfg::kTileElems;
             const float *st_g = st_v + Cfg::kTileElems;
-            float ys[LT], Ls[LT];
-            float gw, gu;
+            TileRows<LT> R;
+            float gw, gu, M;
             if (n == LT) {
-                grads_forward<LT, true>(st_k + lane, st_v + lane, n, cin, q, ys, Ls);
-                grads_reverse<LT, true>(st_k + lane, st_v + lane, st_g + lane, n, z, q.u, q.w, ys,
-                                        Ls, gw, gu);
+                const bool fx = grads_forward<LT, true>(st_k + lane, st_v + lane, n, cin, z, q, R, M);
+                grads_reverse<LT, true>(st_k + lane, st_v + lane, st_g + lane, n, z, q, R, fx, M,
+                                        gw, gu);
             } else {
-                grads_forward<LT, false>(st_k + lane, st_v + lane, n, cin, q, ys, Ls);
-                grads_reverse<LT, false>(st_k + lane, st_v + lane, st_g + lane, n, z, q.u, q.w, ys,
-                                         Ls, gw, gu);
+                grads_forward<LT, false>(st_k + lane, st_v + lane, n, cin, z, q, R, M);
+                grads_reverse<LT, false>(st_k + lane, st_v + lane, st_g + lane, n, z, q, R, false,
+                                         M, gw, gu);
             }
             // gk, gv leave from the stage by TMA (rows >= T and channels >= C
             // are clipped); a stage goes back once its stores have read it:

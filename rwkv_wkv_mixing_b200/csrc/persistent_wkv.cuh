@@ -182,10 +182,12 @@ __device__ __forceinline__ void rows_pass1(const float *sk, const float *sv, int
 // denominator stays above e^-69 (so nothing that matters flushes to zero) and
 // e^u below 2^64.  den_t >= e^{u + k_t - M} once e^{k_t - M} itself cannot
 // flush (k_t - M >= -69 when u >= 0), and den_t >= b_in e^{p_in - M - t w}.
+// (`floor`: the log of the least denominator the bound must guarantee.)
 __device__ __forceinline__ bool sweep_is_safe(float kmin, float M, const WkvOp<float, 1>::State &cin,
-                                              const WkvOp<float, 1>::Param &q, int n) {
-    const bool by_token = kmin + fminf(q.u, 0.f) - M >= -69.f;
-    const bool by_carry = cin.b >= 1.f && cin.p - M - static_cast<float>(n) * q.w >= -69.f;
+                                              const WkvOp<float, 1>::Param &q, int n,
+                                              float floor = -69.f) {
+    const bool by_token = kmin + fminf(q.u, 0.f) - M >= floor;
+    const bool by_carry = cin.b >= 1.f && cin.p - M - static_cast<float>(n) * q.w >= floor;
     return (by_token || by_carry) && q.u <= 44.f;
 }
 

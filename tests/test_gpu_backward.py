@@ -102,6 +102,28 @@ def test_backward_extreme_values(m):
     compare(m, x, gy, "backward extreme", sums_rel=1e-3)
 
 
+def test_backward_every_reverse_frame(m):
+    """Keys spread wide enough (N(0, 10)) that some 32-step segments keep the
+    forward pass's fixed reference but not the reverse one (a denominator
+    between e^-69 and e^-30), fast decays (w up to e^2) that leave the state
+    after a segment far above the segment's frame, and plain channels beside
+    them: every combination of fixed and per-step passes in one launch."""
+    rng = np.random.default_rng(11)
+    B, T, C = 2, 640, 64
+    k = rng.normal(0, 1, (B, T, C)).astype(np.float32)
+    k[:, :, ::2] *= 10.0
+    v = rng.normal(0, 1, (B, T, C)).astype(np.float32)
+    w = np.exp(rng.uniform(-3, 2, C)).astype(np.float32)
+    u = rng.normal(0, 1, C).astype(np.float32)
+    gy = rng.normal(0, 1, (B, T, C)).astype(np.float32)
+
+    class X:
+        pass
+    x = X()
+    x.w, x.u, x.k, x.v = w, u, k, v
+    compare(m, x, gy, "backward reverse frames", sums_rel=1e-3)
+
+
 def test_backward_identities_at_full_size(m):
     """wkv_169m (B=8 T=1024 C=768): every gradient against the float64
     recurrence; the k-shift identity sum_j gk_j = 0 and the constant identity
