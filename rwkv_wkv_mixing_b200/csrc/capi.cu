@@ -487,6 +487,9 @@ wkv_status dispatch_reg_wkv(const typename WkvOp<float, 1, GATED>::Args &args, i
 #ifndef WKV_PS_128
 #define WKV_PS_128 4, 4, 6
 #endif
+#ifndef WKV_PS_64_BF16
+#define WKV_PS_64_BF16 4, 6, 12
+#endif
 template <class Op, class = void>
 struct PackedIo : std::false_type {};
 template <class Op>
@@ -579,8 +582,12 @@ wkv_status dispatch(const typename Op::Args &args, int64_t B, int64_t T, int64_t
             case 8: return launch_chunked<Op, 8, 8>(args, B, T, C, dt, stream, dev);
             case 32: return launch_chunked<Op, 32, 8>(args, B, T, C, dt, stream, dev);
             case 64:
-                return tma ? launch_persistent<Op, 64, 4, 6, 12>(args, B, T, C, dt, stream, dev)
-                           : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
+                if constexpr (PackedIo<Op>::value)
+                    return tma ? launch_persistent<Op, 64, WKV_PS_64_BF16>(args, B, T, C, dt, stream, dev)
+                               : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
+                else
+                    return tma ? launch_persistent<Op, 64, 4, 6, 12>(args, B, T, C, dt, stream, dev)
+                               : launch_chunked<Op, 64, 8>(args, B, T, C, dt, stream, dev);
             case 256:
                 return tma ? launch_persistent<Op, 256, 8, 2, 3>(args, B, T, C, dt, stream, dev)
                            : launch_chunked<Op, 256, 8>(args, B, T, C, dt, stream, dev);

@@ -145,25 +145,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// ---- 16-byte asynchronous copies global -> shared (L2 only) -----------------
-// the copy lands in shared memory without holding registers; it reads L2
-// (.cg), so it sees what other thread blocks have published to L2, possibly
-// a moment out of date
-__device__ __forceinline__ void cp_async_16_l2(void *smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)),
-                 "l"(gmem_src)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// wait until every cp.async this thread committed has landed
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-
 // ---- flags between thread blocks -----------------------------------------
 __device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long *p) {
     unsigned long long v;

@@ -214,67 +214,6 @@ __device__ __forceinline__ bool lookback_channel(const Workspace &ws, const Geom
     }
 }
 
-// The first H records a tile's look-back reads (tiles tile - S, ..., tile -
-// H S), copied into shared memory with cp.async before pass 1: slot[i * 32]
-// for hop i of this lane.  Hops before the first segment are left alone (a
-// look-back never reads past the first segment, whose tiles publish the
-// state after themselves).
-template <class Op, int H>
-__device__ __forceinline__ void lookback_prefetch_smem(const Workspace &ws, const Geometry &g,
-                                                       int tile, int lane, int j, uint4 *slot) {
-    constexpr int CPT = Op::CPT, CG = 32 * CPT;
-    const long long S = g.tiles_per_seg;
-#pragma unroll
-    for (int i = 0; i < H; ++i) {
-        const long long q = static_cast<long long>(tile) - (i + 1) * S;
-        if (q >= 0) cp_async_16_l2(slot + i * 32, ws.records + q * CG + lane * CPT + j);
-    }
-    cp_async_commit();
-}
-
-// Decoupled look-back for channel j of this lane, as lookback_channel, with
-// the records read H hops at a time through shared memory: `slot[i * 32]`
-// holds hop i from the current position (the first batch was copied by
-// lookback_prefetch_smem before pass 1, and the caller has waited for it).
-// The lane folds the batch newest first; when it meets a record that is not
-// current yet, or has folded the whole batch, it copies the next H hops from
-// where it stands (cp.async, no registers held) and carries on.  Returns
-// false if a record never appeared within the poll budget.
-template <class Op, int LT, int H>
-__device__ __forceinline__ bool lookback_channel_prefetched(const Workspace &ws, const Geometry &g,
-                                                            int tile, unsigned long long epoch,
-                                                            const typename Op::Param &prm, int lane,
-                                                            int j, typename Op::State &run,
-                                                            uint4 *slot) {
-    const long long S = g.tiles_per_seg;
-    run = Op::identity();
-    float run_len = 0.f;
-    long long base = tile;  // the batch in `slot` holds tiles base - S, ..., base - H S
-    long long polls = 0;
-    for (;;) {
-        int i = 0;
-        for (; i < H; ++i) {
-            const long long q = base - (i + 1) * S;
-            if (q < 0) return false;  // cannot happen: first-segment tiles always end the fold
-            const uint4 r = slot[i * 32];
-            const unsigned long long tag = record_tag(r);
-            if ((tag >> 18) != epoch || (tag & 3u) == 0u) break;  // not published yet
-            const typename Op::State val = Op::unpack(__uint_as_float(r.x), __uint_as_float(r.y),
-                                                      static_cast<uint32_t>(tag >> 2) & 0xffffu);
-            run = Op::combine(val, run, run_len, prm);
-            run_len += static_cast<float>(LT);
-            if ((tag & 3u) == kFlagIncl) return true;
-        }
-        base -= i * S;
-        if (i < H) {  // waiting for a record: back off before reading it again
-            if (++polls > g.spin_limit) return false;
-            __nanosleep(32);
-        }
-        lookback_prefetch_smem<Op, H>(ws, g, static_cast<int>(base), lane, j, slot);
-        cp_async_wait_all();
-    }
-}
-
 // all CPT channels of this lane, one after another; false (in every lane
 // that gave up) if a record never appeared within the poll budget
 template <class Op, int LT>
