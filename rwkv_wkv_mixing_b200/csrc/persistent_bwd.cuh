@@ -295,6 +295,10 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
                     bulk_load(dp + CG, a.w + c0, pbytes, &full_bar[s]);
                 }
             }
+            // every tile of this block is loaded or assigned: the next grid in
+            // the stream may start launching its blocks (its own
+            // griddepcontrol.wait still waits for this grid to complete)
+            allow_dependent_launch();
         }
         __syncwarp();
     } else {
@@ -765,6 +769,10 @@ __global__ void __launch_bounds__(BwdGradsCfg<NCW, NSTAGE>::kThreads, 1)
                 tma_load_3d(dst + Cfg::kTileBytes, &map_v, &full_bar[s], c0, seg * LT, b);
                 tma_load_3d(dst + 2 * Cfg::kTileBytes, &map_gy, &full_bar[s], c0, seg * LT, b);
             }
+            // every tile of this block is loaded or assigned: the next grid in
+            // the stream may start launching its blocks (its own
+            // griddepcontrol.wait still waits for this grid to complete)
+            allow_dependent_launch();
         }
         __syncwarp();
     } else {

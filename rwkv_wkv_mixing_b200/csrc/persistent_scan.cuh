@@ -235,6 +235,10 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
                                     c0 * Op::kScalarsPerIo, seg * LT, b);
                 }
             }
+            // every tile of this block is loaded or assigned: the next grid in
+            // the stream may start launching its blocks (its own
+            // griddepcontrol.wait still waits for this grid to complete)
+            allow_dependent_launch();
         }
         __syncwarp();
     } else {

@@ -370,6 +370,10 @@ __global__ void __launch_bounds__(RegWkvCfg<LT, NWG, NC, NSTAGE, GATED>::kThread
                     bulk_load(dp + CG, args.w + c0, pbytes, &full_bar[s]);
                 }
             }
+            // every tile of this block is loaded or assigned: the next grid in
+            // the stream may start launching its blocks (its own
+            // griddepcontrol.wait still waits for this grid to complete)
+            allow_dependent_launch();
         }
         __syncwarp();
     } else {
