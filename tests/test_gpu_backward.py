@@ -102,6 +102,25 @@ def test_backward_extreme_values(m):
     compare(m, x, gy, "backward extreme", sums_rel=1e-3)
 
 
+def test_backward_repeated_calls_with_a_forward_between(m):
+    """The gradient step's kernels keep counters (the forward look-back's
+    tickets and epoch, the gw/gu sum's counters) in per-stream workspaces the
+    forward kernels share: calls back to back, with a forward call in
+    between, must each find them reset."""
+    x = workloads.make_wkv("wkv_169m", B=2, T=1000, C=96, seed=21)
+    gy = np.random.default_rng(21).normal(0, 1, x.k.shape).astype(np.float32)
+    want = oracle.wkv_backward_rnn(x.w, x.u, x.k, x.v, gy)
+    w, u, k, v, g = dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(gy)
+    for call in range(3):
+        out = m.wkv_backward(w, u, k, v, g)
+        m.wkv_forward(w, u, k, v)
+        torch.cuda.synchronize()
+        for name, got, wv, rel in zip(("gk", "gv", "gw", "gu"), out, want,
+                                      (1e-4, 1e-4, 2e-4, 2e-4)):
+            check(got.double().cpu().numpy(), wv, rel, f"call {call} {name}")
+    m.wkv_device_status()  # raises if a device-side wait gave up
+
+
 def test_backward_every_reverse_frame(m):
     """Keys spread wide enough (N(0, 10)) that some 32-step segments keep the
     forward pass's fixed reference but not the reverse one (a denominator
