@@ -94,16 +94,16 @@ def read_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# the sources the tiled WKV / scan kernels are built from (their dispatch
-# included); a recorded DRAM-traffic figure is only reported while these are
-# unchanged
-TILED_KERNEL_SOURCES = ("capi.cu", "persistent_scan.cuh", "persistent_wkv.cuh", "chunked_scan.cuh",
-                        "scan_common.cuh", "wkv_ops.cuh", "ptx.cuh")
+# the sources every kernel is built from (their dispatch included); a
+# recorded DRAM-traffic figure is only reported while these are unchanged
+KERNEL_SOURCES = ("capi.cu", "persistent_scan.cuh", "persistent_wkv.cuh", "persistent_bwd.cuh",
+                  "chunked_scan.cuh", "scan_common.cuh", "wkv_ops.cuh", "lru_ops.cuh",
+                  "wkv_backward.cuh", "serial_wkv.cuh", "token_shift.cuh", "ptx.cuh")
 
 
 def src_hash():
     h = hashlib.sha256()
-    for name in TILED_KERNEL_SOURCES:
+    for name in KERNEL_SOURCES:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
