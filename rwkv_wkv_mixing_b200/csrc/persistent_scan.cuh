@@ -34,6 +34,11 @@ namespace wkvb {
 
 constexpr unsigned long long kBarrierWaitNs = 4000000000ull;  // 4 s
 
+// look-back records (hops back in time) a group loads before pass 1
+#ifndef WKV_LB_PREFETCH
+#define WKV_LB_PREFETCH 1
+#endif
+
 // stage waits: 0 = suspend in mbarrier try_wait; N > 0 = poll with
 // mbarrier test_wait, N ns apart
 #ifndef WKV_FILL_POLL
@@ -311,7 +316,7 @@ __global__ void __launch_bounds__(PersistentCfg<Op, LT, NWG, NC, NSTAGE>::kThrea
             // the tile before this one in time was handed out well before it,
             // so its state is usually published already and lands during pass 1
             const bool lb = chained && seg > 0;
-            ChannelPrefetch<1> pf;
+            ChannelPrefetch<WKV_LB_PREFETCH> pf;
 #pragma unroll
             for (int j = 0; j < CPT; ++j)
                 if (wg == j && lb) lookback_prefetch_channel<Op>(ws, g, tile, lane, j, pf);
