@@ -1080,16 +1080,14 @@ wkv_status launch_bwd_tiled(const WkvBwdArgs &a, int64_t B, int64_t T, int64_t C
     if ((st = launch_pdl(ks, std::min(gs.tiles, sms), BwdStates::kThreads, BwdStates::kSmemBytes,
                          stream, m[0], m[1], m[2], ta, gs, ws)) != WKV_OK)
         return st;
-    const int64_t n_cg = (C + 31) / 32;
-    wkv_bwd_rev_carry_kernel<<<static_cast<unsigned>(B * n_cg), 32 * kCarryWarps, 0, stream>>>(a);
+    const int n_cg = static_cast<int>((C + 31) / 32);
+    if ((st = launch_pdl(wkv_bwd_rev_carry_kernel, static_cast<int>(B) * n_cg, 32 * kCarryWarps, 0,
+                         stream, a)) != WKV_OK)
+        return st;
     if ((st = launch_pdl(kg, std::min(gg.tiles, sms), BwdGrads::kThreads, BwdGrads::kSmemBytes,
                          stream, m[3], m[4], m[5], m[6], m[7], ta, gg, ws)) != WKV_OK)
         return st;
-    wkv_bwd_reduce_kernel<<<static_cast<unsigned>(n_cg * kReduceParts), 32 * kReduceWarps, 0,
-                            stream>>>(a);
-    const cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
-    return WKV_OK;
+    return launch_pdl(wkv_bwd_reduce_kernel, n_cg * kReduceParts, 32 * kReduceWarps, 0, stream, a);
 }
 
 }  // namespace
