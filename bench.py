@@ -25,6 +25,10 @@ steps run; null when none landed inside it), and the number of library
 kernel launches timed.  The CPU oracle is timed on all of this host's cores
 and on one core.
 
+``--shape B,T,C`` runs a workload's distributions at another shape (the
+same kernel on a smaller case, for profiler captures); the JSON line's
+config says so.
+
 ``--impl reference`` times the CPU oracle instead (the only reference this
 project has: a plain float64 implementation of the pages' definition), on a
 bounded sample of the same workload, and prints the same line with
