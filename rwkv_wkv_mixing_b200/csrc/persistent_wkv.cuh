@@ -116,7 +116,7 @@ __device__ __forceinline__ WkvOp<float, 1>::State resum_f32(const float *sk, con
     const Op::Param qq[1] = {q};
     const float ref[1] = {Op::largest_exponent(sk, n, 0, q)};
     float a2[1], b2[1];
-    Op::chunk_sums<LS>(sk, sv, n, qq, ref, a2, b2);
+    Op::chunk_sums<LS, 8>(sk, sv, n, qq, ref, a2, b2);
     return {a2[0], b2[0], ref[0]};
 }
 

@@ -17,6 +17,21 @@
 namespace wkvb {
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// unroll factor of the full-sub-chunk loops of the packed bf16 passes,
+// without and with the gate (measured: 8 and 4; the gate's larger loop body
+// runs faster with less code, the plain one with more)
+#ifndef WKV_PACKED_UNROLL
+#define WKV_PACKED_UNROLL 8
+#endif
+#ifndef WKV_PACKED_UNROLL_GATED
+#define WKV_PACKED_UNROLL_GATED 4
+#endif
+// ... and of the scalar (fp32, one channel a thread) passes (32, the whole
+// sub-chunk: wkv_long 298.7 against 306.8 us with 8)
+#ifndef WKV_SCALAR_UNROLL
+#define WKV_SCALAR_UNROLL 32
+#endif
 // log-scale of "no tokens yet": finite, so differences of two such values
 // stay finite, and e^(kNoScale - anything real) is exactly zero
 constexpr float kNoScale = -1e30f;
@@ -166,6 +181,8 @@ struct WkvOp {
     static constexpr bool kPacked = sizeof(IO) == 2 && CPT == 2;
     static constexpr bool kGated = GATED;
     static constexpr bool kSerialForm = true;  // has the per-step form of serial_wkv.cuh
+    static constexpr int kPackedUnroll = GATED ? WKV_PACKED_UNROLL_GATED : WKV_PACKED_UNROLL;
+    static constexpr int kScalarUnroll = WKV_SCALAR_UNROLL;
     struct Param {
         float u, w;  // bonus and decay (natural units)
         float U, D;  // e^u, e^{-w}
@@ -273,7 +290,7 @@ struct WkvOp {
             const __nv_bfloat16 ninf = __ushort_as_bfloat16(0xff80u), pinf = __ushort_as_bfloat16(0x7f80u);
             __nv_bfloat162 hx = __halves2bfloat162(ninf, ninf), hn = __halves2bfloat162(pinf, pinf);
             if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kPackedUnroll)
                 for (int i = 0; i < LS; ++i) {
                     const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(p0 + i * CG);
                     hx = __hmax2(hx, k2);
@@ -298,7 +315,7 @@ struct WkvOp {
                 kn[j] = -kNoScale;
             }
             if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kScalarUnroll)
                 for (int i = 0; i < LS; ++i) {
                     float k[CPT];
                     Vec<IO, CPT>::load(p0 + i * CG, k);
@@ -324,7 +341,9 @@ struct WkvOp {
 
     // round 2: a = sum_i e^{k_i - (end-i) w - ref} v_i, b = the same without
     // v_i, over n rows ending at row n-1
-    template <int LS>
+    // (U: unroll factor of the scalar full-sub-chunk loop; the register-
+    // resident kernels' rare re-sum path keeps 8, its code small)
+    template <int LS, int U = kScalarUnroll>
     __device__ __forceinline__ static void chunk_sums(const IO *p0, const IO *p1, int n,
                                                       const Param (&q)[CPT],
                                                       const float (&ref)[CPT], float (&a)[CPT],
@@ -353,7 +372,7 @@ struct WkvOp {
                 b2 = __fadd2_rn(b2, e);
             };
             if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kPackedUnroll)
                 for (int i = 0; i < LS; ++i) one(i, static_cast<float>(i - (LS - 1)));
             } else {
                 for (int i = 0; i < n; ++i) one(i, static_cast<float>(i - (n - 1)));
@@ -365,7 +384,7 @@ struct WkvOp {
             return;
         }
         if (n == LS) {
-#pragma unroll 8
+#pragma unroll(U)
             for (int i = 0; i < LS; ++i) {
                 float k[CPT], v[CPT];
                 Vec<IO, CPT>::load(p0 + i * CG, k);
@@ -504,7 +523,7 @@ struct WkvOp {
         }
         if (fast) {
             if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kScalarUnroll)
                 for (int i = 0; i < LS; ++i)
                     fast_step(p0 + i * CG, p1 + i * CG, p2 + i * CG, out + i * ostride, valid, M,
                               M2, A, Bs, q);
@@ -566,7 +585,7 @@ struct WkvOp {
             if (valid) Vec<IO, CPT>::store(out + i * ostride, y);
         };
         if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kPackedUnroll)
             for (int i = 0; i < LS; ++i) one(i);
         } else {
             for (int i = 0; i < n; ++i) one(i);
