@@ -24,6 +24,11 @@
 
 namespace wkvb {
 
+// unroll factor of the full-sub-chunk loops
+#ifndef WKV_LRU_UNROLL
+#define WKV_LRU_UNROLL 8
+#endif
+
 struct LruOp {
     using io_t = float2;
     static constexpr int CPT = 1;
@@ -31,6 +36,7 @@ struct LruOp {
     static constexpr int NV = 2;
     static constexpr int NIN = 1;            // u only
     static constexpr int kScalarsPerIo = 2;  // tensor maps see (re, im) as two floats
+    static constexpr int kLruUnroll = WKV_LRU_UNROLL;
     static constexpr bool kGated = false;
     static constexpr bool kSerialForm = false;
     struct Param {
@@ -121,7 +127,7 @@ struct LruOp {
                                                      Scratch (&)[1]) {
         float xr = 0.f, xi = 0.f;
         if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kLruUnroll)
             for (int i = 0; i < LS; ++i) step(xr, xi, p0[i * CG], q[0]);
         } else {
             for (int i = 0; i < n; ++i) step(xr, xi, p0[i * CG], q[0]);
@@ -136,7 +142,7 @@ struct LruOp {
                                                  float2 *out, size_t ostride, bool valid) {
         float xr = carry[0].r, xi = carry[0].i;
         if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kLruUnroll)
             for (int i = 0; i < LS; ++i) {
                 step(xr, xi, p0[i * CG], q[0]);
                 if (valid) out[i * ostride] = make_float2(xr, xi);

@@ -29,6 +29,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 #endif
 // ... and of the scalar (fp32, one channel a thread) passes (32, the whole
 // sub-chunk: wkv_long 298.7 against 306.8 us with 8)
+#ifndef WKV_SCAN_UNROLL
+#define WKV_SCAN_UNROLL 8
+#endif
+#ifndef WKV_SCAN_UNROLL_BF16
+#define WKV_SCAN_UNROLL_BF16 8
+#endif
 #ifndef WKV_SCALAR_UNROLL
 #define WKV_SCALAR_UNROLL 32
 #endif
@@ -627,6 +633,7 @@ template <typename IO, int CPT_>
 struct ScanOpT {
     using io_t = IO;
     static constexpr int CPT = CPT_;
+    static constexpr int kScanUnroll = sizeof(IO) == 2 ? WKV_SCAN_UNROLL_BF16 : WKV_SCAN_UNROLL;
     static constexpr int CG = 32 * CPT;
     static constexpr int NV = 2;
     static constexpr int NIN = 2;
@@ -682,7 +689,7 @@ struct ScanOpT {
             H[j] = 0.f;
         }
         if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kScanUnroll)
             for (int i = 0; i < LS; ++i) {
                 float a[CPT], b[CPT];
                 Vec<IO, CPT>::load(p0 + i * CG, a);
@@ -718,7 +725,7 @@ struct ScanOpT {
 #pragma unroll
         for (int j = 0; j < CPT; ++j) H[j] = carry[j].H;
         if (n == LS) {
-#pragma unroll 8
+#pragma unroll(kScanUnroll)
             for (int i = 0; i < LS; ++i) {
                 float a[CPT], b[CPT];
                 Vec<IO, CPT>::load(p0 + i * CG, a);
