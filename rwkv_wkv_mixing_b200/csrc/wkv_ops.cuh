@@ -287,7 +287,7 @@ struct WkvOp {
             return (x - r) * kLog2e;
     }
 
-    // round 1: largest and smallest key of each channel over n rows
+    // first sweep: largest and smallest key of each channel over n rows
     template <int LS>
     __device__ __forceinline__ static void key_range(const IO *p0, int n, float (&kx)[CPT],
                                                      float (&kn)[CPT]) {
@@ -345,7 +345,7 @@ struct WkvOp {
         }
     }
 
-    // round 2: a = sum_i e^{k_i - (end-i) w - ref} v_i, b = the same without
+    // second sweep: a = sum_i e^{k_i - (end-i) w - ref} v_i, b = the same without
     // v_i, over n rows ending at row n-1
     // (U: unroll factor of the scalar full-sub-chunk loop; the register-
     // resident kernels' rare re-sum path keeps 8, its code small)
