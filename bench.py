@@ -105,11 +105,41 @@ KERNEL_SOURCES = ("capi.cu", "persistent_scan.cuh", "persistent_wkv.cuh", "persi
                   "wkv_backward.cuh", "serial_wkv.cuh", "token_shift.cuh", "ptx.cuh")
 
 
-def src_hash():
+def _code_only(text):
+    """C/C++ source without comments and with whitespace collapsed, so that
+    an edit of comments alone does not count as a change of the kernels."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif c in "\"'":  # string or character literal, kept whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def src_hash(read=None):
+    """Hash of the code of every kernel source (comments and whitespace
+    ignored); `read(name)` returns a source's text (default: the file)."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(CSRC, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        if read is None:
+            with open(os.path.join(CSRC, name), encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(name)
+        h.update(name.encode() + b"\0" + _code_only(text).encode())
     return h.hexdigest()[:16]
 
 
