@@ -55,6 +55,36 @@ def test_a_tile_that_never_publishes_times_out_cleanly(m, steps):
     assert np.abs(y.double().cpu().numpy() - want).max() <= tol
 
 
+def test_gradients_time_out_cleanly_when_a_tile_never_publishes(m):
+    """The gradient step's first pass carries the forward state between
+    128-step tiles by the same look-back: a silent tile makes the waits
+    behind it run out; its channels' gradients come out NaN (the reverse
+    sums then carry the NaN back to the start of the chain), the other
+    channels' are exact, the status word says so, and the next call is
+    correct again."""
+    B, T, C = 1, 1024, 64            # two 32-channel chains of eight tiles
+    x = workloads.make_wkv("wkv_169m", B=B, T=T, C=C, seed=103)
+    gy = np.random.default_rng(103).normal(0, 1, x.k.shape).astype(np.float32)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to("cuda")   # noqa: E731
+    w, u, k, v, g = d(x.w), d(x.u), d(x.k), d(x.v), d(gy)
+    want = oracle.wkv_backward_rnn(x.w, x.u, x.k, x.v, gy)
+    m.wkv_device_status()
+    m.wkv_set_fault_injection(4, 4096)   # segment 2 of channel group 0 stays silent
+    got = [t.double().cpu().numpy() for t in m.wkv_backward(w, u, k, v, g)]
+    with pytest.raises(m.WkvError) as err:
+        m.wkv_device_status()
+    assert err.value.status == m.WKV_ERR_TIMEOUT
+    for name, gv_, wv, rel in zip(("gk", "gv", "gw", "gu"), got, want, (1e-4, 1e-4, 2e-4, 2e-4)):
+        assert np.isnan(gv_[..., :32]).all(), f"{name}: the silent chain's gradients must be NaN"
+        scale = float(np.abs(wv[..., 32:]).max())
+        assert np.abs(gv_[..., 32:] - wv[..., 32:]).max() <= rel * scale, name
+    m.wkv_set_fault_injection(-1, 0)
+    got = [t.double().cpu().numpy() for t in m.wkv_backward(w, u, k, v, g)]
+    m.wkv_device_status()
+    for name, gv_, wv, rel in zip(("gk", "gv", "gw", "gu"), got, want, (1e-4, 1e-4, 2e-4, 2e-4)):
+        assert np.abs(gv_ - wv).max() <= rel * float(np.abs(wv).max()), name
+
+
 def test_fault_injection_arguments_are_checked(m):
     assert m.lib.wkv_set_fault_injection(-2, 0) == m.WKV_ERR_INVALID_ARG
     assert m.lib.wkv_set_fault_injection(0, -1) == m.WKV_ERR_INVALID_ARG
