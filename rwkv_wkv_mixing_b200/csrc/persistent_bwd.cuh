@@ -733,7 +733,6 @@ __global__ void __launch_bounds__(BwdGradsCfg<NCW, NSTAGE>::kThreads, 1)
         fence_mbar_init();
         s_abort = 0;
     }
-    grid_dependency_wait();
     __syncthreads();
     volatile int *abort_flag = &s_abort;
 
@@ -777,6 +776,14 @@ __global__ void __launch_bounds__(BwdGradsCfg<NCW, NSTAGE>::kThreads, 1)
         __syncwarp();
     } else {
         // ---------------- compute warps: ring iterations cw, cw + NCW, ... ----
+        // The producer loads k, v and gy without waiting for the grids before
+        // this one in the stream: the gradient step's first kernels write
+        // none of them (only the scratch), and this grid's blocks are
+        // launched only after those kernels' blocks have all started, i.e.
+        // after the first of them has itself waited for everything before
+        // the step.  What this warp reads from the scratch, and every store,
+        // comes after the wait for the previous grid to complete.
+        grid_dependency_wait();
         const int cw = warp - 1;
         const size_t C = static_cast<size_t>(g.C);
         int held = -1;  // the stage of this warp's stores still in flight

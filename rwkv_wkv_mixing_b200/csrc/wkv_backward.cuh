@@ -324,10 +324,12 @@ __global__ void __launch_bounds__(32 * kCarryWarps) wkv_bwd_rev_carry_kernel(con
     __shared__ RevState part[kCarryWarps][32];
     __shared__ int part_n[kCarryWarps];
     // launched as a programmatic dependent of the summaries' kernel on the
-    // tiled path: nothing global is read before it has finished (a no-op
-    // for an ordinary launch); the next kernel may start launching at once
-    grid_dependency_wait();
+    // tiled path: the next kernel (the gradient tiles, whose producer starts
+    // loading k, v, gy at once) may start launching as soon as every block
+    // of this one runs; nothing global is read here before the summaries'
+    // kernel has finished (both no-ops for an ordinary launch)
     allow_dependent_launch();
+    grid_dependency_wait();
     const int cb = (a.C + 31) / 32;
     const int b = blockIdx.x / cb, lane = threadIdx.x % 32, wi = threadIdx.x / 32;
     const int c = (blockIdx.x % cb) * 32 + lane;
@@ -422,9 +424,11 @@ __global__ void __launch_bounds__(kBwdThreads, 4) wkv_bwd_grads_kernel(const Wkv
 __global__ void __launch_bounds__(32 * kReduceWarps) wkv_bwd_reduce_kernel(const WkvBwdArgs a) {
     __shared__ float part[2][kReduceWarps][32];
     __shared__ bool last;
-    // as in wkv_bwd_rev_carry_kernel: wait for the partials' kernel
-    grid_dependency_wait();
+    // as in wkv_bwd_rev_carry_kernel: the next grid in the stream may start
+    // launching at once (its own wait covers this one); the partials are read
+    // only after their kernel has finished
     allow_dependent_launch();
+    grid_dependency_wait();
     const int lane = threadIdx.x % 32, wi = threadIdx.x / 32;
     const int cg = blockIdx.x / kReduceParts, pi = blockIdx.x % kReduceParts;
     const int c = cg * 32 + lane;
