@@ -129,11 +129,17 @@ def _code_only(text):
     return " ".join("".join(out).split())
 
 
-def src_hash(read=None):
-    """Hash of the code of every kernel source (comments and whitespace
-    ignored); `read(name)` returns a source's text (default: the file)."""
+# The gradient kernels' own headers: no forward kernel is built from them.
+GRAD_ONLY_SOURCES = ("persistent_bwd.cuh", "wkv_backward.cuh")
+FORWARD_SOURCES = tuple(n for n in KERNEL_SOURCES if n not in GRAD_ONLY_SOURCES)
+
+
+def src_hash(read=None, names=KERNEL_SOURCES):
+    """Hash of the code of the named kernel sources (default: every one;
+    comments and whitespace ignored); `read(name)` returns a source's text
+    (default: the file)."""
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in names:
         if read is None:
             with open(os.path.join(CSRC, name), encoding="utf-8") as f:
                 text = f.read()
@@ -145,14 +151,18 @@ def src_hash(read=None):
 
 def recorded_traffic(workload):
     """DRAM bytes per launch from a committed ncu capture, if it was taken on
-    the kernel sources as they are now; otherwise None."""
+    the kernel sources as they are now (those the entry names, every kernel
+    source when it names none); otherwise None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(workload)
     except Exception:
         return None
-    if not rec or rec.get("src_sha") != src_hash():
+    if not rec:
+        return None
+    names = tuple(rec.get("sources") or KERNEL_SOURCES)
+    if not set(names) <= set(KERNEL_SOURCES) or rec.get("src_sha") != src_hash(names=names):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -40,3 +40,32 @@ def test_recorded_traffic_entries_are_consistent():
             abs(e["dram_bytes_per_launch"] - e["dram_read_bytes"] - e["dram_write_bytes"]) <= 2, name
         assert "--clock-control none" in e["command"], name
         assert len(e["src_sha"]) == 16, name
+        assert set(e.get("sources") or bench.KERNEL_SOURCES) <= set(bench.KERNEL_SOURCES), name
+        if name.endswith("_bwd"):   # the gradient kernels are built from every source
+            assert not e.get("sources"), name
+
+
+def test_forward_sources_leave_out_only_the_gradient_headers():
+    assert set(bench.KERNEL_SOURCES) - set(bench.FORWARD_SOURCES) == set(bench.GRAD_ONLY_SOURCES)
+    # no forward source pulls in a gradient header
+    for name in bench.FORWARD_SOURCES:
+        if name == "capi.cu":   # the library's entry points, gradients included
+            continue
+        with open(os.path.join(bench.CSRC, name), encoding="utf-8") as f:
+            text = f.read()
+        for g in bench.GRAD_ONLY_SOURCES:
+            assert f'#include "{g}"' not in text, (name, g)
+
+
+def test_recorded_traffic_is_keyed_to_the_entry_sources(tmp_path, monkeypatch):
+    fwd = bench.src_hash(names=bench.FORWARD_SOURCES)
+    rec = {"a": {"src_sha": fwd, "sources": list(bench.FORWARD_SOURCES), "dram_bytes_per_launch": 7},
+           "b": {"src_sha": fwd, "dram_bytes_per_launch": 8},        # no list: every source
+           "c": {"src_sha": fwd, "sources": ["nope.cu"], "dram_bytes_per_launch": 9}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("a") == 7
+    assert bench.recorded_traffic("b") is None
+    assert bench.recorded_traffic("c") is None
+    assert bench.recorded_traffic("missing") is None
