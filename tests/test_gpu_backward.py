@@ -121,6 +121,34 @@ def test_backward_repeated_calls_with_a_forward_between(m):
     m.wkv_device_status()  # raises if a device-side wait gave up
 
 
+def test_backward_inputs_written_just_before_each_call(m):
+    """The gradient pass starts loading k, v and gy before waiting for the
+    step's first kernels (which write only the scratch): each call's gy
+    (and k) comes from a kernel launched on the same stream right before the
+    call, different every time, and without a synchronisation between the
+    calls; every call must see its own inputs.  gk, gv, gw, gu are linear
+    in gy, and scaling by a power of two is exact in floating point."""
+    x = workloads.make_wkv("wkv_169m", B=2, T=1000, C=96, seed=23)
+    gy0 = np.random.default_rng(23).normal(0, 1, x.k.shape).astype(np.float32)
+    want = oracle.wkv_backward_rnn(x.w, x.u, x.k, x.v, gy0)
+    w, u, k0, v, g0 = dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(gy0)
+    k = torch.empty_like(k0)
+    g = torch.empty_like(g0)
+    outs = []
+    for call in range(6):
+        k.copy_(k0 + 0.0)             # rewritten by a kernel just before the call
+        torch.mul(g0, float(2 ** call), out=g)
+        outs.append([t.clone() for t in m.wkv_backward(w, u, k, v, g)])
+        k.zero_()                     # and overwritten right after it
+        g.fill_(float("nan"))
+    torch.cuda.synchronize()
+    for call, out in enumerate(outs):
+        for name, got, wv, rel in zip(("gk", "gv", "gw", "gu"), out, want,
+                                      (1e-4, 1e-4, 2e-4, 2e-4)):
+            check(got.double().cpu().numpy() / 2 ** call, wv, rel, f"call {call} {name}")
+    m.wkv_device_status()
+
+
 def test_backward_every_reverse_frame(m):
     """Keys spread wide enough (N(0, 10)) that some 32-step segments keep the
     forward pass's fixed reference but not the reverse one (a denominator
