@@ -986,11 +986,13 @@ wkv_status wkv_host_common(int64_t B, int64_t T, int64_t C, const float *w, cons
 #define WKV_BWD_TILED 1
 #endif
 // states kernel: 128-step tiles, three groups of four compute warps (one
-// 32-step segment each) and a carry warp, three stages; gradients kernel:
+// 32-step segment each) and a carry warp, four stages of k and v (each
+// group's gy tile in its own buffer; five were 14 % slower on B=1 T=32768:
+// more tiles of one chain in flight); gradients kernel:
 // eleven compute warps (168 registers: three warps per SM sub-partition),
 // sixteen 32-step stages of k, v and gy
 #ifndef WKV_BWD_STATES_CFG
-#define WKV_BWD_STATES_CFG 128, 4, 3, 3
+#define WKV_BWD_STATES_CFG 128, 4, 3, 4
 #endif
 #ifndef WKV_BWD_GRADS_CFG
 #define WKV_BWD_GRADS_CFG 11, 16

@@ -10,7 +10,10 @@
 //     compute warp owns one 32-step segment of a tile: it writes the forward
 //     state before its segment, computes y_t and ln D_t of the segment from
 //     it, and writes the segment's reverse summary (the sums over its own
-//     outputs, from the zero state).  k, v and gy are read once.
+//     outputs, from the zero state).  k and v come through the ring of
+//     stages; a group's gy tile, needed only in pass 2, is loaded by TMA into
+//     the group's own buffer when the group starts the tile, so a stage goes
+//     back after pass 1 and four of them fit.  k, v and gy are read once.
 //  2. wkv_bwd_rev_carry_kernel (wkv_backward.cuh), backwards over segments:
 //     the reverse state after each segment.
 //  3. wkv_bwd_grads_tiles_kernel: every 32-step x 32-channel tile on its own,
@@ -69,12 +72,12 @@ struct BwdStatesCfg {
     static constexpr int NGW = NWG + 1;  // warps per group: NWG compute, 1 carry
     static constexpr int kThreads = (1 + NC * NGW) * 32;
     static constexpr size_t kTileElems = static_cast<size_t>(LT) * CG;
-    // a stage: the k, v and gy tiles, then the tile's u and w ([CG] fp32 each)
-    static constexpr size_t kParamOffset = 3 * kTileElems * sizeof(float);
+    // a stage: the k and v tiles, then the tile's u and w ([CG] fp32 each)
+    static constexpr size_t kParamOffset = 2 * kTileElems * sizeof(float);
     static constexpr size_t kStageBytes = kParamOffset + 2 * CG * sizeof(float);
     static constexpr int kHops = WKV_REG_LOOKBACK_HOPS;
-    // per group: the gy tile (copied out of the stage in pass 1, read in pass
-    // 2), then two slots (double-buffered) of the compute warps' summaries
+    // per group: the gy tile (loaded by TMA when the group starts a tile,
+    // read in pass 2), then two slots (double-buffered) of the compute warps' summaries
     // [NWG][3][CG], of the carry [3][CG] and of the tile aggregate [3][CG]
     static constexpr size_t kGyBytes = kTileElems * sizeof(float);
     static constexpr size_t kSumFloats = static_cast<size_t>(NWG) * 3 * CG;
@@ -206,12 +209,15 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
     constexpr int CG = Cfg::CG, LS = Cfg::LS, NV = 3, NGW = Cfg::NGW;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *s_stage = smem;  // [NSTAGE] x (k, v, gy tiles, u[CG], w[CG])
+    unsigned char *s_stage = smem;  // [NSTAGE] x (k, v tiles, u[CG], w[CG])
     unsigned char *s_groups = smem + NSTAGE * Cfg::kStageBytes;  // [NC] x kGroupBytes
     __shared__ __align__(8) uint64_t full_bar[NSTAGE];
     __shared__ __align__(8) uint64_t empty_bar[NSTAGE];
     // per group and slot: the compute warps have read the slot's carries
     __shared__ __align__(8) uint64_t free_bar[NC][2];
+    // per group: its gy tile has landed (phase i: the group's i-th tile)
+    __shared__ __align__(8) uint64_t gy_bar[NC];
+    __shared__ int s_gy_loads[NC];     // gy tiles each group has asked for
     __shared__ int s_meta[NSTAGE];     // tile id per stage, -1 = no more tiles
     __shared__ int s_fill_it[NSTAGE];  // ring iteration the stage was last filled for
     __shared__ int s_last_it[NSTAGE];  // last ring iteration loaded into each stage
@@ -232,11 +238,14 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
             s_last_it[s] = -1;
             s_fill_it[s] = -1;
         }
-        for (int q = 0; q < NC; ++q)
+        for (int q = 0; q < NC; ++q) {
             for (int k = 0; k < 2; ++k) {
                 mbar_init(&free_bar[q][k], NWG);
                 s_count[q][k] = 0;
             }
+            mbar_init(&gy_bar[q], 1);
+            s_gy_loads[q] = 0;
+        }
         fence_mbar_init();
         s_abort = 0;
         s_next_it = 0;
@@ -288,8 +297,6 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
                     tma_load_3d(dst, &map_k, &full_bar[s], c0, seg * LT, b);
                     tma_load_3d(dst + Cfg::kTileElems * sizeof(float), &map_v, &full_bar[s], c0,
                                 seg * LT, b);
-                    tma_load_3d(dst + 2 * Cfg::kTileElems * sizeof(float), &map_gy, &full_bar[s],
-                                c0, seg * LT, b);
                     float *dp = reinterpret_cast<float *>(dst + Cfg::kParamOffset);
                     bulk_load(dp, a.u + c0, pbytes, &full_bar[s]);
                     bulk_load(dp + CG, a.w + c0, pbytes, &full_bar[s]);
@@ -406,13 +413,20 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
                 const unsigned char *st_base = s_stage + static_cast<size_t>(s) * Cfg::kStageBytes;
                 const float *s_k = reinterpret_cast<const float *>(st_base);
                 const float *s_v = s_k + Cfg::kTileElems;
-                const float *s_gy = s_v + Cfg::kTileElems;
                 const Param prm = staged_param(
                     reinterpret_cast<const float *>(st_base + Cfg::kParamOffset), lane, c, g.C);
+                // the tile's gy into the group's buffer, landing during pass 1
+                // and the carry: every compute warp of the group is past pass
+                // 2 of the previous tile here (the barrier above), so nothing
+                // reads the buffer any more
+                if (wg == 0 && lane == 0) {
+                    fence_proxy_async_smem();  // those reads before the async-proxy write
+                    s_gy_loads[grp] = i + 1;
+                    mbar_arrive_expect_tx(&gy_bar[grp], static_cast<uint32_t>(Cfg::kGyBytes));
+                    tma_load_3d(g_gy, &map_gy, &gy_bar[grp], c - lane, t0, b);
+                }
 
-                // pass 1: the segment into registers, weights and summary; the
-                // segment's gy rows to the group's tile (this lane's column of
-                // this warp's rows: read back in pass 2 by this lane alone)
+                // pass 1: the segment into registers, weights and summary
                 const int s0 = wg * LS;
                 const int nval = max(0, min(LS, g.T - (t0 + s0)));
                 LaneRows<LS> R;
@@ -425,10 +439,6 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
                         rows_pass1<LS, false>(pk, pv, nval, prm, R, st);
 #pragma unroll
                     for (int q = 0; q < NV; ++q) g_sum[(wg * NV + q) * CG + lane] = Op::get(st, q);
-                    const float *pg = s_gy + s0 * CG + lane;
-                    float *po = g_gy + s0 * CG + lane;
-#pragma unroll 8
-                    for (int ii = 0; ii < LS; ++ii) po[ii * CG] = pg[ii * CG];
                 }
                 // the warp that summarises last folds the group's summaries
                 __syncwarp();
@@ -483,7 +493,10 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
                 if (lane == 0) mbar_arrive(&free_bar[grp][k]);  // the slot may be reused
 
                 // pass 2: the forward state before the segment, y_t and ln D_t,
-                // and the segment's reverse summary, to the scratch
+                // and the segment's reverse summary, to the scratch (gy from
+                // the group's buffer once it has landed)
+                if (!warp_wait_phase(&gy_bar[grp], static_cast<uint32_t>(i & 1), abort_flag, ws))
+                    continue;  // the block is giving up: the next barrier sends the warps home
                 if (nval > 0) {
                     // segment (b, (t0 + s0) / LS) of the scratch
                     const int segi = b * a.S + (t0 + s0) / LS;
@@ -516,12 +529,21 @@ __global__ void __launch_bounds__(BwdStatesCfg<LT, NWG, NC, NSTAGE>::kThreads, 1
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) {
         // an aborted block must not exit with tile loads still landing in its
-        // shared memory: wait (bounded) for the last load of every stage
+        // shared memory: wait (bounded) for the last load of every stage and
+        // every group's last gy tile
         for (int s = 0; s < NSTAGE; ++s) {
             const int it = s_last_it[s];
             if (it < 0) continue;
             const unsigned long long t0 = global_timer_ns();
             while (!mbar_try_wait(&full_bar[s], (it / NSTAGE) & 1)) {
+                if (global_timer_ns() - t0 > kBarrierWaitNs) break;
+            }
+        }
+        for (int q = 0; q < NC; ++q) {
+            const int n = s_gy_loads[q];
+            if (n == 0) continue;
+            const unsigned long long t0 = global_timer_ns();
+            while (!mbar_try_wait(&gy_bar[q], static_cast<uint32_t>((n - 1) & 1))) {
                 if (global_timer_ns() - t0 > kBarrierWaitNs) break;
             }
         }
