@@ -1089,6 +1089,9 @@ wkv_status launch_bwd_tiled(const WkvBwdArgs &a, int64_t B, int64_t T, int64_t C
     if ((st = launch_pdl(kg, std::min(gg.tiles, sms), BwdGrads::kThreads, BwdGrads::kSmemBytes,
                          stream, m[3], m[4], m[5], m[6], m[7], ta, gg, ws)) != WKV_OK)
         return st;
+    // gw, gu: one level while the (row, segment)s are few, else two
+    if (static_cast<int64_t>(a.B) * a.S <= kReduceOneLevelRows)
+        return launch_pdl(wkv_bwd_reduce_one_kernel, n_cg, 32 * kReduceOneWarps, 0, stream, a);
     return launch_pdl(wkv_bwd_reduce_kernel, n_cg * kReduceParts, 32 * kReduceWarps, 0, stream, a);
 }
 

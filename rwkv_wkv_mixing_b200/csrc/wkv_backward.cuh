@@ -479,4 +479,41 @@ __global__ void __launch_bounds__(32 * kReduceWarps) wkv_bwd_reduce_kernel(const
     }
 }
 
+// The same sum in one level, for up to kReduceOneLevelRows (row, segment)s:
+// block cg's warp wi adds rows wi, wi + kReduceOneWarps, ... of the channel
+// group, and its first warp adds the warps' sums in warp order.  One pass
+// over the partials and no cross-block counter.
+constexpr int kReduceOneWarps = 32;
+constexpr int kReduceOneLevelRows = 32 * kReduceOneWarps;
+__global__ void __launch_bounds__(32 * kReduceOneWarps) wkv_bwd_reduce_one_kernel(const WkvBwdArgs a) {
+    __shared__ float part[2][kReduceOneWarps][32];
+    // as in wkv_bwd_rev_carry_kernel
+    allow_dependent_launch();
+    grid_dependency_wait();
+    const int lane = threadIdx.x % 32, wi = threadIdx.x / 32;
+    const int c = blockIdx.x * 32 + lane;
+    const int nbs = a.B * a.S;
+    float gw = 0.f, gu = 0.f;
+    if (c < a.C) {
+#pragma unroll 8
+        for (int bs = wi; bs < nbs; bs += kReduceOneWarps) {
+            gw += a.partial[static_cast<size_t>(bs) * 2 * a.C + c];
+            gu += a.partial[(static_cast<size_t>(bs) * 2 + 1) * a.C + c];
+        }
+    }
+    part[0][wi][lane] = gw;
+    part[1][wi][lane] = gu;
+    __syncthreads();
+    if (wi == 0 && c < a.C) {
+        gw = 0.f;
+        gu = 0.f;
+        for (int i = 0; i < kReduceOneWarps; ++i) {
+            gw += part[0][i][lane];
+            gu += part[1][i][lane];
+        }
+        a.gw[c] = gw;
+        a.gu[c] = gu;
+    }
+}
+
 }  // namespace wkvb
