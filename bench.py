@@ -100,9 +100,9 @@ def read_peaks():
 
 # the sources every kernel is built from (their dispatch included); a
 # recorded DRAM-traffic figure is only reported while these are unchanged
-KERNEL_SOURCES = ("capi.cu", "persistent_scan.cuh", "persistent_wkv.cuh", "persistent_bwd.cuh",
-                  "chunked_scan.cuh", "scan_common.cuh", "wkv_ops.cuh", "lru_ops.cuh",
-                  "wkv_backward.cuh", "serial_wkv.cuh", "token_shift.cuh", "ptx.cuh")
+KERNEL_SOURCES = ("capi.cu", "capi_backward.cuh", "persistent_scan.cuh", "persistent_wkv.cuh",
+                  "persistent_bwd.cuh", "chunked_scan.cuh", "scan_common.cuh", "wkv_ops.cuh",
+                  "lru_ops.cuh", "wkv_backward.cuh", "serial_wkv.cuh", "token_shift.cuh", "ptx.cuh")
 
 
 def _code_only(text):
@@ -129,8 +129,9 @@ def _code_only(text):
     return " ".join("".join(out).split())
 
 
-# The gradient kernels' own headers: no forward kernel is built from them.
-GRAD_ONLY_SOURCES = ("persistent_bwd.cuh", "wkv_backward.cuh")
+# The gradients' own sources (kernels and host side): no forward kernel is
+# built from them.
+GRAD_ONLY_SOURCES = ("capi_backward.cuh", "persistent_bwd.cuh", "wkv_backward.cuh")
 FORWARD_SOURCES = tuple(n for n in KERNEL_SOURCES if n not in GRAD_ONLY_SOURCES)
 
 
