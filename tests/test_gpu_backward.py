@@ -53,10 +53,11 @@ def compare(m, x, gy, what, sums_rel=2e-4):
 # C = 33 and 130 (rows not a multiple of 16 bytes) take the per-segment
 # kernels; the others the tiled ones (128-step tiles, 32-step segments):
 # one segment, one partial tile, several tiles with ragged tails in time
-# and channels, long chains
+# and channels, long chains; B=9 T=3800 has 1071 rows x segments, beyond
+# the one-level gw, gu sum (1024), so its two-level sum runs on the tiled path
 SHAPES = [(1, 1, 4), (2, 5, 32), (2, 64, 40), (3, 300, 33), (1, 1024, 64), (4, 700, 130),
           (1, 4100, 40), (2, 257, 96), (1, 31, 8), (2, 129, 36), (1, 128, 32), (3, 2000, 100),
-          (2, 4129, 64)]
+          (2, 4129, 64), (9, 3800, 64)]
 
 
 @pytest.mark.parametrize("B,T,C", SHAPES)
