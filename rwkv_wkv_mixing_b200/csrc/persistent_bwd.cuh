@@ -22,7 +22,8 @@
 //     are written over the staged k and v and leave by TMA stores, the gw and
 //     gu of the segment go to the scratch.  k, v, gy are read a second time,
 //     gk and gv written once.
-//  4. wkv_bwd_reduce_kernel (wkv_backward.cuh): gw, gu added in a fixed order.
+//  4. wkv_bwd_reduce_one_kernel, or for more than 1024 rows x segments
+//     wkv_bwd_reduce_kernel (wkv_backward.cuh): gw, gu added in a fixed order.
 // HBM traffic per element: 32 bytes of k, v, gy, gk, gv, plus 1.25 bytes of
 // segment states (8 floats written, 8 read, 5 read and written by the
 // reverse scan, 2 partials, per 32 steps).
