@@ -150,6 +150,31 @@ def test_backward_inputs_written_just_before_each_call(m):
     m.wkv_device_status()
 
 
+def test_backward_on_two_streams_concurrently(m):
+    """Two gradient steps in flight at once on two streams: each stream has
+    its own scratch, look-back workspace and sum counters."""
+    xs = [workloads.make_wkv("wkv_169m", B=2, T=1500, C=64, seed=s) for s in (31, 32)]
+    gys = [np.random.default_rng(s).normal(0, 1, x.k.shape).astype(np.float32)
+           for s, x in zip((31, 32), xs)]
+    ins = [(dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(g)) for x, g in zip(xs, gys)]
+    streams = [torch.cuda.Stream() for _ in xs]
+    torch.cuda.synchronize()
+    outs = []
+    for rep in range(3):
+        for st, a in zip(streams, ins):
+            with torch.cuda.stream(st):
+                outs.append((rep, [t for t in m.wkv_backward(*a, stream=st)]))
+    torch.cuda.synchronize()
+    for st in streams:
+        m.wkv_device_status(st)
+    wants = [oracle.wkv_backward_rnn(x.w, x.u, x.k, x.v, g) for x, g in zip(xs, gys)]
+    for i, (rep, out) in enumerate(outs):
+        want = wants[i % 2]
+        for name, got, wv, rel in zip(("gk", "gv", "gw", "gu"), out, want,
+                                      (1e-4, 1e-4, 2e-4, 2e-4)):
+            check(got.double().cpu().numpy(), wv, rel, f"stream {i % 2} call {rep} {name}")
+
+
 def test_backward_every_reverse_frame(m):
     """Keys spread wide enough (N(0, 10)) that some 32-step segments keep the
     forward pass's fixed reference but not the reverse one (a denominator
