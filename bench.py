@@ -100,9 +100,10 @@ def read_peaks():
 
 # the sources every kernel is built from (their dispatch included); a
 # recorded DRAM-traffic figure is only reported while these are unchanged
-KERNEL_SOURCES = ("capi.cu", "capi_backward.cuh", "persistent_scan.cuh", "persistent_wkv.cuh",
-                  "persistent_bwd.cuh", "chunked_scan.cuh", "scan_common.cuh", "wkv_ops.cuh",
-                  "lru_ops.cuh", "wkv_backward.cuh", "serial_wkv.cuh", "token_shift.cuh", "ptx.cuh")
+KERNEL_SOURCES = ("capi.cu", "capi_backward.cuh", "capi_host.cuh", "persistent_scan.cuh",
+                  "persistent_wkv.cuh", "persistent_bwd.cuh", "chunked_scan.cuh", "scan_common.cuh",
+                  "wkv_ops.cuh", "lru_ops.cuh", "wkv_backward.cuh", "serial_wkv.cuh",
+                  "token_shift.cuh", "ptx.cuh")
 
 
 def _code_only(text):
@@ -130,9 +131,12 @@ def _code_only(text):
 
 
 # The gradients' own sources (kernels and host side): no forward kernel is
-# built from them.
+# built from them.  The host-buffer pipeline: no device kernel is.
 GRAD_ONLY_SOURCES = ("capi_backward.cuh", "persistent_bwd.cuh", "wkv_backward.cuh")
-FORWARD_SOURCES = tuple(n for n in KERNEL_SOURCES if n not in GRAD_ONLY_SOURCES)
+HOST_ONLY_SOURCES = ("capi_host.cuh",)
+FORWARD_SOURCES = tuple(n for n in KERNEL_SOURCES
+                        if n not in GRAD_ONLY_SOURCES and n not in HOST_ONLY_SOURCES)
+GRAD_SOURCES = tuple(n for n in KERNEL_SOURCES if n not in HOST_ONLY_SOURCES)
 
 
 def src_hash(read=None, names=KERNEL_SOURCES):

@@ -294,9 +294,10 @@ WKV_API wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C,
  * is host memory; NULL h0 = zeros).  The call copies the inputs to the
  * device, runs the kernel and copies the outputs back, and returns when they
  * are in the output buffer (synchronous; no stream argument).  The work is cut
- * into up to 8 independent chunks -- batch rows, or 64-channel-aligned channel
- * slices when B is 1 -- pipelined over three internal streams so the uploads of
- * one chunk overlap the compute and download of another.  Page-locked host
+ * into up to 8 independent chunks of at least 16 MB of input -- batch rows, or
+ * 64-channel-aligned channel slices when B is 1 -- pipelined over three
+ * internal streams so the uploads of one chunk overlap the compute and
+ * download of another.  Page-locked host
  * memory (cudaHostAlloc / cudaHostRegister) gives full overlap; pageable memory
  * works but its copies are staged by the driver.  The library allocates device
  * staging (three chunks of inputs, outputs and parameters) on first use and

@@ -41,20 +41,27 @@ def test_recorded_traffic_entries_are_consistent():
         assert "--clock-control none" in e["command"], name
         assert len(e["src_sha"]) == 16, name
         assert set(e.get("sources") or bench.KERNEL_SOURCES) <= set(bench.KERNEL_SOURCES), name
-        if name.endswith("_bwd"):   # the gradient kernels are built from every source
-            assert not e.get("sources"), name
+        if name.endswith("_bwd"):   # the gradient kernels: every source but the host pipeline
+            assert tuple(e["sources"]) == bench.GRAD_SOURCES, name
+        else:
+            assert tuple(e["sources"]) == bench.FORWARD_SOURCES, name
 
 
-def test_forward_sources_leave_out_only_the_gradient_headers():
-    assert set(bench.KERNEL_SOURCES) - set(bench.FORWARD_SOURCES) == set(bench.GRAD_ONLY_SOURCES)
-    # no forward source pulls in a gradient header
+def test_forward_sources_leave_out_only_the_gradient_and_host_pipeline_sources():
+    assert set(bench.KERNEL_SOURCES) - set(bench.FORWARD_SOURCES) == \
+        set(bench.GRAD_ONLY_SOURCES) | set(bench.HOST_ONLY_SOURCES)
+    assert set(bench.KERNEL_SOURCES) - set(bench.GRAD_SOURCES) == set(bench.HOST_ONLY_SOURCES)
+    # no device source pulls in a gradient header or the host pipeline
     for name in bench.FORWARD_SOURCES:
-        if name == "capi.cu":   # the library's entry points, gradients included
+        if name == "capi.cu":   # the library's entry points, all of them
             continue
         with open(os.path.join(bench.CSRC, name), encoding="utf-8") as f:
             text = f.read()
-        for g in bench.GRAD_ONLY_SOURCES:
+        for g in bench.GRAD_ONLY_SOURCES + bench.HOST_ONLY_SOURCES:
             assert f'#include "{g}"' not in text, (name, g)
+    # the host pipeline defines no kernel
+    with open(os.path.join(bench.CSRC, "capi_host.cuh"), encoding="utf-8") as f:
+        assert "__global__" not in f.read()
 
 
 def test_recorded_traffic_is_keyed_to_the_entry_sources(tmp_path, monkeypatch):

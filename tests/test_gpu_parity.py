@@ -512,10 +512,12 @@ def test_many_back_to_back_launches(m, op):
 # ---------------------------------------------------------------------------
 # host-buffer entry points (chunked, overlapped copy / compute pipeline)
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("B,T,C,pinned", [(8, 700, 96, True),     # chunks of batch rows
-                                          (1, 1500, 512, True),   # channel slices, 2-D copies
-                                          (3, 300, 40, False),    # pageable memory
-                                          (1, 50, 33, True)])     # one chunk
+# (calls are cut into chunks of at least 16 MB of input, up to 8 of them)
+@pytest.mark.parametrize("B,T,C,pinned", [(8, 2048, 512, True),   # 4 chunks of batch rows
+                                          (1, 16384, 1024, True),  # 8 channel slices, 2-D copies
+                                          (3, 4000, 512, False),  # pageable memory, 3 chunks
+                                          (8, 700, 96, True),     # one chunk
+                                          (1, 50, 33, True)])     # one chunk, any shape
 def test_wkv_host_entry_point(m, B, T, C, pinned):
     x = workloads.make_wkv("wkv_169m", B=B, T=T, C=C, seed=B + T + C)
     h = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory() if pinned \
@@ -534,7 +536,7 @@ def test_wkv_bf16_host_entry_point(m):
     assert_close(y.float().double().numpy(), want, 2e-2 * np.abs(x.v).max(), "bf16 host")
 
 
-@pytest.mark.parametrize("B,T,D", [(16, 600, 64), (1, 700, 256)])
+@pytest.mark.parametrize("B,T,D", [(16, 600, 64), (16, 4096, 256), (1, 16384, 512)])
 def test_scan_host_entry_point(m, B, T, D):
     x = workloads.make_scan("scan_mingru", B=B, T=T, D=D, seed=91, with_h0=True)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()   # noqa: E731
