@@ -107,19 +107,21 @@ __device__ __forceinline__ unsigned long long record_tag(uint4 r) {
 // Count this block as finished; the last of the `blocks` increments a
 // launch makes resets the ticket counter and advances the epoch for the next
 // launch.  Every block has taken its tickets and finished all look-back reads
-// by this point.
+// by this point.  Thread `tid` (0) is the one that took the block's tickets:
+// its count is a release, so those tickets come before it, and the last
+// count acquires every earlier one, so the reset comes after every ticket of
+// the launch.  The next launch sees the reset and the new epoch by the
+// kernel boundary.
 __device__ __forceinline__ void finish_launch(const Workspace &ws, bool chained, int tid,
                                               unsigned blocks) {
     if (!chained) return;
     __syncthreads();
     if (tid == 0) {
-        __threadfence();
-        const unsigned int prev = atomicAdd(ws.done, 1u);
+        const unsigned int prev = atom_add_acq_rel_gpu(ws.done, 1u);
         if (prev == blocks - 1u) {
             atomicExch(ws.ticket, 0u);
             atomicExch(ws.done, 0u);
             atomicAdd(ws.epoch, 1ull);
-            __threadfence();
         }
     }
 }
